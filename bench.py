@@ -1,0 +1,451 @@
+"""Benchmark of the HGA hot path on B200: routed prefill tok/s at 64K context
+(the headline value) and decode µs/step, with roofline, CPU-oracle baseline,
+end-to-end (host-buffer) throughput and SM clocks, printed as one JSON line.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl hga|reference]
+
+For N > 1 launch with torch.distributed.run: every rank runs its own
+independent sequence (weak scaling, no collective on the data path); times
+are the max over ranks and `value` counts the tokens of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_rope_b200 import synth  # noqa: E402
+
+METRIC = "routed attn prefill tok/s & decode µs/step at 64K; % of HBM/TC roofline"
+PREFILL = "prefill_64k"
+DECODES = ("decode_16x32k", "tiered_decode_4x64k")
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return dict(hbm=float(pk["hbm_gbs"]), tc=float(pk["bf16_tflops"]),
+                    tc_sustained=float(pk["bf16_tflops_sustained"]), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, tc=1590.0, tc_sustained=1400.0, src="fallback")
+
+
+# ------------------------------------------------------------ distributed
+class Dist:
+    def __init__(self, n_gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+        else:
+            torch.cuda.set_device(0)
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of this GPU's SM clock and throttle reasons."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- timing
+class Events:
+    def __init__(self, n):
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    def rec(self, i, stream):
+        self.ev[i].record(stream)
+
+    def ms(self, a, b):
+        return self.ev[a].elapsed_time(self.ev[b])
+
+
+def prefill_flops(cfg, n_sel_groups: np.ndarray) -> float:
+    """Algorithmic FLOPs of one prefill attention launch: 4*d per (query row,
+    visible key) pair (QK^T and PV, 2 FLOPs per multiply-add). Visible keys of
+    query token t of chunk j: routed groups*16 + full forced chunks before j
+    + (t - jC + 1) keys of the current chunk (causal)."""
+    C, d, gq = cfg.chunk_size, cfg.head_dim, cfg.n_q_heads // cfg.n_kv_heads
+    total = 0
+    nC = cfg.n_chunks
+    for j in range(nC):
+        s_end = min(cfg.n_sink, j + 1)
+        n_forced = s_end + (j + 1 - max(s_end, j - cfg.n_local))
+        n_tok = min((j + 1) * C, cfg.seq_len) - j * C
+        base = (n_forced - 1) * C
+        per_tok = n_tok * base + n_tok * (n_tok + 1) // 2
+        routed = int(n_sel_groups[..., j].sum()) * 16 * n_tok
+        total += gq * (per_tok * cfg.batch * cfg.n_kv_heads + routed)
+    return 4.0 * d * total
+
+
+def run_prefill(args, dist, peaks):
+    from long_context_rope_b200 import hga, pipeline
+    w = synth.WORKLOADS[args.workload]
+    cfg = hga.config_from(w)
+    seed = synth.seed_for_rank(args.seed, dist.rank)
+    x = synth.draw(w, seed=seed)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    st = torch.cuda.current_stream()
+    k_raw = x["k_raw"].to(dev)
+    v = x["v"].to(dev)
+    q_rot = pipeline.rotate_queries(cfg, x["q_raw"].to(dev))
+    cs, gs = pipeline.alloc_summaries(cfg, dev)
+    k_rot = torch.empty_like(k_raw)
+    rb = pipeline.alloc_route(cfg, dev)
+    out = torch.empty_like(q_rot)
+
+    def step(ev=None, base=0):
+        if ev:
+            ev.rec(base, st)
+        pipeline.summaries(cfg, k_raw, cs, gs, k_rot)
+        if ev:
+            ev.rec(base + 1, st)
+        hga.route_chunks(cfg, q_rot, cs, rb.qbar, rb.sel_chunks, rb.n_sel_chunks)
+        if ev:
+            ev.rec(base + 2, st)
+        hga.route_groups(cfg, rb.qbar, gs, rb.sel_chunks, rb.n_sel_chunks, rb.sel_groups,
+                         rb.n_sel_groups)
+        if ev:
+            ev.rec(base + 3, st)
+        hga.attend(cfg, q_rot, k_rot, v, rb.sel_groups, rb.n_sel_groups, out)
+        if ev:
+            ev.rec(base + 4, st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if hga.get_device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    flops = prefill_flops(cfg, rb.n_sel_groups.cpu().numpy())
+
+    K = args.steps
+    ev = Events(5 * K)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        start.record(st)
+        for i in range(K):
+            step(ev, 5 * i)
+        stop.record(st)
+        torch.cuda.synchronize()
+    dist.barrier()
+    total_ms = start.elapsed_time(stop)
+    stage = {n: [] for n in ("summaries", "route_chunks", "route_groups", "attend")}
+    for i in range(K):
+        for s_i, n in enumerate(stage):
+            stage[n].append(ev.ms(5 * i + s_i, 5 * i + s_i + 1))
+    attend_ms = float(np.mean(stage["attend"]))
+    res = dict(total_ms=dist.max(total_ms), attend_ms=dist.max(attend_ms),
+               stage_ms={n: float(np.mean(vs)) for n, vs in stage.items()},
+               flops=flops, tokens=w.batch * w.q_len, clocks=clk.summary(),
+               launches_per_step=5)
+
+    # end to end through the public API with host buffers (pinned), H2D + D2H inside
+    if not args.no_e2e:
+        hk, hv, hq = (t.cpu().pin_memory() for t in (k_raw, v, q_rot))
+        ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        e_k, e_v, e_q = torch.empty_like(k_raw), torch.empty_like(v), torch.empty_like(q_rot)
+        e_out = torch.empty_like(out)
+
+        def e2e_step():
+            e_k.copy_(hk, non_blocking=True)
+            e_v.copy_(hv, non_blocking=True)
+            e_q.copy_(hq, non_blocking=True)
+            pipeline.prefill(cfg, e_k, e_v, e_q, cs, gs, k_rot, rb, e_out)
+            ho.copy_(e_out, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(1, min(K, 5))
+        dist.barrier()
+        torch.cuda.synchronize()
+        start.record(st)
+        for _ in range(n_e2e):
+            e2e_step()
+        stop.record(st)
+        torch.cuda.synchronize()
+        dist.barrier()
+        e2e_ms = dist.max(start.elapsed_time(stop)) / n_e2e
+        res["e2e"] = dict(ms=e2e_ms, h2d=hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 2,
+                          d2h=ho.numel() * 2)
+    res["cfg"] = cfg
+    return res
+
+
+def run_decode(name, args, dist):
+    from long_context_rope_b200 import hga, pipeline
+    w = synth.WORKLOADS[name]
+    cfg = hga.config_from(w)
+    x = synth.draw(w, seed=synth.seed_for_rank(args.seed, dist.rank))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    st = torch.cuda.current_stream()
+    k_raw = x["k_raw"].to(dev)
+    cs, gs = pipeline.alloc_summaries(cfg, dev)
+    k_rot = torch.empty_like(k_raw)
+    pipeline.summaries(cfg, k_raw, cs, gs, k_rot)
+    del k_raw
+    q_rot = pipeline.rotate_queries(cfg, x["q_raw"].to(dev))
+    rb = pipeline.alloc_route(cfg, dev)
+    out = torch.empty_like(q_rot)
+    gat = pipeline.alloc_gathered(cfg, dev)
+    if w.tiered:
+        k_host = torch.empty(k_rot.shape, dtype=k_rot.dtype, pin_memory=True)
+        k_host.copy_(k_rot)
+        v_host = x["v"].pin_memory()
+        del k_rot
+        W = hga.window_slots(cfg)
+        shape = (w.batch, w.n_kv_heads, W * w.chunk_size, w.head_dim)
+        k_win = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+        v_win = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+        pipeline.fill_windows(cfg, k_host, v_host, k_win, v_win)
+        cfg_w = cfg.copy(kv_layout=hga.HGA_KV_WINDOWS)
+
+        def step():
+            pipeline.decode(cfg_w, q_rot, cs, gs, k_win, v_win, rb, out, gathered=gat,
+                            k_src=k_host, v_src=v_host, src_is_host=True)
+        launches = 5
+        moved = int(0)
+    else:
+        v = x["v"].to(dev)
+
+        def step():
+            pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out)
+        launches = 4
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if hga.get_device_error() != 0:
+        raise RuntimeError(f"device error word set in {name}")
+    n_sel = rb.n_sel_groups.cpu().numpy()
+    moved = int(n_sel.sum()) * 16 * w.head_dim * 2 * 2  # routed K+V bytes
+    K = max(args.steps, 20)
+    ev = Events(2 * K)
+    for i in range(K):
+        flush.fill_(i & 0xff)  # write a buffer larger than L2 between steps
+        ev.rec(2 * i, st)
+        step()
+        ev.rec(2 * i + 1, st)
+    torch.cuda.synchronize()
+    times = [ev.ms(2 * i, 2 * i + 1) * 1000.0 for i in range(K)]
+    us = dist.max(float(np.median(times)))
+    return dict(workload=name, us_per_step=us, us_min=float(np.min(times)), steps=K,
+                launches_per_step=launches, routed_kv_bytes=moved,
+                host_link_gbs=(moved / (us * 1e-6) / 1e9) if w.tiered else None)
+
+
+def cpu_baseline(args, n_chunks_sample=4):
+    """The oracle, as it stands, on a bounded sample of the 64K workload:
+    whole-sequence work (key rotation, summaries) timed once and charged per
+    token; per-query-chunk work (query rotation, q-bar, routing, attention)
+    timed on `n_chunks_sample` query chunks."""
+    from oracle import hga_oracle as O
+    w = synth.WORKLOADS[args.workload]
+    x = synth.draw(w, seed=args.seed)
+    cfg = O.cfg_of(w)
+    k_raw = x["k_raw"].float().numpy()
+    q_raw = x["q_raw"].float().numpy()
+    v = x["v"].float().numpy()
+    t0 = time.perf_counter()
+    k_rot = np.empty_like(k_raw)
+    for h in range(w.n_kv_heads):
+        k_rot[0, h] = O.rope_f32(cfg, k_raw[0, h][:, None, :], 0, True)[:, 0, :]
+    cs, gs = O.build_summaries(cfg, k_raw)
+    t_seq = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    js = sorted(rng.choice(np.arange(1, w.n_chunks), size=n_chunks_sample, replace=False).tolist())
+    t1 = time.perf_counter()
+    for j in js:
+        C = w.chunk_size
+        cj = O.cfg_of(w, q_begin=j * C, q_len=C)
+        q_rot = O.rope_f32(cfg, q_raw[0, j * C:(j + 1) * C], j * C, True)[None]
+        qb = O.qbar(cj, q_rot)
+        sel, nsel, _ = O.route_chunks(cj, qb, cs, False)
+        gsel, gnsel, _ = O.route_groups(cj, qb, gs, sel, nsel, False)
+        O.attend(cj, q_rot, k_rot, v, gsel, gnsel)
+    t_chunks = time.perf_counter() - t1
+    tok = n_chunks_sample * w.chunk_size
+    sec_per_tok = t_seq / w.seq_len + t_chunks / tok
+    return dict(value=1.0 / sec_per_tok, unit="tok/s", cores=O.num_threads(), kind="oracle",
+                sample=(f"{args.workload}: key rotation + summaries of all {w.n_chunks} chunks "
+                        f"({t_seq:.2f} s, charged per token) + rotation, q-bar, routing and "
+                        f"attention of {n_chunks_sample} query chunks {js} ({t_chunks:.2f} s)"),
+                seconds=t_seq + t_chunks)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="hga", choices=["hga", "reference"])
+    ap.add_argument("--workload", default=PREFILL)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    peaks = load_peaks()
+    w = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        vals = []
+        cb = None
+        for i in range(args.warmup + args.steps):
+            cb = cpu_baseline(args, n_chunks_sample=1)
+            if i >= args.warmup:
+                vals.append(cb["value"])
+        v = float(np.median(vals))
+        line = {"metric": METRIC, "value": v, "unit": "tok/s", "impl": "reference",
+                "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": cb["seconds"] * 1000.0,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic",
+                "config": {"workload": args.workload, "seq_len": w.seq_len, "batch": w.batch},
+                "cpu_baseline": {"value": v, "unit": "tok/s", "cores": cb["cores"],
+                                 "kind": "oracle", "sample": cb["sample"]},
+                "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    dist = Dist(args.gpus)
+    try:
+        pre = run_prefill(args, dist, peaks)
+        decodes = []
+        if not args.no_decode:
+            for name in DECODES:
+                decodes.append(run_decode(name, args, dist))
+        n = dist.world
+        value = n * pre["tokens"] / (pre["total_ms"] / args.steps / 1000.0)
+        ach = pre["flops"] / (pre["attend_ms"] * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": n,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": pre["total_ms"] / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded planted-topic generator)",
+            "config": {"workload": args.workload, "batch": w.batch, "seq_len": w.seq_len,
+                       "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim,
+                       "routing": f"C{w.chunk_size} G{w.groups_per_chunk} sink{w.n_sink} "
+                                  f"local{w.n_local} kc{w.top_k_chunks} kg{w.top_k_groups}",
+                       "l2": "inputs larger than L2 (Q 512 MiB, K/V 128 MiB per step)",
+                       "parallelism": f"independent sequence per rank x{n}"},
+            "stage_ms": pre["stage_ms"],
+            "roofline": {"kernel": "hga_attend (prefill)", "bound": "tensor",
+                         "achieved": ach, "peak": peaks["tc_sustained"], "unit": "TFLOP/s",
+                         "frac": ach / peaks["tc_sustained"], "traffic": None,
+                         "flops_per_launch": pre["flops"],
+                         "peak_note": f"bf16 sustained, {peaks['src']}"},
+            "gpu_launches": pre["launches_per_step"] * args.steps,
+            "clocks": pre["clocks"],
+        }
+        if "e2e" in pre:
+            e = pre["e2e"]
+            line["e2e"] = {"value": n * pre["tokens"] / (e["ms"] / 1000.0), "unit": "tok/s",
+                           "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"]}
+        if decodes:
+            line["decode"] = decodes
+        if n == 1 and dist.rank == 0 and not args.no_cpu_baseline:
+            cb = cpu_baseline(args)
+            cb.pop("seconds")
+            line["cpu_baseline"] = cb
+        if dist.rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,191 @@
+/*
+ * hga.h -- C ABI of libhga.so, the B200 (sm_100a) hot path of Hierarchical
+ * Global Attention (HGA).
+ *
+ * The operations follow the statement of the method in "Technische
+ * Samenvatting: Hierarchical Global Attention (HGA)" (gist.science), section
+ * "Methodologie", subsection "Kernmechanisme", items 1-4, and section
+ * "Geheugenarchitectuur" (hot/cold K/V tiers). Where that page is silent the
+ * readings are the same as the CPU oracle's:
+ *   - RoPE uses half-split pairing: pair i = (dim i, dim i + d/2), frequency
+ *     theta_i = rope_theta^(-2i/d), angle = position * theta_i. Pairs
+ *     0..n_high_freq_pairs-1 are the high-frequency pairs.
+ *   - A token set's representative position is the mean of its positions.
+ *   - The routing query of (sequence, KV head, query chunk) is the mean of the
+ *     rotated queries over the chunk's query tokens and the KV head's query
+ *     heads ("q-bar"); scores are plain fp32 dot products.
+ *   - Top-k counts only the non-forced earlier chunks (clamped to what is
+ *     available); the group top-k is global over all groups of the chosen
+ *     chunks. Ties: higher score first, then lower index; NaN ranks last.
+ *     Lists are returned in ascending index order, padded with -1.
+ *   - A query at position p attends to the keys of its set at positions <= p.
+ *
+ * Conventions for every call:
+ *   - All pointers are device pointers unless stated otherwise. The caller owns
+ *     every buffer and keeps it alive until the stream has passed the call.
+ *     Inputs are never modified. The library allocates no memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Work is only enqueued; nothing blocks the host except
+ *     hga_get_device_error.
+ *   - Arguments are validated on the host before anything is launched; a call
+ *     that returns an error has launched nothing. Every data pointer must be
+ *     16-byte aligned.
+ *   - Index lists produced by the library are device-side and never copied to
+ *     the host. Kernels that read a caller-supplied list check every entry;
+ *     an entry out of range, an entry naming a forced chunk, or a list that is
+ *     not strictly ascending sets the device error word (read it with
+ *     hga_get_device_error) and the entry is skipped. No kernel traps.
+ *   - Layouts (row-major, innermost last):
+ *       queries / outputs   [B, q_len, Hq, d]       (token q_begin + t at row t)
+ *       keys / values       [B, Hkv, L, d]          (full store, HGA_KV_FULL)
+ *       chunk summaries     [B, Hkv, nC, d] fp32    nC = ceil(L / C)
+ *       group summaries     [B, Hkv, nC * G, d] fp32
+ *       q-bar               [B, Hkv, nQC, d] fp32   query chunks of the span
+ *       chunk selections    [B, Hkv, nQC, top_k_chunks] int32
+ *       group selections    [B, Hkv, nQC, top_k_groups] int32 (global group
+ *                           index = chunk * G + group within the chunk)
+ *       selection counts    [B, Hkv, nQC] int32
+ *       gathered K / V      [B, Hkv, nQC, top_k_groups * g, d], g = C / G
+ *     nQC counts the chunks touched by the query span [q_begin, q_begin+q_len).
+ */
+#ifndef HGA_H
+#define HGA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HGA_OK = 0,
+    HGA_ERR_NULL = -1,         /* a required pointer is NULL */
+    HGA_ERR_SHAPE = -2,        /* sizes inconsistent or out of the supported range */
+    HGA_ERR_ALIGN = -3,        /* a data pointer is not 16-byte aligned */
+    HGA_ERR_CONFIG = -4,       /* routing or RoPE parameters invalid */
+    HGA_ERR_CUDA = -5,         /* a CUDA call failed (this launch or an earlier async error) */
+    HGA_ERR_DEVICE_INDEX = -6, /* a kernel met an invalid entry in a caller-supplied list */
+    HGA_ERR_TIMEOUT = -7,      /* a bounded device-side wait gave up */
+    HGA_ERR_UNSUPPORTED = -8,  /* valid arguments, combination not implemented */
+    HGA_ERR_MEMORY = -9        /* a pointer is not in the memory space the call needs */
+} hga_status;
+
+typedef enum { HGA_BF16 = 0, HGA_F32 = 1 } hga_dtype;
+
+/* Where hga_attend finds the forced (always visible) chunks.
+ * HGA_KV_FULL:    k_res / v_res are the full store [B, Hkv, L, d].
+ * HGA_KV_WINDOWS: k_res / v_res hold only the forced chunks of the decode
+ *                 query chunk j = (L-1)/C, packed in ascending chunk order:
+ *                 [B, Hkv, W * C, d] with W = n_sink + n_local + 1 slots
+ *                 (the hot tier of "Geheugenarchitectuur"). Decode only. */
+typedef enum { HGA_KV_FULL = 0, HGA_KV_WINDOWS = 1 } hga_kv_layout;
+
+typedef struct {
+    int32_t batch;             /* B */
+    int32_t seq_len;           /* L: tokens in the K/V history (context length) */
+    int32_t n_q_heads;         /* Hq */
+    int32_t n_kv_heads;        /* Hkv; Hq % Hkv == 0 (GQA) */
+    int32_t head_dim;          /* d: 64 or 128 */
+    int32_t chunk_size;        /* C ("Kernmechanisme" item 1: fixed chunks, e.g. C=64) */
+    int32_t groups_per_chunk;  /* G; group size g = C / G must be 16 */
+    int32_t n_sink;            /* initial chunks always visible */
+    int32_t n_local;           /* recent chunks before the current one, always visible */
+    int32_t top_k_chunks;      /* level-1 k (>= 1) */
+    int32_t top_k_groups;      /* level-2 k (>= 1) */
+    int32_t n_high_freq_pairs; /* F: pairs 0..F-1 are rotated per token, then averaged */
+    double rope_theta;         /* RoPE base (> 1) */
+    int32_t dtype;             /* hga_dtype of queries, keys, values and outputs */
+    int32_t q_begin;           /* first query position */
+    int32_t q_len;             /* number of query tokens (1 = decode) */
+    int32_t kv_layout;         /* hga_kv_layout, read by hga_attend only */
+} hga_config;
+
+/* Rotate x by RoPE (standard rotary position embedding; the summaries of
+ * "Kernmechanisme" item 3 are built on it). x, x_rot: [n_outer, n_tokens,
+ * n_heads, d] of cfg->dtype; token t sits at position pos0 + t. x_rot may
+ * equal x (in place). Uses cfg->head_dim, rope_theta and dtype only. Typical
+ * uses: queries [B, q_len, Hq, d] with pos0 = q_begin; keys [B*Hkv, L, 1, d]
+ * with pos0 = 0. */
+hga_status hga_apply_rope(const hga_config* cfg, const void* x, void* x_rot, int64_t n_outer,
+                          int64_t n_tokens, int32_t n_heads, int64_t pos0, void* stream);
+
+/* RoPE-aware chunk and group key summaries ("Kernmechanisme" item 3) of the
+ * chunks [chunk_begin, chunk_end) from the pre-RoPE projected keys k_raw
+ * [B, Hkv, L, d]. For a token set S (a group, or a whole chunk) with mean
+ * position pbar: pairs i < F get mean_{t in S} R(p_t theta_i) k_t,i; pairs
+ * i >= F get R(pbar theta_i) mean_{t in S} k_t,i. Only tokens < L count; an
+ * empty group is zero. Writes chunk_sum [B,Hkv,nC,d] and group_sum
+ * [B,Hkv,nC*G,d] (fp32) rows of those chunks and, if k_rot_out is not NULL,
+ * the rotated keys R(p_t) k_t [B,Hkv,L,d] of their tokens in cfg->dtype (the
+ * attention cache). Building chunk by chunk gives bitwise the same result as
+ * building all chunks at once. */
+hga_status hga_build_summaries(const hga_config* cfg, const void* k_raw, float* chunk_sum,
+                               float* group_sum, void* k_rot_out, int32_t chunk_begin,
+                               int32_t chunk_end, void* stream);
+
+/* Level-1 routing ("Kernmechanisme" item 2, Niveau 1, and Deterministische
+ * Zichtbaarheid). For every (b, KV head, query chunk j of the span): q-bar
+ * from q_rot [B, q_len, Hq, d] (written to qbar_out [B,Hkv,nQC,d] fp32), the
+ * scores q-bar . chunk_sum[c] of the candidates c in [0, j) that are not
+ * forced (forced = sinks c < n_sink, locals j-n_local <= c < j, current j),
+ * and the top-min(top_k_chunks, #candidates) of them. Writes sel_chunks and
+ * n_sel_chunks. scores_out (NULL or [B,Hkv,nQC,nC] fp32) receives every
+ * candidate's score and NaN elsewhere. */
+hga_status hga_route_chunks(const hga_config* cfg, const void* q_rot, const float* chunk_sum,
+                            float* qbar_out, int32_t* sel_chunks, int32_t* n_sel_chunks,
+                            float* scores_out, void* stream);
+
+/* Level-2 routing ("Kernmechanisme" item 2, Niveau 2): inside the chunks
+ * chosen by hga_route_chunks, score all G groups of every chosen chunk
+ * against q-bar (qbar [B,Hkv,nQC,d] from hga_route_chunks) and keep the
+ * top-min(top_k_groups, G * n_sel) globally. Writes sel_groups and
+ * n_sel_groups. scores_out (NULL or [B,Hkv,nQC,top_k_chunks*G] fp32) holds the
+ * score of group gamma of the s-th chosen chunk at s*G + gamma, NaN where
+ * unused. */
+hga_status hga_route_groups(const hga_config* cfg, const float* qbar, const float* group_sum,
+                            const int32_t* sel_chunks, const int32_t* n_sel_chunks,
+                            int32_t* sel_groups, int32_t* n_sel_groups, float* scores_out,
+                            void* stream);
+
+/* Exact-token retrieval ("Kernmechanisme" item 4; "Geheugenarchitectuur"
+ * cold tier): copy the K and V rows of every selected group into compact
+ * buffers k_dst, v_dst [B, Hkv, nQC, top_k_groups * g, d]; slot s holds the
+ * g rows of the s-th selected group. Slots past n_sel_groups are not written.
+ * k_src, v_src are the full store [B, Hkv, L, d]: device memory when
+ * src_is_host == 0, page-locked host memory mapped into the device address
+ * space (cudaHostAlloc / cudaHostRegister) when src_is_host == 1, read over
+ * the host link. HGA_ERR_MEMORY if a host pointer is not mapped. */
+hga_status hga_gather_kv(const hga_config* cfg, const void* k_src, const void* v_src,
+                         int32_t src_is_host, const int32_t* sel_groups,
+                         const int32_t* n_sel_groups, void* k_dst, void* v_dst, void* stream);
+
+/* Exact softmax attention over the bounded set ("Kernmechanisme" item 4):
+ * for each query token at position p in chunk j and each query head, softmax
+ * (scale 1/sqrt(d), fp32 accumulation) over the keys at positions <= p of
+ * the forced chunks of j and of the selected groups, then the weighted sum of
+ * their values. q_rot [B, q_len, Hq, d]; out [B, q_len, Hq, d].
+ * Forced chunks come from k_res / v_res in cfg->kv_layout. Selected groups
+ * come from k_gat / v_gat (the gathered buffers of hga_gather_kv) when those
+ * are not NULL, else from k_res / v_res (HGA_KV_FULL only) by index. */
+hga_status hga_attend(const hga_config* cfg, const void* q_rot, const void* k_res,
+                      const void* v_res, const void* k_gat, const void* v_gat,
+                      const int32_t* sel_groups, const int32_t* n_sel_groups, void* out,
+                      void* stream);
+
+/* Human-readable name of a status. Never NULL. */
+const char* hga_status_string(hga_status status);
+
+/* Synchronise `stream`, then read and clear the device error word of the
+ * current device. Returns HGA_OK, HGA_ERR_DEVICE_INDEX (detail_out, if not
+ * NULL, receives the first offending kernel's code) or HGA_ERR_CUDA. */
+hga_status hga_get_device_error(void* stream, int32_t* detail_out);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int32_t hga_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HGA_H */

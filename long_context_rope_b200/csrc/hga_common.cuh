@@ -1,0 +1,127 @@
+// hga_common.cuh -- shared device helpers of the HGA kernels (sm_100a).
+//
+// The kernel-side view of an hga_config (Params), the forced-chunk rule of
+// "Kernmechanisme" item 2 (Deterministische Zichtbaarheid), RoPE angles, the
+// orderable key used by every top-k, and the device error word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hga.h"
+
+namespace hga {
+
+constexpr int kMaxHalfDim = 64;      // head_dim <= 128
+constexpr int kGroupRows = 16;       // g = C / G: one group = 16 token rows
+constexpr int kMaxForced = 64;       // n_sink + n_local + 1 chunks at most
+
+// Kernel-side copy of the configuration, passed by value.
+struct Params {
+    int B, L, Hq, Hkv, d, C, G, g, gq;
+    int n_sink, n_local, kc, kg, F;
+    int nC, q_begin, q_len, j0, nQC;
+    int dtype, kv_layout;
+    int* err;                      // device error word (first error wins), never NULL
+    double inv_freq[kMaxHalfDim];  // rope_theta^(-2i/d), computed on the host in double
+};
+
+// Error codes written to the device error word (first error wins).
+enum DevError : int {
+    kDevErrNone = 0,
+    kDevErrChunkIndex = 1,   // a chunk selection entry out of range / forced / not ascending
+    kDevErrGroupIndex = 2,   // a group selection entry out of range / forced / not ascending
+    kDevErrCount = 3,        // a selection count above its k
+    kDevErrTimeout = 4,      // a bounded wait gave up
+};
+
+__device__ __forceinline__ void raise_dev_error(const Params& p, int code) {
+    atomicCAS(p.err, 0, code);
+}
+
+// Forced chunks of query chunk j in ascending order without duplicates:
+// sinks [0, min(n_sink, j+1)) then locals [max(end of sinks, j - n_local), j].
+__host__ __device__ __forceinline__ int forced_chunks(const Params& p, int j, int* out) {
+    int n = 0;
+    int s_end = p.n_sink < j + 1 ? p.n_sink : j + 1;
+    for (int c = 0; c < s_end; ++c) out[n++] = c;
+    int l_begin = j - p.n_local > s_end ? j - p.n_local : s_end;
+    for (int c = l_begin; c <= j; ++c) out[n++] = c;
+    return n;
+}
+
+__host__ __device__ __forceinline__ bool is_forced(const Params& p, int j, int c) {
+    return c == j || (c >= 0 && c < p.n_sink && c <= j) || (c < j && c >= j - p.n_local);
+}
+
+// cos / sin of position * inv_freq. The product is formed and reduced to
+// [-pi, pi] in double (Cody-Waite style reduction by 2*pi), then the fp32
+// library sincosf is applied to the reduced angle.
+__device__ __forceinline__ void rope_cs(double pos, double inv_freq, float& c, float& s) {
+    double a = pos * inv_freq;
+    double k = rint(a * 0.15915494309189535);
+    double r = fma(-k, 6.283185307179586, a);
+    sincosf((float)r, &s, &c);
+}
+
+// Total order used by every top-k: a larger key ranks first. Higher score
+// first; -0 equals +0; NaN ranks below every number; ties go to the lower
+// index. Valid keys are > 0 (the low word is ~index with index < 2^31).
+__device__ __forceinline__ unsigned long long rank_key(float score, int index) {
+    uint32_t hi;
+    if (score != score) {
+        hi = 0u;
+    } else {
+        score += 0.0f;  // -0 -> +0
+        uint32_t b = __float_as_uint(score);
+        hi = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    }
+    return ((unsigned long long)hi << 32) | (unsigned long long)(~(uint32_t)index);
+}
+
+__device__ __forceinline__ int rank_key_index(unsigned long long key) {
+    return (int)(~(uint32_t)(key & 0xffffffffull));
+}
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        unsigned long long o = __shfl_xor_sync(0xffffffffu, v, off);
+        v = o > v ? o : v;
+    }
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+    return v;
+}
+
+// 8 bf16 <-> 8 floats through one 16-byte vector.
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 t = __bfloat1622float2(h[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+
+__device__ __forceinline__ uint4 f32x8_to_bf16(const float* f) {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    return u;
+}
+
+}  // namespace hga

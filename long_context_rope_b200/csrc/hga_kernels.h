@@ -1,0 +1,66 @@
+// hga_kernels.h -- internal launchers behind the C ABI (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hga_common.cuh"
+
+namespace hga {
+
+// Largest number of 16-row key blocks one attention unit may hold:
+// G * (n_sink + n_local + 1) forced blocks plus top_k_groups routed ones.
+constexpr int kMaxBlocks = 512;
+// Largest number of chunks the routing kernels keep in shared memory.
+constexpr int kMaxChunks = 16384;
+
+cudaError_t launch_rope(const Params& p, const void* x, void* y, int64_t n_outer,
+                        int64_t n_tokens, int n_heads, int64_t pos0, cudaStream_t st);
+
+cudaError_t launch_summaries(const Params& p, const void* k_raw, float* chunk_sum,
+                             float* group_sum, void* k_rot, int chunk_begin, int chunk_end,
+                             cudaStream_t st);
+
+cudaError_t launch_qbar(const Params& p, const void* q_rot, float* qbar, cudaStream_t st);
+
+cudaError_t launch_route_chunks(const Params& p, const float* qbar, const float* chunk_sum,
+                                int32_t* sel, int32_t* n_sel, float* scores, cudaStream_t st);
+
+cudaError_t launch_route_groups(const Params& p, const float* qbar, const float* group_sum,
+                                const int32_t* sel_chunks, const int32_t* n_sel_chunks,
+                                int32_t* sel_groups, int32_t* n_sel_groups, float* scores,
+                                cudaStream_t st);
+
+cudaError_t launch_gather(const Params& p, const void* k_src, const void* v_src, bool from_host,
+                          const int32_t* sel_groups, const int32_t* n_sel_groups, void* k_dst,
+                          void* v_dst, cudaStream_t st);
+
+// Where an attention unit finds its keys.
+struct KvSources {
+    const void* k_res;  // full store [B,Hkv,L,d] or forced windows [B,Hkv,W*C,d]
+    const void* v_res;
+    const void* k_gat;  // gathered [B,Hkv,nQC,kg*16,d] or nullptr (index mode)
+    const void* v_gat;
+};
+
+cudaError_t launch_attend_simt(const Params& p, const void* q_rot, const KvSources& kv,
+                               const int32_t* sel_groups, const int32_t* n_sel_groups,
+                               void* out, cudaStream_t st);
+
+// True when the tcgen05 prefill kernel covers this configuration (bf16,
+// d = 128, 8 query heads per KV head, prefill, full resident store, index mode).
+bool tc_kernel_supports(const Params& p, bool gathered);
+
+cudaError_t launch_attend_tc(const Params& p, const void* q_rot, const KvSources& kv,
+                             const int32_t* sel_groups, const int32_t* n_sel_groups, void* out,
+                             cudaStream_t st);
+
+// True when the cluster / MMA decode kernel covers this configuration
+// (bf16, d = 128, one query token, gq <= 8, L % 16 == 0, <= 128 key blocks).
+bool decode_kernel_supports(const Params& p);
+
+cudaError_t launch_attend_decode(const Params& p, const void* q_rot, const KvSources& kv,
+                                 const int32_t* sel_groups, const int32_t* n_sel_groups,
+                                 void* out, cudaStream_t st);
+
+}  // namespace hga

@@ -1,0 +1,118 @@
+"""The HGA hot path end to end on one GPU, through the C ABI.
+
+Allocates the device buffers of a configuration (torch supplies the memory)
+and calls the library's entry points in order:
+
+  prefill: hga_build_summaries -> hga_route_chunks -> hga_route_groups
+           -> hga_attend (index mode: the kernel fetches routed groups itself)
+  decode:  hga_route_chunks -> hga_route_groups -> [hga_gather_kv] -> hga_attend
+           (summaries are built once beforehand, as for a KV cache)
+
+Nothing here computes: every step is a kernel of libhga.so.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import torch
+
+from . import hga
+
+
+@dataclasses.dataclass
+class RouteBuffers:
+    qbar: torch.Tensor
+    sel_chunks: torch.Tensor
+    n_sel_chunks: torch.Tensor
+    sel_groups: torch.Tensor
+    n_sel_groups: torch.Tensor
+    chunk_scores: Optional[torch.Tensor] = None
+    group_scores: Optional[torch.Tensor] = None
+
+
+def alloc_summaries(cfg: hga.HgaConfig, device="cuda"):
+    B, H, d, nC, G = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.n_chunks, cfg.groups_per_chunk
+    cs = torch.empty(B, H, nC, d, dtype=torch.float32, device=device)
+    gs = torch.empty(B, H, nC * G, d, dtype=torch.float32, device=device)
+    return cs, gs
+
+
+def alloc_route(cfg: hga.HgaConfig, device="cuda", with_scores: bool = False) -> RouteBuffers:
+    B, H, d, nQC = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.n_qchunks
+    i32 = dict(dtype=torch.int32, device=device)
+    rb = RouteBuffers(
+        qbar=torch.empty(B, H, nQC, d, dtype=torch.float32, device=device),
+        sel_chunks=torch.empty(B, H, nQC, cfg.top_k_chunks, **i32),
+        n_sel_chunks=torch.empty(B, H, nQC, **i32),
+        sel_groups=torch.empty(B, H, nQC, cfg.top_k_groups, **i32),
+        n_sel_groups=torch.empty(B, H, nQC, **i32))
+    if with_scores:
+        rb.chunk_scores = torch.empty(B, H, nQC, cfg.n_chunks, dtype=torch.float32, device=device)
+        rb.group_scores = torch.empty(B, H, nQC, cfg.top_k_chunks * cfg.groups_per_chunk,
+                                      dtype=torch.float32, device=device)
+    return rb
+
+
+def alloc_gathered(cfg: hga.HgaConfig, device="cuda"):
+    shape = (cfg.batch, cfg.n_kv_heads, cfg.n_qchunks, cfg.top_k_groups * cfg.group_size,
+             cfg.head_dim)
+    return (torch.zeros(shape, dtype=cfg.torch_dtype(), device=device),
+            torch.zeros(shape, dtype=cfg.torch_dtype(), device=device))
+
+
+def rotate_queries(cfg: hga.HgaConfig, q_raw: torch.Tensor, stream=None) -> torch.Tensor:
+    q_rot = torch.empty_like(q_raw)
+    hga.apply_rope(cfg, q_raw, q_rot, cfg.batch, cfg.q_len, cfg.n_q_heads, cfg.q_begin, stream)
+    return q_rot
+
+
+def summaries(cfg: hga.HgaConfig, k_raw, cs, gs, k_rot=None, stream=None):
+    hga.build_summaries(cfg, k_raw, cs, gs, k_rot, 0, cfg.n_chunks, stream)
+
+
+def route(cfg: hga.HgaConfig, q_rot, cs, gs, rb: RouteBuffers, stream=None):
+    hga.route_chunks(cfg, q_rot, cs, rb.qbar, rb.sel_chunks, rb.n_sel_chunks, rb.chunk_scores,
+                     stream)
+    hga.route_groups(cfg, rb.qbar, gs, rb.sel_chunks, rb.n_sel_chunks, rb.sel_groups,
+                     rb.n_sel_groups, rb.group_scores, stream)
+
+
+def prefill(cfg: hga.HgaConfig, k_raw, v, q_rot, cs, gs, k_rot, rb: RouteBuffers, out,
+            stream=None):
+    """One pass of the prefill hot path (summaries, routing, attention)."""
+    summaries(cfg, k_raw, cs, gs, k_rot, stream)
+    route(cfg, q_rot, cs, gs, rb, stream)
+    hga.attend(cfg, q_rot, k_rot, v, rb.sel_groups, rb.n_sel_groups, out, stream=stream)
+
+
+def decode(cfg: hga.HgaConfig, q_rot, cs, gs, k_res, v_res, rb: RouteBuffers, out,
+           gathered=None, k_src=None, v_src=None, src_is_host=False, stream=None):
+    """One decode step: routing, optional gather into `gathered` (k, v) from
+    k_src/v_src, attention (forced chunks from k_res/v_res)."""
+    route(cfg, q_rot, cs, gs, rb, stream)
+    if gathered is not None:
+        hga.gather_kv(cfg, k_src, v_src, src_is_host, rb.sel_groups, rb.n_sel_groups,
+                      gathered[0], gathered[1], stream)
+        hga.attend(cfg, q_rot, k_res, v_res, rb.sel_groups, rb.n_sel_groups, out,
+                   k_gat=gathered[0], v_gat=gathered[1], stream=stream)
+    else:
+        hga.attend(cfg, q_rot, k_res, v_res, rb.sel_groups, rb.n_sel_groups, out, stream=stream)
+
+
+def forced_window_chunks(cfg: hga.HgaConfig):
+    """Forced chunks of the decode query chunk, ascending (the slot order of
+    the HGA_KV_WINDOWS buffer)."""
+    j = (cfg.seq_len - 1) // cfg.chunk_size
+    s_end = min(cfg.n_sink, j + 1)
+    return list(range(s_end)) + list(range(max(s_end, j - cfg.n_local), j + 1))
+
+
+def fill_windows(cfg: hga.HgaConfig, k_full, v_full, k_win, v_win):
+    """Copy the forced chunks of the decode query chunk from the full store
+    (host or device) into the resident window buffers (device). Copies only."""
+    C = cfg.chunk_size
+    for w, c in enumerate(forced_window_chunks(cfg)):
+        hi = min((c + 1) * C, cfg.seq_len)
+        k_win[:, :, w * C: w * C + hi - c * C].copy_(k_full[:, :, c * C: hi], non_blocking=True)
+        v_win[:, :, w * C: w * C + hi - c * C].copy_(v_full[:, :, c * C: hi], non_blocking=True)

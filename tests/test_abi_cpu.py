@@ -1,0 +1,74 @@
+"""The C-ABI library loads, exports every symbol include/hga.h declares, and
+rejects invalid arguments on the host (no GPU needed, no compute launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "hga.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:hga_status|const char\*|int32_t)\s+(hga_\w+)\s*\(",
+                                 text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def hga():
+    from long_context_rope_b200 import build
+    build.build()
+    from long_context_rope_b200 import hga as mod
+    return mod
+
+
+def test_exports_every_declared_symbol(hga):
+    names = _declared()
+    assert len(names) >= 9, names
+    for n in names:
+        assert hasattr(hga.library(), n), n
+
+
+def test_struct_layout_matches_header(hga):
+    # 12 int32 (48 bytes), a double at offset 48, 4 int32: 72 bytes, 8-byte aligned
+    assert ctypes.sizeof(hga.HgaConfig) == 72
+    assert hga.HgaConfig.rope_theta.offset == 48
+
+
+def _cfg(hga, **kw):
+    from long_context_rope_b200 import synth
+    return hga.config_from(synth.WORKLOADS["prefill_4k"], **kw)
+
+
+def test_status_strings(hga):
+    for code, name in hga.STATUS.items():
+        assert hga.library().hga_status_string(code).decode().startswith(name)
+
+
+def test_host_validation_without_gpu(hga):
+    L = hga.library()
+    P = 16 * 1024  # any aligned non-null value: nothing is dereferenced on these paths
+    by = ctypes.byref
+    assert L.hga_attend(None, P, P, P, None, None, P, P, P, None) == -1
+    assert L.hga_attend(by(_cfg(hga)), P, P, P, None, None, None, P, P, None) == -1
+    assert L.hga_attend(by(_cfg(hga)), P + 4, P, P, None, None, P, P, P, None) == -3
+    assert L.hga_attend(by(_cfg(hga)), P, P, P, P, None, P, P, P, None) == -1
+    assert L.hga_attend(by(_cfg(hga, head_dim=96)), P, P, P, None, None, P, P, P, None) == -8
+    assert L.hga_attend(by(_cfg(hga, top_k_chunks=0)), P, P, P, None, None, P, P, P, None) == -4
+    assert L.hga_attend(by(_cfg(hga, n_q_heads=30)), P, P, P, None, None, P, P, P, None) == -2
+    assert L.hga_attend(by(_cfg(hga, q_begin=4000, q_len=100)), P, P, P, None, None, P, P, P,
+                        None) == -2
+    assert L.hga_attend(by(_cfg(hga, rope_theta=0.5)), P, P, P, None, None, P, P, P, None) == -4
+    assert L.hga_attend(by(_cfg(hga, chunk_size=48)), P, P, P, None, None, P, P, P, None) == -8
+    assert L.hga_attend(by(_cfg(hga, n_high_freq_pairs=65)), P, P, P, None, None, P, P, P,
+                        None) == -4
+    assert L.hga_attend(by(_cfg(hga, kv_layout=1)), P, P, P, None, None, P, P, P, None) == -8
+    assert L.hga_build_summaries(by(_cfg(hga)), P, P, P, None, 5, 3, None) == -2
+    assert L.hga_build_summaries(by(_cfg(hga)), P, P, P, None, 0, 65, None) == -2
+    assert L.hga_build_summaries(by(_cfg(hga)), P, P, P, None, 3, 3, None) == 0  # empty range
+    assert L.hga_route_chunks(by(_cfg(hga)), P, P, None, P, P, None, None) == -1
+    assert L.hga_route_groups(by(_cfg(hga)), P, P, P, P, P + 8, P, None, None) == -3
+    assert L.hga_gather_kv(by(_cfg(hga)), P, P, 0, P, P, None, P, None) == -1
+    assert L.hga_apply_rope(by(_cfg(hga)), P, P, 1, 4, 0, 0, None) == -2
+    assert L.hga_apply_rope(by(_cfg(hga)), P, P, 0, 4, 1, 0, None) == 0  # nothing to do

@@ -1,0 +1,306 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Every input comes from the seeded generator; each side computes every
+intermediate itself (the oracle never receives a value the GPU produced).
+Stages compared: rotated queries and keys, chunk and group summaries, q-bar,
+routing scores, selections (with the near-tie exemption), and outputs on
+the units whose routing agrees. Tolerances: tests/parity_util.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+from long_context_rope_b200 import synth
+from oracle import hga_oracle as O
+from parity_util import (OUT_TOL, assert_close, check_chunk_selection_matches_own_scores,
+                         check_group_selection_matches_own_scores, compare_selections)
+
+pytestmark = pytest.mark.gpu
+
+
+def _mods():
+    from long_context_rope_b200 import hga, pipeline
+    return hga, pipeline
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy() if t.dtype != torch.int32 else t.cpu().numpy()
+
+
+def bf16_ulp_check(name, got, ref, max_frac=1e-3):
+    """Rounded-to-bf16 values from two computations of the same real number
+    (an fp32 rotation on the GPU, a double one in the oracle): equal, or one
+    bf16 ulp apart, in a small fraction of elements. Near cancellation the
+    fp32 rotation carries an absolute error of a few 1e-7 times the input
+    magnitude (inputs here are O(10) at most), hence the 1e-5 floor."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    diff = got != ref
+    ulp = np.abs(ref) * 2.0 ** -7 + 1e-5
+    assert np.all(np.abs(got - ref)[diff] <= ulp[diff] * 1.0001), f"{name}: beyond one bf16 ulp"
+    assert diff.mean() <= max_frac, f"{name}: {diff.mean():.2e} of elements differ"
+
+
+def _bf16_or_f32(w, a):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    return t.to(w.torch_dtype())
+
+
+def run_gpu_prefill(w, x, r=None):
+    """The GPU prefill path. Rotation and summaries start from the raw drawn
+    inputs. When the oracle's results `r` are given, routing and attention
+    take the oracle's bf16 rotated queries and keys as their inputs (the
+    queries arrive rotated at the routing boundary; sharing them keeps bf16
+    rounding-boundary flips of the two rotations out of the routing decisions);
+    the GPU's own rotations are compared separately."""
+    hga, pipeline = _mods()
+    cfg = hga.config_from(w)
+    k_raw, v, q_raw = (x[n].cuda() for n in ("k_raw", "v", "q_raw"))
+    q_rot = pipeline.rotate_queries(cfg, q_raw)
+    cs, gs = pipeline.alloc_summaries(cfg)
+    k_rot = torch.empty_like(k_raw)
+    rb = pipeline.alloc_route(cfg, with_scores=True)
+    out = torch.full_like(q_rot, float("nan"))
+    pipeline.summaries(cfg, k_raw, cs, gs, k_rot)
+    q_use = _bf16_or_f32(w, r["q_rot"]).cuda() if r is not None else q_rot
+    k_use = _bf16_or_f32(w, r["k_rot"]).cuda() if r is not None else k_rot
+    pipeline.route(cfg, q_use, cs, gs, rb)
+    hga.attend(cfg, q_use, k_use, v, rb.sel_groups, rb.n_sel_groups, out)
+    assert hga.get_device_error() == 0
+    return dict(q_rot=_np(q_rot), k_rot=_np(k_rot), chunk_sum=_np(cs), group_sum=_np(gs),
+                qbar=_np(rb.qbar), sel_chunks=_np(rb.sel_chunks), n_sel_chunks=_np(rb.n_sel_chunks),
+                chunk_scores=_np(rb.chunk_scores), sel_groups=_np(rb.sel_groups),
+                n_sel_groups=_np(rb.n_sel_groups), group_scores=_np(rb.group_scores),
+                out=_np(out))
+
+
+def compare_routing(w, g, r):
+    """Stage-by-stage routing parity. Returns the boolean mask (per problem)
+    of identical group selections."""
+    kc, kg, G = w.top_k_chunks, w.top_k_groups, w.groups_per_chunk
+    # scores of every candidate; NaN marks non-candidates identically
+    assert np.array_equal(np.isnan(g["chunk_scores"]), np.isnan(r["chunk_scores"]))
+    rs = np.nan_to_num(r["chunk_scores"])
+    scale = np.abs(rs).max(axis=-1, keepdims=True) + 1e-6
+    assert_close("chunk scores / scale", np.nan_to_num(g["chunk_scores"]) / scale, rs / scale,
+                 atol=2e-5)
+    rsc = r["chunk_scores"].reshape(-1, r["chunk_scores"].shape[-1])
+    same_c = compare_selections("chunks", g["sel_chunks"], g["n_sel_chunks"], r["sel_chunks"],
+                                r["n_sel_chunks"], lambda p, x: rsc[p, x])
+    check_chunk_selection_matches_own_scores(g["sel_chunks"], g["n_sel_chunks"],
+                                             g["chunk_scores"], kc)
+    check_group_selection_matches_own_scores(g["sel_groups"], g["n_sel_groups"],
+                                             g["group_scores"], g["sel_chunks"],
+                                             g["n_sel_chunks"], G, kg)
+    # groups: where the chunk selections agree, the candidate lists agree
+    rgs = r["group_scores"].reshape(-1, r["group_scores"].shape[-1])
+    ggs = g["group_scores"].reshape(-1, g["group_scores"].shape[-1])
+    rsel_c = r["sel_chunks"].reshape(-1, kc)
+    idx = np.flatnonzero(same_c)
+    assert np.array_equal(np.isnan(ggs[idx]), np.isnan(rgs[idx]))
+    gscale = np.abs(np.nan_to_num(rgs[idx])).max(axis=-1, keepdims=True) + 1e-6
+    assert_close("group scores / scale", np.nan_to_num(ggs[idx]) / gscale,
+                 np.nan_to_num(rgs[idx]) / gscale, atol=2e-5)
+
+    def ref_group_score(p, gi):
+        pos = list(rsel_c[p]).index(gi // G) * G + gi % G
+        return rgs[p, pos]
+
+    gsg = g["sel_groups"].reshape(-1, kg)[idx]
+    gng = g["n_sel_groups"].reshape(-1)[idx]
+    rsg = r["sel_groups"].reshape(-1, kg)[idx]
+    rng_ = r["n_sel_groups"].reshape(-1)[idx]
+    same_g_sub = compare_selections("groups", gsg, gng, rsg, rng_,
+                                    lambda p, x: ref_group_score(idx[p], x))
+    same = np.zeros_like(same_c)
+    same[idx[same_g_sub]] = True
+    assert same.mean() >= 0.99, f"only {same.mean():.3f} of problems route identically"
+    return same
+
+
+def compare_outputs(w, g_out, r_out, same, units=None):
+    """Max-abs parity of the outputs of the units whose routing agrees."""
+    B, H, C, gq = w.batch, w.n_kv_heads, w.chunk_size, w.n_q_heads // w.n_kv_heads
+    j0 = w.q_begin // C
+    nQC = (w.q_begin + w.q_len - 1) // C - j0 + 1
+    if units is None:
+        units = [(b, h, jj) for b in range(B) for h in range(H) for jj in range(nQC)]
+    tol = OUT_TOL[w.dtype]
+    worst = 0.0
+    n_cmp = 0
+    for (b, h, jj) in units:
+        if not same[(b * H + h) * nQC + jj]:
+            continue
+        j = j0 + jj
+        t0 = max(j * C, w.q_begin) - w.q_begin
+        t1 = min((j + 1) * C, w.q_begin + w.q_len) - w.q_begin
+        gg = g_out[b, t0:t1, h * gq:(h + 1) * gq]
+        rr = r_out[b, t0:t1, h * gq:(h + 1) * gq]
+        assert np.isfinite(gg).all()
+        worst = max(worst, float(np.abs(gg - rr).max()))
+        n_cmp += 1
+    assert n_cmp > 0
+    assert worst <= tol, f"max abs error {worst} > {tol}"
+    return worst
+
+
+def compare_prefill(w, x, units=None):
+    r = O.pipeline(w, x, units=units)
+    g = run_gpu_prefill(w, x, r)
+    rot_check = (lambda n, a, b: bf16_ulp_check(n, a, b)) if w.dtype == "bf16" else (
+        lambda n, a, b: assert_close(n, a, b, atol=1e-5, rtol=1e-6))
+    rot_check("q_rot", g["q_rot"], r["q_rot"])
+    rot_check("k_rot", g["k_rot"], r["k_rot"])
+    assert_close("chunk_sum", g["chunk_sum"], r["chunk_sum"], atol=2e-5, rtol=2e-5)
+    assert_close("group_sum", g["group_sum"], r["group_sum"], atol=2e-5, rtol=2e-5)
+    assert_close("qbar", g["qbar"], r["qbar"], atol=2e-5, rtol=2e-5)
+    same = compare_routing(w, g, r)
+    if units is not None:
+        units = [tuple(u) for u in units]
+    return compare_outputs(w, g["out"], r["out"], same, units)
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "prefill_4k"])
+def test_prefill_parity_full(name):
+    w = synth.WORKLOADS[name]
+    x = synth.draw(w, seed=0)
+    worst = compare_prefill(w, x)
+    print(f"{name}: max abs error {worst:.3e}")
+
+
+def test_prefill_end_to_end_from_raw_inputs():
+    """Everything from the raw drawn inputs on both sides (each rotates its own
+    queries and keys). bf16 rounding-boundary flips between the fp32 and the
+    double rotation may move a near-tied routing decision, so this test asks
+    for >= 98% identical routing and checks outputs where routing agrees."""
+    w = synth.WORKLOADS["prefill_4k"]
+    x = synth.draw(w, seed=2)
+    r = O.pipeline(w, x)
+    g = run_gpu_prefill(w, x)
+    same = (g["sel_groups"] == r["sel_groups"]).all(-1) & (g["n_sel_groups"] == r["n_sel_groups"])
+    same &= (g["sel_chunks"] == r["sel_chunks"]).all(-1)
+    assert same.mean() >= 0.98, same.mean()
+    worst = compare_outputs(w, g["out"], r["out"], same.reshape(-1))
+    print(f"end-to-end: {same.mean():.4f} identical routing, max abs error {worst:.3e}")
+
+
+@pytest.mark.parametrize("L,F,dtype", [(1000, 32, "bf16"), (16 * 64 + 16 * 5 + 3, 7, "bf16"),
+                                       (777, 9, "f32")])
+def test_prefill_parity_ragged_small(L, F, dtype):
+    """Ragged context (L % C != 0), several tiles, fewer heads, odd F."""
+    w = synth.WORKLOADS["prefill_4k"].replace(
+        name="ragged", seq_len=L, n_q_heads=8, n_kv_heads=2, n_high_freq_pairs=F, dtype=dtype,
+        top_k_chunks=5, top_k_groups=13, n_local=1, n_sink=2)
+    if dtype == "f32":
+        w = w.replace(head_dim=64)
+    x = synth.draw(w, seed=3)
+    compare_prefill(w, x)
+
+
+def test_prefill_64k_sampled():
+    """The 64K-context workload at full size: every rotation, summary, score
+    and selection, and the outputs of 64 sampled (KV head, query chunk) units."""
+    w = synth.WORKLOADS["prefill_64k"]
+    x = synth.draw(w, seed=0)
+    rng = np.random.default_rng(0)
+    nQC = w.n_chunks
+    units = np.array([[0, int(rng.integers(0, w.n_kv_heads)), int(j)]
+                      for j in sorted(rng.choice(nQC, size=64, replace=False))])
+    units[:4, 2] = [0, 1, nQC - 2, nQC - 1]
+    worst = compare_prefill(w, x, units=units)
+    print(f"prefill_64k sampled: max abs error {worst:.3e}")
+
+
+def _decode_setup(w, x, r):
+    """GPU summaries from the raw keys; the decode query and the attention
+    cache are the oracle's bf16 rotated values (see run_gpu_prefill); the
+    GPU's own rotations are compared against them here."""
+    hga, pipeline = _mods()
+    cfg = hga.config_from(w)
+    k_raw = x["k_raw"].cuda()
+    cs, gs = pipeline.alloc_summaries(cfg)
+    k_rot = torch.empty_like(k_raw)
+    pipeline.summaries(cfg, k_raw, cs, gs, k_rot)
+    del k_raw
+    q_gpu = pipeline.rotate_queries(cfg, x["q_raw"].cuda())
+    bf16_ulp_check("k_rot", _np(k_rot), r["k_rot"])
+    bf16_ulp_check("q_rot", _np(q_gpu), r["q_rot"])
+    k_rot = _bf16_or_f32(w, r["k_rot"]).cuda()
+    q_rot = _bf16_or_f32(w, r["q_rot"]).cuda()
+    return cfg, cs, gs, k_rot, q_rot
+
+
+def _decode_compare(w, r, g_out, rb):
+    g = dict(sel_chunks=_np(rb.sel_chunks), n_sel_chunks=_np(rb.n_sel_chunks),
+             chunk_scores=_np(rb.chunk_scores), sel_groups=_np(rb.sel_groups),
+             n_sel_groups=_np(rb.n_sel_groups), group_scores=_np(rb.group_scores))
+    assert_close("qbar", _np(rb.qbar), r["qbar"], atol=2e-5, rtol=2e-5)
+    same = compare_routing(w, g, r)
+    return compare_outputs(w, _np(g_out), r["out"], same)
+
+
+@pytest.mark.parametrize("mode", ["index", "gathered"])
+def test_decode_16x32k(mode):
+    hga, pipeline = _mods()
+    w = synth.WORKLOADS["decode_16x32k"]
+    x = synth.draw(w, seed=0)
+    r = O.pipeline(w, x)
+    cfg, cs, gs, k_rot, q_rot = _decode_setup(w, x, r)
+    v = x["v"].cuda()
+    rb = pipeline.alloc_route(cfg, with_scores=True)
+    out = torch.full_like(q_rot, float("nan"))
+    if mode == "index":
+        pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out)
+    else:
+        gat = pipeline.alloc_gathered(cfg)
+        pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out, gathered=gat, k_src=k_rot,
+                        v_src=v)
+    assert hga.get_device_error() == 0
+    worst = _decode_compare(w, r, out, rb)
+    print(f"decode {mode}: max abs error {worst:.3e}")
+
+
+def test_tiered_decode_4x64k():
+    """Cold tier in pinned host memory; only the summaries and the forced
+    windows resident in HBM; routed groups gathered over the host link."""
+    hga, pipeline = _mods()
+    w = synth.WORKLOADS["tiered_decode_4x64k"]
+    x = synth.draw(w, seed=0)
+    r = O.pipeline(w, x)
+    cfg, cs, gs, k_rot, q_rot = _decode_setup(w, x, r)
+    k_host = torch.empty(k_rot.shape, dtype=k_rot.dtype, pin_memory=True)
+    k_host.copy_(k_rot)
+    v_host = x["v"].pin_memory()
+    del k_rot
+    cfg_w = cfg.copy(kv_layout=hga.HGA_KV_WINDOWS)
+    W = hga.window_slots(cfg)
+    shape = (w.batch, w.n_kv_heads, W * w.chunk_size, w.head_dim)
+    k_win = torch.zeros(shape, dtype=torch.bfloat16, device="cuda")
+    v_win = torch.zeros(shape, dtype=torch.bfloat16, device="cuda")
+    pipeline.fill_windows(cfg, k_host, v_host, k_win, v_win)
+    rb = pipeline.alloc_route(cfg, with_scores=True)
+    gat = pipeline.alloc_gathered(cfg)
+    out = torch.full_like(q_rot, float("nan"))
+    pipeline.decode(cfg_w, q_rot, cs, gs, k_win, v_win, rb, out, gathered=gat, k_src=k_host,
+                    v_src=v_host, src_is_host=True)
+    assert hga.get_device_error() == 0
+    worst = _decode_compare(w, r, out, rb)
+    print(f"tiered decode: max abs error {worst:.3e}")
+
+
+def test_incremental_summaries_bitwise():
+    """Building the summaries chunk range by chunk range equals one build."""
+    hga, pipeline = _mods()
+    w = synth.WORKLOADS["prefill_4k"]
+    x = synth.draw(w, seed=1)
+    cfg = hga.config_from(w)
+    k_raw = x["k_raw"].cuda()
+    cs1, gs1 = pipeline.alloc_summaries(cfg)
+    kr1 = torch.empty_like(k_raw)
+    hga.build_summaries(cfg, k_raw, cs1, gs1, kr1)
+    cs2, gs2 = pipeline.alloc_summaries(cfg)
+    kr2 = torch.empty_like(k_raw)
+    for c0, c1 in [(0, 1), (1, 7), (7, 40), (40, cfg.n_chunks)]:
+        hga.build_summaries(cfg, k_raw, cs2, gs2, kr2, c0, c1)
+    torch.cuda.synchronize()
+    assert torch.equal(cs1, cs2) and torch.equal(gs1, gs2) and torch.equal(kr1, kr2)
