@@ -288,7 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                 ok = false;
                 break;
             }
-            if (rescale && t >= 1) {
+            // tcgen05.ld/st are warp-collective: the whole warp rescales its
+            // rows when any row needs it (rows that do not use alpha = 1)
+            if (__any_sync(0xffffffffu, rescale && t >= 1)) {
                 ptx::tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {

@@ -1,0 +1,78 @@
+"""Run a few passes of the hot path of one workload, for a profiler to capture.
+
+  python -m long_context_rope_b200.profile_step --workload prefill_64k --steps 2
+  python -m long_context_rope_b200.profile_step --workload decode_16x32k --steps 2
+
+Setup (input draw, query rotation, and for decode the summaries/cache build)
+happens before the steps; each prefill step is summaries -> route_chunks ->
+route_groups -> attend, each decode step route_chunks -> route_groups ->
+[gather] -> attend. Kernel names: summaries_kernel, qbar_kernel,
+route_chunks_kernel, route_groups_kernel, attend_tc_kernel /
+attend_decode_kernel / attend_simt_kernel, gather_*_kernel.
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import sys
+
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from long_context_rope_b200 import hga, pipeline, synth  # noqa: E402
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="prefill_64k")
+    ap.add_argument("--steps", type=int, default=2)
+    ap.add_argument("--gathered", action="store_true", help="decode: gather, then attend")
+    args = ap.parse_args()
+    w = synth.WORKLOADS[args.workload]
+    cfg = hga.config_from(w)
+    x = synth.draw(w, seed=0)
+    k_raw = x["k_raw"].cuda()
+    q_rot = pipeline.rotate_queries(cfg, x["q_raw"].cuda())
+    cs, gs = pipeline.alloc_summaries(cfg)
+    k_rot = torch.empty_like(k_raw)
+    rb = pipeline.alloc_route(cfg)
+    out = torch.empty_like(q_rot)
+    if w.mode == "prefill":
+        v = x["v"].cuda()
+        for _ in range(args.steps):
+            pipeline.prefill(cfg, k_raw, v, q_rot, cs, gs, k_rot, rb, out)
+    else:
+        pipeline.summaries(cfg, k_raw, cs, gs, k_rot)
+        del k_raw
+        if w.tiered:
+            k_host = torch.empty(k_rot.shape, dtype=k_rot.dtype, pin_memory=True)
+            k_host.copy_(k_rot)
+            v_host = x["v"].pin_memory()
+            del k_rot
+            W = hga.window_slots(cfg)
+            shape = (w.batch, w.n_kv_heads, W * w.chunk_size, w.head_dim)
+            k_win = torch.zeros(shape, dtype=torch.bfloat16, device="cuda")
+            v_win = torch.zeros(shape, dtype=torch.bfloat16, device="cuda")
+            pipeline.fill_windows(cfg, k_host, v_host, k_win, v_win)
+            cfg_w = cfg.copy(kv_layout=hga.HGA_KV_WINDOWS)
+            gat = pipeline.alloc_gathered(cfg)
+            for _ in range(args.steps):
+                pipeline.decode(cfg_w, q_rot, cs, gs, k_win, v_win, rb, out, gathered=gat,
+                                k_src=k_host, v_src=v_host, src_is_host=True)
+        else:
+            v = x["v"].cuda()
+            gat = pipeline.alloc_gathered(cfg) if args.gathered else None
+            for _ in range(args.steps):
+                pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out, gathered=gat,
+                                k_src=k_rot, v_src=v)
+    torch.cuda.synchronize()
+    err = hga.get_device_error()
+    print(f"{args.workload}: {args.steps} steps done, device error word {err}")
+    sys.exit(1 if err else 0)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,52 @@
+"""World-size-2 gloo test of the weak-scaling host logic: each rank draws its
+own sequence (different seeds), times are reduced with a max over ranks, and
+the whole-job rate counts every rank's tokens."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from long_context_rope_b200 import dist_util, synth
+        seed = dist_util.rank_seed(0)
+        w = synth.WORKLOADS["tiny_f32"]
+        x = synth.draw(w, seed=seed)
+        first = float(x["k_raw"][0, 0, 0, 0])
+        t = dist_util.max_over_ranks(1.0 + rank)
+        rate = dist_util.whole_job_rate(w.seq_len, t, world)
+        q.put((rank, seed, first, t, rate))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_weak_scaling_host_logic_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, s0, f0, t0, rate0), (r1, s1, f1, t1, rate1) = res
+    assert s0 != s1 and f0 != f1          # independent sequences
+    assert t0 == t1 == 2.0                # max over ranks
+    assert rate0 == rate1 == 2 * 1024 / 2.0
