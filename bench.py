@@ -304,8 +304,29 @@ def run_decode(name, args, dist):
     torch.cuda.synchronize()
     if hga.get_device_error() != 0:
         raise RuntimeError(f"device error word set in {name}")
+    # a decode step is launch-latency bound: capture it once, replay the graph
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+        step()
+    eager_step = step
+
+    def step():
+        graph.replay()
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    if hga.get_device_error() != 0:
+        raise RuntimeError(f"device error word set in {name} (graph)")
     n_sel = rb.n_sel_groups.cpu().numpy()
     moved = int(n_sel.sum()) * 16 * w.head_dim * 2 * 2  # routed K+V bytes
+    # algorithmic HBM bytes of one step (each byte the step must touch, once)
+    n_forced_tok = (min(w.n_sink, w.n_chunks) + w.n_local + 1) * w.chunk_size
+    forced_kv = w.batch * w.n_kv_heads * n_forced_tok * w.head_dim * 2 * 2
+    chunk_sums = w.batch * w.n_kv_heads * w.n_chunks * w.head_dim * 4
+    group_sums = int(rb.n_sel_chunks.cpu().numpy().sum()) * w.groups_per_chunk * w.head_dim * 4
+    q_o = 2 * w.batch * w.n_q_heads * w.head_dim * 2
+    hbm_bytes = forced_kv + chunk_sums + group_sums + q_o + (2 * moved if w.tiered else moved)
     K = max(args.steps, 20)
     ev = Events(2 * K)
     for i in range(K):
@@ -316,9 +337,39 @@ def run_decode(name, args, dist):
     torch.cuda.synchronize()
     times = [ev.ms(2 * i, 2 * i + 1) * 1000.0 for i in range(K)]
     us = dist.max(float(np.median(times)))
+    # the same step launched eagerly (host launch overhead included), for reference
+    ev2 = Events(2 * 5)
+    for i in range(5):
+        flush.fill_(i & 0xff)
+        ev2.rec(2 * i, st)
+        eager_step()
+        ev2.rec(2 * i + 1, st)
+    torch.cuda.synchronize()
+    eager_us = float(np.median([ev2.ms(2 * i, 2 * i + 1) * 1000.0 for i in range(5)]))
+    del graph
     return dict(workload=name, us_per_step=us, us_min=float(np.min(times)), steps=K,
+                hbm_bytes_per_step=hbm_bytes, hbm_gbs=hbm_bytes / (us * 1e-6) / 1e9,
+                hbm_frac=hbm_bytes / (us * 1e-6) / 1e9 / load_peaks()["hbm"],
+                us_per_step_eager=eager_us, cuda_graph=True,
                 launches_per_step=launches, routed_kv_bytes=moved,
                 host_link_gbs=(moved / (us * 1e-6) / 1e9) if w.tiered else None)
+
+
+def host_link_peak_gbs(dev) -> float:
+    """Measured pinned host -> device copy bandwidth (256 MiB, best of 5): the
+    denominator of the host-link (cold tier) gather."""
+    src = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(src.shape, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+    best = 0.0
+    for _ in range(6):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        dst.copy_(src, non_blocking=True)
+        b.record(st)
+        torch.cuda.synchronize()
+        best = max(best, src.numel() / (a.elapsed_time(b) * 1e-3) / 1e9)
+    return best
 
 
 def cpu_baseline(args, n_chunks_sample=4):
@@ -405,8 +456,13 @@ def main():
         pre = run_prefill(args, dist, peaks)
         decodes = []
         if not args.no_decode:
+            link = host_link_peak_gbs(torch.device("cuda", torch.cuda.current_device()))
             for name in DECODES:
-                decodes.append(run_decode(name, args, dist))
+                d = run_decode(name, args, dist)
+                if d.get("host_link_gbs") is not None:
+                    d["host_link_peak_gbs"] = link
+                    d["host_link_frac"] = d["host_link_gbs"] / link
+                decodes.append(d)
         n = dist.world
         value = n * pre["tokens"] / (pre["total_ms"] / args.steps / 1000.0)
         ach = pre["flops"] / (pre["attend_ms"] * 1e-3) / 1e12

@@ -30,40 +30,67 @@ __device__ __forceinline__ int checked_group_entry(const Params& p, int j, const
     return gi;
 }
 
-// Fill blk_row / blk_pos for query chunk j (index jj within the span) and
-// return the number of blocks. Forced chunks come first in ascending order,
-// then the routed groups in list order. Blocks that start at or past L are
-// dropped. Rows of the resident store: the token position (HGA_KV_FULL) or
-// slot * C + 16 * gamma (HGA_KV_WINDOWS). Rows of the gathered buffer:
-// kSrcGathered | 16 * slot. Run by one thread.
-__device__ __forceinline__ int build_key_blocks(const Params& p, int j, const int32_t* list,
-                                                int n_list, bool gathered, int* blk_row,
-                                                int* blk_pos, int cap) {
-    int forced[kMaxForced];
-    const int nf = forced_chunks(p, j, forced);
+// Fill blk_row / blk_pos for query chunk j and return the number of blocks
+// (in every lane). Called by all 32 lanes of one warp. Forced chunks come
+// first in ascending order, then the routed groups in list order; blocks
+// that start at or past L are dropped; invalid list entries are skipped (and
+// recorded in the device error word). Rows of the resident store: the token
+// position (HGA_KV_FULL) or slot * C + 16 * gamma (HGA_KV_WINDOWS). Rows of
+// the gathered buffer: kSrcGathered | 16 * slot. The caller guarantees the
+// output capacity (G * forced chunks + top_k_groups <= kMaxBlocks).
+__device__ __forceinline__ int build_key_blocks_warp(const Params& p, int j, const int32_t* list,
+                                                     int n_list, bool gathered, int* blk_row,
+                                                     int* blk_pos) {
+    const int lane = threadIdx.x & 31;
+    const int s_end = p.n_sink < j + 1 ? p.n_sink : j + 1;
+    const int l_begin = j - p.n_local > s_end ? j - p.n_local : s_end;
+    const int nf = s_end + (j + 1 - l_begin);
     const bool windows = p.kv_layout == HGA_KV_WINDOWS;
     int nb = 0;
-    for (int w = 0; w < nf; ++w) {
-        const int c = forced[w];
-        for (int gm = 0; gm < p.G; ++gm) {
-            const int pos = c * p.C + kGroupRows * gm;
-            if (pos >= p.L || nb >= cap) continue;
-            blk_row[nb] = windows ? w * p.C + kGroupRows * gm : pos;
-            blk_pos[nb] = pos;
-            ++nb;
+    for (int i0 = 0; i0 < nf * p.G; i0 += 32) {
+        const int i = i0 + lane;
+        int pos = 0, row = 0;
+        bool ok = false;
+        if (i < nf * p.G) {
+            const int w = i / p.G, gm = i % p.G;
+            const int c = w < s_end ? w : l_begin + (w - s_end);
+            pos = c * p.C + kGroupRows * gm;
+            row = windows ? w * p.C + kGroupRows * gm : pos;
+            ok = pos < p.L;
         }
+        const unsigned m = __ballot_sync(0xffffffffu, ok);
+        if (ok) {
+            const int at = nb + __popc(m & ((1u << lane) - 1u));
+            blk_row[at] = row;
+            blk_pos[at] = pos;
+        }
+        nb += __popc(m);
     }
     if (n_list < 0 || n_list > p.kg) {
-        raise_dev_error(p, kDevErrCount);
+        if (lane == 0) raise_dev_error(p, kDevErrCount);
         n_list = n_list < 0 ? 0 : p.kg;
     }
-    for (int s = 0; s < n_list; ++s) {
-        const int gi = checked_group_entry(p, j, list, s);
-        if (gi < 0 || nb >= cap) continue;
-        const int pos = gi * kGroupRows;
-        blk_row[nb] = gathered ? (kSrcGathered | (kGroupRows * s)) : pos;
-        blk_pos[nb] = pos;
-        ++nb;
+    for (int s0 = 0; s0 < n_list; s0 += 32) {
+        const int s = s0 + lane;
+        int gi = -1;
+        if (s < n_list) {
+            gi = list[s];
+            const int prev = s > 0 ? list[s - 1] : -1;
+            const int c = gi >= 0 ? gi / p.G : -1;
+            const bool ok = gi >= 0 && c < j && !is_forced(p, j, c) && (s == 0 || gi > prev);
+            if (!ok) {
+                raise_dev_error(p, kDevErrGroupIndex);
+                gi = -1;
+            }
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, gi >= 0);
+        if (gi >= 0) {
+            const int at = nb + __popc(m & ((1u << lane) - 1u));
+            const int pos = gi * kGroupRows;
+            blk_row[at] = gathered ? (kSrcGathered | (kGroupRows * s)) : pos;
+            blk_pos[at] = pos;
+        }
+        nb += __popc(m);
     }
     return nb;
 }

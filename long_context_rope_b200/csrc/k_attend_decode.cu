@@ -29,6 +29,7 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kMaxLoc = 8;                 // key blocks per CTA
+constexpr int kMaxCluster = 16;            // CTAs per (sequence, KV head)
 constexpr int kBlkBytes = kGroupRows * kD * 2;  // 4 KiB per block per tensor
 constexpr int kSP = kMaxLoc * 16 + 4;      // fp32 score row pitch
 constexpr int kPP = kMaxLoc * 16 + 8;      // bf16 probability row pitch (conflict-free)
@@ -71,9 +72,12 @@ __global__ void __launch_bounds__(256) attend_decode_kernel(const __grid_constan
     const int g = lane >> 2, t4 = lane & 3;
     const int qpos = p.q_begin;
 
+    if (warp == 0) {
+        const int nb_w = build_key_blocks_warp(p, j, sel + prob * p.kg, nsel[prob], gathered != 0,
+                                               sm.blk_row, sm.blk_pos);
+        if (lane == 0) sm.nb = nb_w;
+    }
     if (tid == 0) {
-        sm.nb = build_key_blocks(p, j, sel + prob * p.kg, nsel[prob], gathered != 0, sm.blk_row,
-                                 sm.blk_pos, kMaxBlocks);
         sm.bad = 0;
         ptx::mbar_init(&sm.bar_k, 1);
         ptx::mbar_init(&sm.bar_v, 1);
@@ -205,20 +209,32 @@ __global__ void __launch_bounds__(256) attend_decode_kernel(const __grid_constan
     // ---- merge the CL partials of head n in CTA n % CL
     for (int n = r; n < p.gq; n += CL) {
         if (tid < kD) {
-            float M = -INFINITY;
-            for (int c = 0; c < CL; ++c) {
-                const DecodeSmem* rs = cluster.map_shared_rank(&sm, c);
-                M = fmaxf(M, rs->m[n]);
+            // issue every remote (distributed shared memory) load first, then combine
+            float mc[kMaxCluster], lc[kMaxCluster], oc[kMaxCluster];
+#pragma unroll
+            for (int c = 0; c < kMaxCluster; ++c) {
+                if (c < CL) {
+                    const DecodeSmem* rs = cluster.map_shared_rank(&sm, c);
+                    mc[c] = rs->m[n];
+                    lc[c] = rs->l[n];
+                    oc[c] = rs->opart[n][tid];
+                } else {
+                    mc[c] = -INFINITY;
+                    lc[c] = 0.f;
+                    oc[c] = 0.f;
+                }
             }
+            float M = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kMaxCluster; ++c) M = fmaxf(M, mc[c]);
             float num = 0.f, den = 0.f;
             if (M != -INFINITY) {
-                for (int c = 0; c < CL; ++c) {
-                    const DecodeSmem* rs = cluster.map_shared_rank(&sm, c);
-                    const float mc = rs->m[n];
-                    if (mc == -INFINITY) continue;
-                    const float wgt = exp2f(mc - M);
-                    num = fmaf(wgt, rs->opart[n][tid], num);
-                    den = fmaf(wgt, rs->l[n], den);
+#pragma unroll
+                for (int c = 0; c < kMaxCluster; ++c) {
+                    if (mc[c] == -INFINITY) continue;
+                    const float wgt = exp2f(mc[c] - M);
+                    num = fmaf(wgt, oc[c], num);
+                    den = fmaf(wgt, lc[c], den);
                 }
             }
             const float o = den > 0.f ? num / den : 0.f;
@@ -299,7 +315,7 @@ cudaError_t launch_attend_decode(const Params& p, const void* q_rot, const KvSou
 bool decode_kernel_supports(const Params& p) {
     const int nb_max = p.G * (p.n_sink + p.n_local + 1) + p.kg;
     return p.dtype == HGA_BF16 && p.d == kD && p.q_len == 1 && p.gq <= 8 &&
-           p.L % kGroupRows == 0 && nb_max <= 16 * kMaxLoc;
+           p.L % kGroupRows == 0 && nb_max <= kMaxCluster * kMaxLoc;
 }
 
 }  // namespace hga

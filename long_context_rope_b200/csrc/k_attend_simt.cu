@@ -67,10 +67,11 @@ __global__ void __launch_bounds__(128) attend_simt_kernel(Params p, const T* __r
     const int row0 = rb * kRowsPerCta;
     if (row0 >= n_rows) return;
 
-    if (tid == 0) {
+    if (warp == 0) {
         const int32_t* list = sel ? sel + prob * p.kg : nullptr;
         const int n_list = sel ? nsel[prob] : 0;
-        s_nb = build_key_blocks(p, j, list, n_list, gathered, blk_row, blk_pos, kMaxBlocks);
+        const int nb_w = build_key_blocks_warp(p, j, list, n_list, gathered, blk_row, blk_pos);
+        if (lane == 0) s_nb = nb_w;
     }
     for (int x = tid; x < kRowsPerCta * D; x += blockDim.x) {
         const int rr = x / D, e = x % D;

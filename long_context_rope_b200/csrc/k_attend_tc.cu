@@ -7,20 +7,25 @@
 // heads per KV head, one (sequence, KV head, query chunk) unit is a real
 // dense contraction: 512 query rows against up to ~1.8K keys.
 //
-// CTA = 128 query rows (16 tokens x 8 heads) of one unit; 6 warps:
-//   warp 0      TMA producer: the Q tile once, then K and V tiles of 128 keys
-//               assembled from 16-row group blocks (2 stages each);
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of two TMEM
-//               S buffers, O += P V into the TMEM O accumulator;
-//   warps 2..5  softmax: each thread owns one query row (its TMEM lane),
-//               loads its S row, applies the causal / padding mask, keeps an
-//               online max with lazy rescaling of O (only when the max grows
-//               by more than 2^8), writes P (bf16) to shared memory for the
-//               PV MMA, and finally normalises O and stores the output.
-// The key set arrives in arbitrary group order (forced chunks, then routed
-// groups), so each 128-key tile is 8 independent TMA boxes of 16 rows.
-// Every wait is bounded; on a timeout the CTA records a device error,
-// stops its roles, drains its MMAs, frees TMEM and exits.
+// CTA = two M tiles (A, B) of 128 query rows each (16 tokens x 8 heads),
+// sharing every K/V tile; 10 warps:
+//   warp 0      TMA producer: both Q tiles once, then K and V tiles of 128 keys
+//               assembled from 16-row group boxes (two stages each);
+//   warp 1      TMEM owner and MMA issuer. Issue order per key tile t:
+//               PV_A(t), QK_A(t+1), PV_B(t), QK_B(t+1), so the tensor core
+//               works on one M tile while the other's softmax runs;
+//   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B: each thread
+//               owns one query row (its TMEM lane); it loads its S row,
+//               masks (causal / padding), keeps a lazily rescaled running max
+//               (O is rescaled in TMEM only when the max grows by > 2^8),
+//               writes P = 2^(S - max) as bf16 back into TMEM over its S row,
+//               and at the end normalises O and stores the output.
+// TMEM: S_A | S_B | O_A | O_B (128 columns each); P_X lives in the first 64
+// columns of S_X and feeds the PV MMA directly from TMEM. The key set comes
+// in arbitrary group order (forced chunks, then routed groups), so each
+// 128-key tile is 8 independent TMA boxes of 16 rows x 64 columns (x2).
+// Every wait is bounded; on a timeout the CTA records a device error, stops
+// its roles, drains its MMAs, frees TMEM and exits.
 #include "hga_blocks.cuh"
 #include "hga_kernels.h"
 #include "hga_ptx.cuh"
@@ -31,27 +36,28 @@ namespace hga {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kRows = 128;                 // query rows per CTA (M)
-constexpr int kTileKeys = 128;             // keys per tile (N of S, K of PV)
+constexpr int kRows = 128;                 // query rows per M tile
+constexpr int kTileKeys = 128;             // keys per tile
 constexpr int kBlocksPerTile = kTileKeys / kGroupRows;
 constexpr int kPanel = 128 * 128;          // 128 rows x 128 bytes (64 bf16)
 constexpr int kTile = 2 * kPanel;          // 128 x 128 bf16
-constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 512;        // S0 | S1 | O | unused
-constexpr uint32_t kColO = 256;
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
+
+__host__ __device__ constexpr uint32_t col_s(int x) { return (uint32_t)(x * 128); }
+__host__ __device__ constexpr uint32_t col_o(int x) { return (uint32_t)(256 + x * 128); }
 
 struct TcMaps {
     CUtensorMap q, k, v;
 };
 
 struct TcSmem {
-    alignas(1024) uint8_t q[kTile];
+    alignas(1024) uint8_t q[2][kTile];
     alignas(1024) uint8_t k[2][kTile];
     alignas(1024) uint8_t v[2][kTile];
-    alignas(1024) uint8_t p[kTile];
-    uint64_t bar_q, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], s_empty[2];
-    uint64_t p_full, pv_done, drain;
+    uint64_t bar_q, k_full[2], k_empty[2], v_full[2], v_empty[2];
+    uint64_t s_full[2], p_full[2], o_done[2], drain;
     uint32_t tmem_base;
     int nb;
     int abort;
@@ -60,9 +66,8 @@ struct TcSmem {
 };
 
 // Bounded wait shared by the roles of one CTA: gives up after the time limit,
-// when another role of this CTA gave up (*abort), or when any CTA of the
-// grid recorded an error (*err); a give-up sets *abort so the other roles
-// stop too.
+// when another role of this CTA gave up (*abort), or when any CTA of the grid
+// recorded an error (*err); a give-up sets *abort so the other roles stop.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort,
                                          const int* err) {
     const uint64_t t0 = ptx::globaltimer_ns();
@@ -78,6 +83,27 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
     return false;
 }
 
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_s, uint32_t k_s) {
+    constexpr uint32_t id_qk = ptx::idesc_bf16_f32(kRows, kTileKeys, 0, 0);
+#pragma unroll
+    for (int kk = 0; kk < kD / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+        ptx::umma_f16(d_tmem, ptx::smem_desc_sw128(q_s + off, 16, 1024),
+                      ptx::smem_desc_sw128(k_s + off, 16, 1024), id_qk, kk > 0);
+    }
+}
+
+// O (+)= P V with P (bf16) in TMEM columns [p_tmem, p_tmem + 64).
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_s,
+                                         bool accumulate) {
+    constexpr uint32_t id_pv = ptx::idesc_bf16_f32(kRows, kD, 0, 1);
+#pragma unroll
+    for (int kk = 0; kk < kTileKeys / 16; ++kk)
+        ptx::umma_f16_ts(d_tmem, p_tmem + kk * 8,
+                         ptx::smem_desc_sw128(v_s + kk * 2048, kPanel, 1024), id_pv,
+                         (accumulate || kk > 0) ? 1u : 0u);
+}
+
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_constant__ TcMaps maps,
                                                                Params p,
                                                                const int32_t* __restrict__ sel,
@@ -86,35 +112,36 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     extern __shared__ uint8_t smem_raw[];
     TcSmem& sm = *reinterpret_cast<TcSmem*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int mt = blockIdx.x, jj = blockIdx.y;
+    const int pair = blockIdx.x, jj = blockIdx.y;
     const int64_t bh = blockIdx.z;
     const int b = (int)(bh / p.Hkv), h = (int)(bh % p.Hkv);
     const int j = p.j0 + jj;
     const int64_t prob = bh * p.nQC + jj;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int span_end = p.q_begin + p.q_len;
-    const int tok0 = j * p.C + mt * 16;  // first token position of this M tile
-    if (tok0 >= span_end || tok0 + 16 <= p.q_begin) return;
+    const int tok0 = j * p.C + pair * 32;  // first token position of M tile A
+    if (tok0 >= span_end || tok0 + 32 <= p.q_begin) return;
 
-    if (tid == 0) {
-        sm.nb = build_key_blocks(p, j, sel + prob * p.kg, nsel[prob], false, sm.blk_row,
-                                 sm.blk_pos, kMaxBlocks);
-        sm.abort = 0;
-        ptx::mbar_init(&sm.bar_q, 1);
-        for (int s = 0; s < 2; ++s) {
-            ptx::mbar_init(&sm.k_full[s], 1);
-            ptx::mbar_init(&sm.k_empty[s], 1);
-            ptx::mbar_init(&sm.v_full[s], 1);
-            ptx::mbar_init(&sm.v_empty[s], 1);
-            ptx::mbar_init(&sm.s_full[s], 1);
-            ptx::mbar_init(&sm.s_empty[s], 4);
+    if (warp == 0) {
+        const int nb_w = build_key_blocks_warp(p, j, sel + prob * p.kg, nsel[prob], false,
+                                               sm.blk_row, sm.blk_pos);
+        if (lane == 0) {
+            sm.nb = nb_w;
+            sm.abort = 0;
+            ptx::mbar_init(&sm.bar_q, 1);
+            for (int s = 0; s < 2; ++s) {
+                ptx::mbar_init(&sm.k_full[s], 1);
+                ptx::mbar_init(&sm.k_empty[s], 1);
+                ptx::mbar_init(&sm.v_full[s], 1);
+                ptx::mbar_init(&sm.v_empty[s], 1);
+                ptx::mbar_init(&sm.s_full[s], 1);
+                ptx::mbar_init(&sm.p_full[s], 4);
+                ptx::mbar_init(&sm.o_done[s], 1);
+            }
+            ptx::mbar_init(&sm.drain, 1);
+            ptx::fence_mbar_init();
         }
-        ptx::mbar_init(&sm.p_full, 4);
-        ptx::mbar_init(&sm.pv_done, 1);
-        ptx::mbar_init(&sm.drain, 1);
-        ptx::fence_mbar_init();
-    }
-    if (warp == 1) {
+    } else if (warp == 1) {
         ptx::tmem_alloc(&sm.tmem_base, kTmemCols);
         ptx::tmem_relinquish();
     }
@@ -130,9 +157,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         // ------------------------------------------------------ producer
         if (lane == 0 && n_tiles > 0) {
             const int tq = tok0 - p.q_begin;
-            ptx::mbar_arrive_expect_tx(&sm.bar_q, kTile);
-            ptx::tma_load_4d(sm.q, &maps.q, 0, h * 8, tq, b, &sm.bar_q);
-            ptx::tma_load_4d(sm.q + kPanel, &maps.q, 64, h * 8, tq, b, &sm.bar_q);
+            ptx::mbar_arrive_expect_tx(&sm.bar_q, 2 * kTile);
+            for (int x = 0; x < 2; ++x) {
+                ptx::tma_load_4d(sm.q[x], &maps.q, 0, h * 8, tq + 16 * x, b, &sm.bar_q);
+                ptx::tma_load_4d(sm.q[x] + kPanel, &maps.q, 64, h * 8, tq + 16 * x, b, &sm.bar_q);
+            }
             for (int t = 0; t < n_tiles; ++t) {
                 const int s = t & 1;
                 if (t >= 2 && !wait_bar(&sm.k_empty[s], ((t >> 1) - 1) & 1, abort, p.err)) break;
@@ -158,43 +187,41 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0 && n_tiles > 0) {
-            constexpr uint32_t id_qk = ptx::idesc_bf16_f32(kRows, kTileKeys, 0, 0);
-            constexpr uint32_t id_pv = ptx::idesc_bf16_f32(kRows, kD, 0, 1);
-            const uint32_t q_s = ptx::smem_u32(sm.q);
-            const uint32_t p_s = ptx::smem_u32(sm.p);
-            bool ok = wait_bar(&sm.bar_q, 0, abort, p.err);
-            for (int t = 0; ok && t <= n_tiles; ++t) {
-                if (t < n_tiles) {
-                    const int s = t & 1;
-                    if (!wait_bar(&sm.k_full[s], (t >> 1) & 1, abort, p.err)) break;
-                    if (t >= 2 && !wait_bar(&sm.s_empty[s], ((t >> 1) - 1) & 1, abort, p.err)) break;
-                    ptx::tc_fence_after();
-                    const uint32_t k_s = ptx::smem_u32(sm.k[s]);
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-                        ptx::umma_f16(tmem + s * kTileKeys, ptx::smem_desc_sw128(q_s + off, 16, 1024),
-                                      ptx::smem_desc_sw128(k_s + off, 16, 1024), id_qk, kk > 0);
+            const uint32_t q_s[2] = {ptx::smem_u32(sm.q[0]), ptx::smem_u32(sm.q[1])};
+            bool ok = wait_bar(&sm.bar_q, 0, abort, p.err) && wait_bar(&sm.k_full[0], 0, abort, p.err);
+            if (ok) {
+                ptx::tc_fence_after();
+                const uint32_t k0 = ptx::smem_u32(sm.k[0]);
+                issue_qk(tmem + col_s(0), q_s[0], k0);
+                ptx::umma_commit(&sm.s_full[0]);
+                issue_qk(tmem + col_s(1), q_s[1], k0);
+                ptx::umma_commit(&sm.s_full[1]);
+                ptx::umma_commit(&sm.k_empty[0]);
+            }
+            for (int t = 0; ok && t < n_tiles; ++t) {
+                const int s = t & 1, s1 = (t + 1) & 1;
+                const bool more = t + 1 < n_tiles;
+                if (!wait_bar(&sm.v_full[s], (t >> 1) & 1, abort, p.err)) break;
+                if (more && !wait_bar(&sm.k_full[s1], ((t + 1) >> 1) & 1, abort, p.err)) break;
+                const uint32_t v_s = ptx::smem_u32(sm.v[s]);
+                const uint32_t k_s1 = ptx::smem_u32(sm.k[s1]);
+                for (int x = 0; x < 2; ++x) {
+                    if (!wait_bar(&sm.p_full[x], t & 1, abort, p.err)) {
+                        ok = false;
+                        break;
                     }
-                    ptx::umma_commit(&sm.s_full[s]);
-                    ptx::umma_commit(&sm.k_empty[s]);
-                }
-                if (t >= 1) {
-                    const int u = t - 1, s = u & 1;
-                    if (!wait_bar(&sm.p_full, u & 1, abort, p.err)) break;
-                    if (!wait_bar(&sm.v_full[s], (u >> 1) & 1, abort, p.err)) break;
                     ptx::tc_fence_after();
-                    const uint32_t v_s = ptx::smem_u32(sm.v[s]);
-#pragma unroll
-                    for (int kk = 0; kk < kTileKeys / 16; ++kk) {
-                        const uint32_t aoff = (kk >> 2) * kPanel + (kk & 3) * 32;
-                        ptx::umma_f16(tmem + kColO, ptx::smem_desc_sw128(p_s + aoff, 16, 1024),
-                                      ptx::smem_desc_sw128(v_s + kk * 2048, kPanel, 1024), id_pv,
-                                      (u > 0 || kk > 0) ? 1u : 0u);
+                    issue_pv(tmem + col_o(x), tmem + col_s(x), v_s, t > 0);
+                    if (more) {
+                        issue_qk(tmem + col_s(x), q_s[x], k_s1);
+                        ptx::umma_commit(&sm.s_full[x]);
+                    } else {
+                        ptx::umma_commit(&sm.o_done[x]);
                     }
-                    ptx::umma_commit(&sm.pv_done);
-                    ptx::umma_commit(&sm.v_empty[s]);
                 }
+                if (!ok) break;
+                ptx::umma_commit(&sm.v_empty[s]);
+                if (more) ptx::umma_commit(&sm.k_empty[s1]);
             }
             // drain: every MMA issued above has completed before TMEM is freed
             ptx::umma_commit(&sm.drain);
@@ -205,42 +232,39 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         }
     } else {
         // ------------------------------------------------------ softmax
-        const int q4 = warp & 3;
+        const int x = (warp - 2) >> 2;                  // M tile of this warpgroup
+        const int q4 = warp & 3;                        // TMEM lane quarter
         const int r = q4 * 32 + lane;                   // row = TMEM lane
         const int head = r & 7;
-        const int qpos = tok0 + (r >> 3);
+        const int tokx = tok0 + 16 * x;
+        const int qpos = tokx + (r >> 3);
         const bool row_ok = qpos >= p.q_begin && qpos < span_end;
-        const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        const uint32_t s_addr = tmem + lane_off + col_s(x);
+        const uint32_t o_addr = tmem + lane_off + col_o(x);
         const float sc = 1.4426950408889634f / sqrtf((float)kD);
         float m_used = -INFINITY, l = 0.f;
         bool ok = n_tiles > 0;
-        uint8_t* prow = sm.p + r * 128;
         for (int t = 0; ok && t < n_tiles; ++t) {
-            const int s = t & 1;
-            if (!__all_sync(0xffffffffu, wait_bar(&sm.s_full[s], (t >> 1) & 1, abort, p.err))) {
+            if (!__all_sync(0xffffffffu, wait_bar(&sm.s_full[x], t & 1, abort, p.err))) {
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
-            float x[kTileKeys];
+            float sx[kTileKeys];
             {
-                uint32_t* xr = reinterpret_cast<uint32_t*>(x);
+                uint32_t* xr = reinterpret_cast<uint32_t*>(sx);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) ptx::tmem_ld32(lane_addr + s * kTileKeys + 32 * c, xr + 32 * c);
+                for (int c = 0; c < 4; ++c) ptx::tmem_ld32(s_addr + 32 * c, xr + 32 * c);
                 ptx::tmem_wait_ld();
             }
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&sm.s_empty[s]);
             // mask (causal within the current chunk; padding past the set)
             const int blk0 = t * kBlocksPerTile;
             bool need_mask = blk0 + kBlocksPerTile > nb;
-            if (!need_mask) {
 #pragma unroll
-                for (int i = 0; i < kBlocksPerTile; ++i)
-                    need_mask |= sm.blk_pos[blk0 + i] + kGroupRows - 1 > tok0;
-            }
-            float mt_ = -INFINITY;
+            for (int i = 0; i < kBlocksPerTile; ++i)
+                need_mask |= (blk0 + i < nb) && (sm.blk_pos[blk0 + i] + kGroupRows - 1 > tokx);
+            float mraw = -INFINITY;
             if (need_mask) {
 #pragma unroll
                 for (int i = 0; i < kBlocksPerTile; ++i) {
@@ -248,74 +272,63 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
 #pragma unroll
                     for (int e = 0; e < kGroupRows; ++e) {
                         const int c = i * kGroupRows + e;
-                        x[c] = (kp + e <= qpos) ? x[c] * sc : -INFINITY;
-                        mt_ = fmaxf(mt_, x[c]);
+                        sx[c] = (kp + e <= qpos) ? sx[c] : -INFINITY;
+                        mraw = fmaxf(mraw, sx[c]);
                     }
                 }
             } else {
 #pragma unroll
-                for (int c = 0; c < kTileKeys; ++c) {
-                    x[c] *= sc;
-                    mt_ = fmaxf(mt_, x[c]);
-                }
+                for (int c = 0; c < kTileKeys; ++c) mraw = fmaxf(mraw, sx[c]);
             }
-            const float m_new = fmaxf(m_used, mt_);
+            const float m_new = fmaxf(m_used, mraw * sc);
             bool rescale = false;
             float alpha = 1.f;
             if (m_new != -INFINITY) {
                 if (m_used == -INFINITY) {
                     m_used = m_new;
                 } else if (m_new > m_used + kRescaleLog2) {
-                    alpha = exp2f(m_used - m_new);
+                    alpha = ptx::ex2_approx(m_used - m_new);
                     m_used = m_new;
                     rescale = true;
                 }
             }
-            // probabilities (bf16-rounded; the sum uses the rounded values)
+            // P = 2^(S*sc - m), rounded to bf16; the row sum uses the rounded values
             uint32_t pk[kTileKeys / 2];
             float lsum = 0.f;
+            const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
 #pragma unroll
             for (int c = 0; c < kTileKeys; c += 2) {
-                const float p0 = m_used == -INFINITY ? 0.f : exp2f(x[c] - m_used);
-                const float p1 = m_used == -INFINITY ? 0.f : exp2f(x[c + 1] - m_used);
+                const float p0 = ptx::ex2_approx(fmaf(sx[c], sc, neg_m));
+                const float p1 = ptx::ex2_approx(fmaf(sx[c + 1], sc, neg_m));
                 __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
                 const float2 f2 = __bfloat1622float2(b2);
                 lsum += f2.x + f2.y;
                 pk[c / 2] = *reinterpret_cast<uint32_t*>(&b2);
             }
-            // the previous PV must be done before P is overwritten or O rescaled
-            if (t >= 1 && !__all_sync(0xffffffffu, wait_bar(&sm.pv_done, (t - 1) & 1, abort, p.err))) {
-                ok = false;
-                break;
-            }
             // tcgen05.ld/st are warp-collective: the whole warp rescales its
-            // rows when any row needs it (rows that do not use alpha = 1)
+            // rows when any row needs it (rows that do not use alpha = 1).
+            // PV of the previous tile has completed: S of this tile was issued
+            // after it on the same (in-order) tensor-core queue.
             if (__any_sync(0xffffffffu, rescale && t >= 1)) {
-                ptx::tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t o[32];
-                    ptx::tmem_ld32(lane_addr + kColO + 32 * c, o);
+                    ptx::tmem_ld32(o_addr + 32 * c, o);
                     ptx::tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    ptx::tmem_st32(lane_addr + kColO + 32 * c, o);
+                    ptx::tmem_st32(o_addr + 32 * c, o);
                 }
-                ptx::tmem_wait_st();
             }
             l = l * alpha + lsum;
-#pragma unroll
-            for (int q = 0; q < kTileKeys / 8; ++q) {
-                const int phys = (q & 7) ^ (r & 7);
-                uint4 v4 = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-                *reinterpret_cast<uint4*>(prow + (q >> 3) * kPanel + phys * 16) = v4;
-            }
-            ptx::fence_proxy_async_smem();
+            ptx::tmem_st32(s_addr, pk);
+            ptx::tmem_st32(s_addr + 32, pk + 32);
+            ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&sm.p_full);
+            if (lane == 0) ptx::mbar_arrive(&sm.p_full[x]);
         }
-        if (ok && __all_sync(0xffffffffu, wait_bar(&sm.pv_done, (n_tiles - 1) & 1, abort, p.err))) {
+        if (ok && __all_sync(0xffffffffu, wait_bar(&sm.o_done[x], 0, abort, p.err))) {
             ptx::tc_fence_after();
             const float inv = l > 0.f ? 1.0f / l : 0.f;
             __nv_bfloat16* orow =
@@ -323,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
-                ptx::tmem_ld32(lane_addr + kColO + 32 * c, o);
+                ptx::tmem_ld32(o_addr + 32 * c, o);
                 ptx::tmem_wait_ld();
                 if (row_ok) {
 #pragma unroll
@@ -355,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
 
 bool tc_kernel_supports(const Params& p, bool gathered) {
     return p.dtype == HGA_BF16 && p.d == kD && p.gq == 8 && p.q_len > 1 && !gathered &&
-           p.kv_layout == HGA_KV_FULL && p.C % 16 == 0;
+           p.kv_layout == HGA_KV_FULL && p.C % 32 == 0;
 }
 
 cudaError_t launch_attend_tc(const Params& p, const void* q_rot, const KvSources& kv,
@@ -375,7 +388,7 @@ cudaError_t launch_attend_tc(const Params& p, const void* q_rot, const KvSources
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    dim3 grid(p.C / 16, p.nQC, (unsigned)BH);
+    dim3 grid(p.C / 32, p.nQC, (unsigned)BH);
     attend_tc_kernel<<<grid, kThreads, smem, st>>>(maps, p, sel_groups, n_sel_groups,
                                                    (__nv_bfloat16*)out);
     return cudaGetLastError();

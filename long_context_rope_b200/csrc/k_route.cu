@@ -15,6 +15,9 @@
 // top-k by repeated warp arg-max and compacts the winners in ascending order.
 #include <cooperative_groups.h>
 
+#include <mutex>
+#include <set>
+
 #include "hga_kernels.h"
 
 namespace cg = cooperative_groups;
@@ -101,37 +104,75 @@ __device__ __forceinline__ void load_row(const float* row, int lane, float* v) {
 
 constexpr int kRowsInFlight = 8;
 
-// Leader warp: keep the top k of keys[0..n) (0 = absent), marking winners
-// with 1, then write them in ascending position order to out[0..k_cap)
-// (padded with -1) mapping position x -> idx_of(x). Returns the count kept.
+__host__ __device__ __forceinline__ int next_pow2(int n) {
+    int m = 1;
+    while (m < n) m <<= 1;
+    return m;
+}
+
+// Whole CTA: keep the top k of keys[0..n) (key 0 = absent; a key's low word
+// holds its candidate position) and write their mapped indices idx_of(x) in
+// ascending position order to out[0..k_cap), padded with -1. keys must have
+// room for next_pow2(n) entries; flags for ceil(n / 32) words. Sorting
+// (bitonic, descending) plus a position bitmap keeps every step parallel.
+// Returns the number kept (valid in warp 0).
 template <typename IndexOf>
-__device__ int select_and_compact(unsigned long long* keys, int n, int k, int k_cap,
-                                  int32_t* out, IndexOf idx_of) {
-    const int lane = threadIdx.x & 31;
-    int kept = 0;
-    for (; kept < k; ++kept) {
-        unsigned long long best = 0;
-        for (int x = lane; x < n; x += 32) {
-            unsigned long long v = keys[x];
-            best = v > best ? v : best;
+__device__ int cta_topk_compact(unsigned long long* keys, unsigned* flags, int n, int k,
+                                int k_cap, int32_t* out, IndexOf idx_of) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n2 = next_pow2(n);
+    const int nwords = (n + 31) >> 5;
+    for (int i = n + tid; i < n2; i += blockDim.x) keys[i] = 0ull;
+    for (int w = tid; w < nwords; w += blockDim.x) flags[w] = 0u;
+    __syncthreads();
+    for (int kk = 2; kk <= n2; kk <<= 1) {
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+            for (int i = tid; i < n2; i += blockDim.x) {
+                const int ixj = i ^ jj;
+                if (ixj > i) {
+                    const unsigned long long a = keys[i], b = keys[ixj];
+                    const bool desc = (i & kk) == 0;
+                    if ((a < b) == desc) {
+                        keys[i] = b;
+                        keys[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
         }
-        best = warp_max_u64(best);
-        if (best <= 1ull) break;
-        // the winning position: the lane that holds it marks it
-        for (int x = lane; x < n; x += 32)
-            if (keys[x] == best) keys[x] = 1ull;
-        __syncwarp();
     }
+    const int top = k < n ? k : n;
+    for (int i = tid; i < top; i += blockDim.x) {
+        const unsigned long long key = keys[i];
+        if (key > 1ull) {
+            const int x = rank_key_index(key);
+            atomicOr(&flags[x >> 5], 1u << (x & 31));
+        }
+    }
+    __syncthreads();
     int base = 0;
-    for (int x0 = 0; x0 < n; x0 += 32) {
-        const int x = x0 + lane;
-        const bool is = x < n && keys[x] == 1ull;
-        const unsigned m = __ballot_sync(0xffffffffu, is);
-        if (is) out[base + __popc(m & ((1u << lane) - 1u))] = idx_of(x);
-        base += __popc(m);
+    if (warp == 0) {
+        for (int w0 = 0; w0 < nwords; w0 += 32) {
+            const int w = w0 + lane;
+            unsigned f = w < nwords ? flags[w] : 0u;
+            const int c = __popc(f);
+            int incl = c;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            int o = base + incl - c;
+            while (f) {
+                const int bit = __ffs(f) - 1;
+                f &= f - 1u;
+                out[o++] = idx_of(w * 32 + bit);
+            }
+            base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        for (int s = base + lane; s < k_cap; s += 32) out[s] = -1;
     }
-    for (int s = kept + lane; s < k_cap; s += 32) out[s] = -1;
-    return kept;
+    return base;
 }
 
 // Level 1. Grid (CL, nQC, B*Hkv), cluster (CL, 1, 1), 256 threads.
@@ -194,10 +235,11 @@ __global__ void __launch_bounds__(256) route_chunks_kernel(Params p, const float
         for (int c = j + threadIdx.x; c < p.nC; c += blockDim.x)
             scores[prob * p.nC + c] = __int_as_float(0x7fc00000);
     cluster.sync();
-    if (r != 0 || warp != 0) return;
-    int kept = select_and_compact(keys, j, p.kc, p.kc, sel + prob * p.kc,
-                                  [](int x) { return x; });
-    if (lane == 0) nsel[prob] = kept;
+    if (r != 0) return;
+    unsigned* flags = reinterpret_cast<unsigned*>(keys + next_pow2(p.nC));
+    const int kept = cta_topk_compact(keys, flags, j, p.kc, p.kc, sel + prob * p.kc,
+                                      [](int x) { return x; });
+    if (threadIdx.x == 0) nsel[prob] = kept;
 }
 
 // Level 2. Grid (CL, nQC, B*Hkv), cluster (CL, 1, 1), 256 threads.
@@ -269,8 +311,9 @@ __global__ void __launch_bounds__(256) route_groups_kernel(
             const int x = x0 + lane;
             if (x < x_hi) {
                 const int c = s_chunk[x / p.G];
-                const int gi = c * p.G + x % p.G;
-                lk[x] = c < 0 ? 0ull : rank_key(s, gi);
+                // ties break on the candidate position x: candidates are in
+                // ascending global group order, so this equals breaking on gi
+                lk[x] = c < 0 ? 0ull : rank_key(s, x);
                 if (scores)
                     scores[prob * p.kc * p.G + x] = c < 0 ? __int_as_float(0x7fc00000) : s;
             }
@@ -280,11 +323,24 @@ __global__ void __launch_bounds__(256) route_groups_kernel(
         for (int x = ncand + threadIdx.x; x < p.kc * p.G; x += blockDim.x)
             scores[prob * p.kc * p.G + x] = __int_as_float(0x7fc00000);
     cluster.sync();
-    if (r != 0 || warp != 0) return;
+    if (r != 0) return;
     const int G = p.G;
-    int kept = select_and_compact(keys, ncand, p.kg, p.kg, sel_groups + prob * p.kg,
-                                  [&](int x) { return s_chunk[x / G] * G + x % G; });
-    if (lane == 0) n_sel_groups[prob] = kept;
+    unsigned* flags = reinterpret_cast<unsigned*>(keys + next_pow2(p.kc * p.G));
+    const int kept = cta_topk_compact(keys, flags, ncand, p.kg, p.kg, sel_groups + prob * p.kg,
+                                      [&](int x) { return s_chunk[x / G] * G + x % G; });
+    if (threadIdx.x == 0) n_sel_groups[prob] = kept;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per process (a driver
+// call per launch would add host latency to every decode step).
+cudaError_t allow_smem(const void* fn, size_t bytes) {
+    static std::mutex mu;
+    static std::set<const void*> done;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count(fn)) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) done.insert(fn);
+    return e;
 }
 
 cudaError_t launch_cluster(const void* fn, dim3 grid, int block, size_t smem, int cl,
@@ -333,14 +389,14 @@ cudaError_t launch_route_chunks(const Params& p, const float* qbar, const float*
                                 int32_t* sel, int32_t* n_sel, float* scores, cudaStream_t st) {
     if (p.nQC == 0) return cudaSuccess;
     const int cl = chunk_cluster(p);
-    size_t smem = (size_t)p.nC * sizeof(unsigned long long);
+    size_t smem = (size_t)next_pow2(p.nC) * sizeof(unsigned long long) +
+                  (size_t)((p.nC + 31) / 32) * sizeof(unsigned);
     dim3 grid(cl, p.nQC, p.B * p.Hkv);
     Params pp = p;
     void* args[] = {&pp, (void*)&qbar, (void*)&chunk_sum, &sel, &n_sel, &scores};
     const void* fn = p.d == 128 ? (const void*)route_chunks_kernel<4>
                                 : (const void*)route_chunks_kernel<2>;
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(smem > 48 * 1024 ? smem : 48 * 1024));
+    cudaError_t e = allow_smem(fn, kMaxChunks * (sizeof(unsigned long long) + 1));
     if (e != cudaSuccess) return e;
     return launch_cluster(fn, grid, 256, smem, cl, st, args);
 }
@@ -352,15 +408,15 @@ cudaError_t launch_route_groups(const Params& p, const float* qbar, const float*
     if (p.nQC == 0) return cudaSuccess;
     const int64_t problems = (int64_t)p.B * p.Hkv * p.nQC;
     const int cl = problems >= 1024 ? 1 : 4;
-    size_t smem = (size_t)p.kc * p.G * sizeof(unsigned long long);
+    size_t smem = (size_t)next_pow2(p.kc * p.G) * sizeof(unsigned long long) +
+                  (size_t)((p.kc * p.G + 31) / 32) * sizeof(unsigned);
     dim3 grid(cl, p.nQC, p.B * p.Hkv);
     Params pp = p;
     void* args[] = {&pp, (void*)&qbar, (void*)&group_sum, (void*)&sel_chunks,
                     (void*)&n_sel_chunks, &sel_groups, &n_sel_groups, &scores};
     const void* fn = p.d == 128 ? (const void*)route_groups_kernel<4>
                                 : (const void*)route_groups_kernel<2>;
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(smem > 48 * 1024 ? smem : 48 * 1024));
+    cudaError_t e = allow_smem(fn, 8192 * (sizeof(unsigned long long) + 1));
     if (e != cudaSuccess) return e;
     return launch_cluster(fn, grid, 256, smem, cl, st, args);
 }
