@@ -176,9 +176,11 @@ hga_status hga_route_chunks(const hga_config* cfg, const void* q_rot, const floa
         return HGA_ERR_ALIGN;
     HGA_ATTACH_ERR(p);
     cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = launch_qbar(p, q_rot, qbar_out, st);
-    if (e != cudaSuccess) return HGA_ERR_CUDA;
-    return launched(launch_route_chunks(p, qbar_out, chunk_sum, sel_chunks, n_sel_chunks,
+    if (!route_chunks_fuses_qbar(p)) {
+        cudaError_t e = launch_qbar(p, q_rot, qbar_out, st);
+        if (e != cudaSuccess) return HGA_ERR_CUDA;
+    }
+    return launched(launch_route_chunks(p, q_rot, qbar_out, chunk_sum, sel_chunks, n_sel_chunks,
                                         scores_out, st));
 }
 

@@ -23,8 +23,20 @@ cudaError_t launch_summaries(const Params& p, const void* k_raw, float* chunk_su
 
 cudaError_t launch_qbar(const Params& p, const void* q_rot, float* qbar, cudaStream_t st);
 
-cudaError_t launch_route_chunks(const Params& p, const float* qbar, const float* chunk_sum,
-                                int32_t* sel, int32_t* n_sel, float* scores, cudaStream_t st);
+// Level-1 routing. q-bar must already be in `qbar` unless
+// route_chunks_fuses_qbar(p), in which case the kernel forms it from q_rot
+// and writes it to `qbar` (few query tokens: decode).
+bool route_chunks_fuses_qbar(const Params& p);
+cudaError_t launch_route_chunks(const Params& p, const void* q_rot, float* qbar,
+                                const float* chunk_sum, int32_t* sel, int32_t* n_sel,
+                                float* scores, cudaStream_t st);
+
+// Prefill form of level-1 routing: 16 query chunks per CTA share one pass
+// over the chunk-summary table (needs nQC >= 8 and nC <= 2048).
+bool route_chunks_tiled_supports(const Params& p);
+cudaError_t launch_route_chunks_tiled(const Params& p, const float* qbar, const float* chunk_sum,
+                                      int32_t* sel, int32_t* n_sel, float* scores,
+                                      cudaStream_t st);
 
 cudaError_t launch_route_groups(const Params& p, const float* qbar, const float* group_sum,
                                 const int32_t* sel_chunks, const int32_t* n_sel_chunks,

@@ -70,9 +70,11 @@ __global__ void __launch_bounds__(256) qbar_kernel(Params p, const T* __restrict
             float acc[V];
 #pragma unroll
             for (int e = 0; e < V; ++e) acc[e] = 0.f;
+#pragma unroll 2
             for (int64_t pos = pos_lo + tl; pos < pos_hi; pos += TL) {
                 const T* row = q + (((int64_t)b * p.q_len + (pos - p.q_begin)) * p.Hq +
                                     (int64_t)h * p.gq) * p.d + v * V;
+#pragma unroll 8
                 for (int r = 0; r < p.gq; ++r) QVec<T>::add(row + (int64_t)r * p.d, acc);
             }
 #pragma unroll
@@ -177,7 +179,9 @@ __device__ int cta_topk_compact(unsigned long long* keys, unsigned* flags, int n
 
 // Level 1. Grid (CL, nQC, B*Hkv), cluster (CL, 1, 1), 256 threads.
 template <int DPL>
-__global__ void __launch_bounds__(256) route_chunks_kernel(Params p, const float* __restrict__ qbar,
+__global__ void __launch_bounds__(256) route_chunks_kernel(Params p, float* __restrict__ qbar,
+                                                           const void* __restrict__ q_rot,
+                                                           int fuse_qbar,
                                                            const float* __restrict__ cs,
                                                            int32_t* __restrict__ sel,
                                                            int32_t* __restrict__ nsel,
@@ -194,7 +198,40 @@ __global__ void __launch_bounds__(256) route_chunks_kernel(Params p, const float
     unsigned long long* lk = cluster.map_shared_rank(keys, 0);
 
     float q[DPL];
-    {
+    if (fuse_qbar) {
+        // few query tokens (decode): every CTA forms q-bar itself from the
+        // rotated queries (a few KB), rank 0 publishes it for level 2
+        const int64_t span_end = (int64_t)p.q_begin + p.q_len;
+        const int64_t pos_lo = (int64_t)j * p.C > p.q_begin ? (int64_t)j * p.C : p.q_begin;
+        const int64_t pos_hi = (int64_t)(j + 1) * p.C < span_end ? (int64_t)(j + 1) * p.C : span_end;
+        const int hk = (int)(bh % p.Hkv);
+        const int64_t b = bh / p.Hkv;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) q[e] = 0.f;
+        for (int64_t pos = pos_lo; pos < pos_hi; ++pos) {
+            const int64_t row0 = ((b * p.q_len + (pos - p.q_begin)) * p.Hq + (int64_t)hk * p.gq) * p.d;
+#pragma unroll 8
+            for (int r2 = 0; r2 < p.gq; ++r2) {
+                const int64_t off = row0 + (int64_t)r2 * p.d + lane * DPL;
+                if (p.dtype == HGA_BF16) {
+                    const __nv_bfloat16* qp = reinterpret_cast<const __nv_bfloat16*>(q_rot) + off;
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) q[e] += __bfloat162float(qp[e]);
+                } else {
+                    const float* qp = reinterpret_cast<const float*>(q_rot) + off;
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) q[e] += qp[e];
+                }
+            }
+        }
+        const float inv_n = 1.0f / (float)((pos_hi - pos_lo) * p.gq);
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) q[e] *= inv_n;
+        if (r == 0 && warp == 0) {
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) qbar[prob * p.d + lane * DPL + e] = q[e];
+        }
+    } else {
         const float* qr = qbar + prob * p.d;
 #pragma unroll
         for (int e = 0; e < DPL; ++e) q[e] = qr[lane * DPL + e];
@@ -385,15 +422,23 @@ static int chunk_cluster(const Params& p) {
     return p.nC >= 256 ? 8 : (p.nC >= 64 ? 4 : 1);
 }
 
-cudaError_t launch_route_chunks(const Params& p, const float* qbar, const float* chunk_sum,
-                                int32_t* sel, int32_t* n_sel, float* scores, cudaStream_t st) {
+bool route_chunks_fuses_qbar(const Params& p) {
+    return !route_chunks_tiled_supports(p) && p.q_len <= 4;
+}
+
+cudaError_t launch_route_chunks(const Params& p, const void* q_rot, float* qbar,
+                                const float* chunk_sum, int32_t* sel, int32_t* n_sel,
+                                float* scores, cudaStream_t st) {
     if (p.nQC == 0) return cudaSuccess;
+    if (route_chunks_tiled_supports(p))
+        return launch_route_chunks_tiled(p, qbar, chunk_sum, sel, n_sel, scores, st);
+    int fuse = route_chunks_fuses_qbar(p) ? 1 : 0;
     const int cl = chunk_cluster(p);
     size_t smem = (size_t)next_pow2(p.nC) * sizeof(unsigned long long) +
                   (size_t)((p.nC + 31) / 32) * sizeof(unsigned);
     dim3 grid(cl, p.nQC, p.B * p.Hkv);
     Params pp = p;
-    void* args[] = {&pp, (void*)&qbar, (void*)&chunk_sum, &sel, &n_sel, &scores};
+    void* args[] = {&pp, (void*)&qbar, (void*)&q_rot, &fuse, (void*)&chunk_sum, &sel, &n_sel, &scores};
     const void* fn = p.d == 128 ? (const void*)route_chunks_kernel<4>
                                 : (const void*)route_chunks_kernel<2>;
     cudaError_t e = allow_smem(fn, kMaxChunks * (sizeof(unsigned long long) + 1));

@@ -1,0 +1,237 @@
+// k_route_tiled.cu -- level-1 routing for many query chunks at once (prefill).
+//
+// "Technische Samenvatting: Hierarchical Global Attention (HGA)"
+// (gist.science), "Kernmechanisme" item 2, Niveau 1: every query chunk
+// scores the table of chunk key summaries of its earlier chunks and keeps the
+// top-k; sink, local and current chunks are always visible and never routed.
+//
+// In prefill all query chunks of one (sequence, KV head) score the same
+// table, so a CTA takes 16 query chunks and streams the table through shared
+// memory once for all of them: a register-blocked fp32 product (each thread
+// 4 query chunks x 4 table rows) writes the 16 score rows to shared memory.
+// Each warp then selects the top-k of its query chunks with a 4-pass radix
+// select (8-bit digits of the order-preserving score key, warp-private
+// histograms) and writes the winners in ascending chunk order. Ties on the
+// threshold score go to the lower chunk index; NaN ranks last.
+#include "hga_kernels.h"
+
+namespace hga {
+
+namespace {
+
+constexpr int kQB = 16;          // query chunks per CTA
+constexpr int kCT = 256;         // table rows per tile
+constexpr int kKS = 32;          // dims per k-slice
+constexpr int kThreads = 256;
+
+// Order-preserving 32-bit key of a score: larger score -> larger key; -0 == +0;
+// NaN -> 0 (below every number).
+__device__ __forceinline__ uint32_t score_key(float s) {
+    if (s != s) return 0u;
+    s += 0.0f;
+    const uint32_t b = __float_as_uint(s);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) route_chunks_tiled_kernel(
+    Params p, const float* __restrict__ qbar, const float* __restrict__ cs,
+    int32_t* __restrict__ sel, int32_t* __restrict__ nsel, float* __restrict__ scores_out) {
+    extern __shared__ __align__(16) float smem_f[];
+    float* qT = smem_f;                         // [D][kQB]   transposed q-bar
+    float* tile = qT + D * kQB;                 // [kKS][kCT] transposed table slice
+    float* sc = tile + kKS * kCT;               // [kQB][ncp] scores
+    const int ncp = (p.nC + 3) & ~3;
+    uint32_t* hist = reinterpret_cast<uint32_t*>(sc + kQB * ncp);  // [8 warps][256]
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t bh = blockIdx.y;
+    const int jj0 = blockIdx.x * kQB;
+    const int nq = p.nQC - jj0 < kQB ? p.nQC - jj0 : kQB;
+    const int j_hi = p.j0 + jj0 + nq;           // chunks [0, j_hi - 1) are candidates at most
+
+    for (int x = tid; x < D * kQB; x += kThreads) {
+        const int q = x % kQB, k = x / kQB;
+        qT[x] = q < nq ? qbar[((bh * p.nQC) + jj0 + q) * D + k] : 0.f;
+    }
+    const float* table = cs + bh * (int64_t)p.nC * D;
+    const int qg = tid & 3;                     // query group: queries 4*qg .. 4*qg+3
+    const int cg = tid >> 2;                    // table group: rows 4*cg .. 4*cg+3 of the tile
+    for (int c0 = 0; c0 < j_hi - 1; c0 += kCT) {
+        float acc[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) acc[a][bb] = 0.f;
+        for (int k0 = 0; k0 < D; k0 += kKS) {
+            __syncthreads();
+            {
+                // row c0 + tid of the table, dims k0 .. k0 + kKS, written transposed
+                const int c = c0 + tid;
+                const bool in = c < p.nC;
+#pragma unroll
+                for (int v = 0; v < kKS / 4; ++v) {
+                    float4 t = in ? __ldg(reinterpret_cast<const float4*>(table + (int64_t)c * D + k0) + v)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                    tile[(4 * v + 0) * kCT + tid] = t.x;
+                    tile[(4 * v + 1) * kCT + tid] = t.y;
+                    tile[(4 * v + 2) * kCT + tid] = t.z;
+                    tile[(4 * v + 3) * kCT + tid] = t.w;
+                }
+            }
+            __syncthreads();
+#pragma unroll 8
+            for (int k = 0; k < kKS; ++k) {
+                const float4 qv = *reinterpret_cast<const float4*>(qT + (k0 + k) * kQB + 4 * qg);
+                const float4 tv = *reinterpret_cast<const float4*>(tile + k * kCT + 4 * cg);
+                const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
+                const float ta[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int bb = 0; bb < 4; ++bb) acc[a][bb] = fmaf(qa[a], ta[bb], acc[a][bb]);
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                const int c = c0 + 4 * cg + bb;
+                if (c < ncp) sc[(4 * qg + a) * ncp + c] = acc[a][bb];
+            }
+    }
+    __syncthreads();
+
+    // ---- per query chunk: radix top-k over its candidates (one warp each)
+    uint32_t* h = hist + warp * 256;
+    for (int q = warp; q < nq; q += kThreads / 32) {
+        const int jj = jj0 + q, j = p.j0 + jj;
+        const int64_t prob = bh * p.nQC + jj;
+        const float* srow = sc + q * ncp;
+        auto cand = [&](int c) { return c < j && !is_forced(p, j, c); };
+        // candidates count
+        int n_cand = 0;
+        for (int c0 = 0; c0 < j; c0 += 32) {
+            const int c = c0 + lane;
+            n_cand += __popc(__ballot_sync(0xffffffffu, c < j && cand(c)));
+        }
+        const int k = p.kc < n_cand ? p.kc : n_cand;
+        uint32_t prefix = 0u, mask = 0u;
+        int need = k;
+        if (k < n_cand) {
+            for (int shift = 24; shift >= 0; shift -= 8) {
+                for (int b = lane; b < 256; b += 32) h[b] = 0u;
+                __syncwarp();
+                for (int c = lane; c < j; c += 32) {
+                    if (!cand(c)) continue;
+                    const uint32_t key = score_key(srow[c]);
+                    if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+                }
+                __syncwarp();
+                // digits in descending order: lane L owns digits 255-8L .. 248-8L
+                uint32_t cnt[8];
+                uint32_t lsum = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    cnt[i] = h[255 - 8 * lane - i];
+                    lsum += cnt[i];
+                }
+                uint32_t incl = lsum;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += v;
+                }
+                const uint32_t excl = incl - lsum;
+                // the lane whose range holds the need-th largest
+                const bool here = excl < (uint32_t)need && (uint32_t)need <= incl;
+                const unsigned hm = __ballot_sync(0xffffffffu, here);
+                const int owner = hm ? __ffs(hm) - 1 : 0;
+                uint32_t digit = 0u, above = 0u;
+                if (lane == owner) {
+                    uint32_t run = excl;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        if (run + cnt[i] >= (uint32_t)need) {
+                            digit = 255u - 8u * lane - i;
+                            above = run;
+                            break;
+                        }
+                        run += cnt[i];
+                    }
+                }
+                digit = __shfl_sync(0xffffffffu, digit, owner);
+                above = __shfl_sync(0xffffffffu, above, owner);
+                need -= (int)above;
+                prefix |= digit << shift;
+                mask |= 255u << shift;
+                __syncwarp();
+            }
+        }
+        // keys > prefix are in; among keys == prefix the first `need` (by index) are in
+        int base = 0, ties = 0;
+        int32_t* out = sel + prob * p.kc;
+        for (int c0 = 0; c0 < j; c0 += 32) {
+            const int c = c0 + lane;
+            bool is = false, tie = false;
+            if (c < j && cand(c)) {
+                if (k >= n_cand) {
+                    is = true;
+                } else {
+                    const uint32_t key = score_key(srow[c]);
+                    is = key > prefix;
+                    tie = key == prefix;
+                }
+            }
+            const unsigned tm = __ballot_sync(0xffffffffu, tie);
+            const int trank = ties + __popc(tm & ((1u << lane) - 1u));
+            is = is || (tie && trank < need);
+            ties += __popc(tm);
+            const unsigned m = __ballot_sync(0xffffffffu, is);
+            if (is) out[base + __popc(m & ((1u << lane) - 1u))] = c;
+            base += __popc(m);
+        }
+        for (int s = base + lane; s < p.kc; s += 32) out[s] = -1;
+        if (lane == 0) nsel[prob] = base;
+        if (scores_out) {
+            float* so = scores_out + prob * p.nC;
+            for (int c = lane; c < p.nC; c += 32)
+                so[c] = cand(c) ? srow[c] : __int_as_float(0x7fc00000);
+        }
+    }
+}
+
+}  // namespace
+
+bool route_chunks_tiled_supports(const Params& p) {
+    return p.nQC >= 8 && p.nC <= 2048 && (p.d == 128 || p.d == 64);
+}
+
+cudaError_t launch_route_chunks_tiled(const Params& p, const float* qbar, const float* chunk_sum,
+                                      int32_t* sel, int32_t* n_sel, float* scores,
+                                      cudaStream_t st) {
+    const int ncp = (p.nC + 3) & ~3;
+    const size_t smem = (size_t)(p.d * kQB + kKS * kCT + kQB * ncp) * sizeof(float) +
+                        (size_t)(kThreads / 32) * 256 * sizeof(uint32_t);
+    dim3 grid((p.nQC + kQB - 1) / kQB, p.B * p.Hkv);
+    const void* fn = p.d == 128 ? (const void*)route_chunks_tiled_kernel<128>
+                                : (const void*)route_chunks_tiled_kernel<64>;
+    static bool attr = false;
+    if (!attr) {
+        const size_t max_smem = (size_t)(128 * kQB + kKS * kCT + kQB * 2048) * sizeof(float) +
+                                (size_t)(kThreads / 32) * 256 * sizeof(uint32_t);
+        cudaError_t e = cudaFuncSetAttribute(route_chunks_tiled_kernel<128>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)max_smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(route_chunks_tiled_kernel<64>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_smem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    Params pp = p;
+    void* args[] = {&pp, (void*)&qbar, (void*)&chunk_sum, &sel, &n_sel, &scores};
+    return cudaLaunchKernel(fn, grid, dim3(kThreads), args, smem, st);
+}
+
+}  // namespace hga
