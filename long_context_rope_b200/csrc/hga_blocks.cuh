@@ -31,17 +31,27 @@ __device__ __forceinline__ int checked_group_entry(const Params& p, int j, const
 }
 
 // Fill blk_row / blk_pos for query chunk j and return the number of blocks
-// (in every lane). Called by all 32 lanes of one warp. Forced chunks come
-// first in ascending order, then the routed groups in list order; blocks
-// that start at or past L are dropped; invalid list entries are skipped (and
-// recorded in the device error word). Rows of the resident store: the token
-// position (HGA_KV_FULL) or slot * C + 16 * gamma (HGA_KV_WINDOWS). Rows of
-// the gathered buffer: kSrcGathered | 16 * slot. The caller guarantees the
-// output capacity (G * forced chunks + top_k_groups <= kMaxBlocks).
+// (in every lane). Called by all 32 lanes of one warp. `list` holds the
+// selection (top_k_groups slots) and `n_list_ptr` its count. Forced chunks
+// come first in ascending order, then the routed groups in list order;
+// blocks that start at or past L are dropped; invalid list entries are
+// skipped (and recorded in the device error word). Rows of the resident
+// store: the token position (HGA_KV_FULL) or slot * C + 16 * gamma
+// (HGA_KV_WINDOWS). Rows of the gathered buffer: kSrcGathered | 16 * slot.
+// The count and the first 128 list slots are loaded in one round trip. The
+// caller guarantees the capacity (G * forced chunks + top_k_groups <= kMaxBlocks).
 __device__ __forceinline__ int build_key_blocks_warp(const Params& p, int j, const int32_t* list,
-                                                     int n_list, bool gathered, int* blk_row,
-                                                     int* blk_pos) {
+                                                     const int32_t* n_list_ptr, bool gathered,
+                                                     int* blk_row, int* blk_pos) {
     const int lane = threadIdx.x & 31;
+    constexpr int kPre = 4;  // slots loaded ahead per lane (128 per warp)
+    int n_list = n_list_ptr ? *n_list_ptr : 0;
+    int pre[kPre];
+#pragma unroll
+    for (int u = 0; u < kPre; ++u) {
+        const int s = lane + 32 * u;
+        pre[u] = (list != nullptr && s < p.kg) ? list[s] : -1;
+    }
     const int s_end = p.n_sink < j + 1 ? p.n_sink : j + 1;
     const int l_begin = j - p.n_local > s_end ? j - p.n_local : s_end;
     const int nf = s_end + (j + 1 - l_begin);
@@ -70,18 +80,27 @@ __device__ __forceinline__ int build_key_blocks_warp(const Params& p, int j, con
         if (lane == 0) raise_dev_error(p, kDevErrCount);
         n_list = n_list < 0 ? 0 : p.kg;
     }
+    int carry = -1;  // list[s0 - 1]
     for (int s0 = 0; s0 < n_list; s0 += 32) {
         const int s = s0 + lane;
-        int gi = -1;
+        const int u = s0 >> 5;
+        int gi = u < kPre ? pre[0] : -1;
+#pragma unroll
+        for (int v = 1; v < kPre; ++v)
+            if (u == v) gi = pre[v];
+        if (u >= kPre && s < n_list) gi = list[s];
+        int prev = __shfl_up_sync(0xffffffffu, gi, 1);
+        if (lane == 0) prev = carry;
+        carry = __shfl_sync(0xffffffffu, gi, 31);
         if (s < n_list) {
-            gi = list[s];
-            const int prev = s > 0 ? list[s - 1] : -1;
             const int c = gi >= 0 ? gi / p.G : -1;
             const bool ok = gi >= 0 && c < j && !is_forced(p, j, c) && (s == 0 || gi > prev);
             if (!ok) {
                 raise_dev_error(p, kDevErrGroupIndex);
                 gi = -1;
             }
+        } else {
+            gi = -1;
         }
         const unsigned m = __ballot_sync(0xffffffffu, gi >= 0);
         if (gi >= 0) {

@@ -65,34 +65,6 @@ __device__ __forceinline__ void rope_cs(double pos, double inv_freq, float& c, f
     sincosf((float)r, &s, &c);
 }
 
-// Total order used by every top-k: a larger key ranks first. Higher score
-// first; -0 equals +0; NaN ranks below every number; ties go to the lower
-// index. Valid keys are > 0 (the low word is ~index with index < 2^31).
-__device__ __forceinline__ unsigned long long rank_key(float score, int index) {
-    uint32_t hi;
-    if (score != score) {
-        hi = 0u;
-    } else {
-        score += 0.0f;  // -0 -> +0
-        uint32_t b = __float_as_uint(score);
-        hi = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-    }
-    return ((unsigned long long)hi << 32) | (unsigned long long)(~(uint32_t)index);
-}
-
-__device__ __forceinline__ int rank_key_index(unsigned long long key) {
-    return (int)(~(uint32_t)(key & 0xffffffffull));
-}
-
-__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        unsigned long long o = __shfl_xor_sync(0xffffffffu, v, off);
-        v = o > v ? o : v;
-    }
-    return v;
-}
-
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);

@@ -8,8 +8,8 @@
 // read once, and the query heads of a KV head share each load (GQA).
 //
 // One cluster of CL CTAs per (sequence, KV head), CL chosen so the grid
-// covers the SMs about once. CTA r owns a contiguous share of the unit's
-// 16-row key blocks and streams them through a 16-stage shared-memory ring
+// fills every SM with two CTAs at once. CTA r owns a contiguous share of the
+// unit's 16-row key blocks and streams them through an 8-stage shared-memory ring
 // filled by TMA (tensor-map tile loads, 128-byte swizzle; one producer
 // thread). Eight consumer warps take every 8th block: S^T[16 keys x 8 heads]
 // = K_blk Q^T and O^T[128 dims x 8 heads] += V^T P^T on warp-level bf16 MMA
@@ -30,7 +30,7 @@ namespace hga {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kStages = 16;                      // ring of key blocks
+constexpr int kStages = 8;                       // ring of key blocks
 constexpr int kBlkBytes = kGroupRows * kD * 2;   // 4 KiB per block per tensor
 constexpr int kConsumers = 8;                    // consumer warps
 constexpr int kThreads = (kConsumers + 1) * 32;  // + one producer warp
@@ -62,7 +62,7 @@ struct DecodeSmem {
     int bad;
 };
 
-__global__ void __launch_bounds__(kThreads, 1) attend_decode_kernel(
+__global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
     const __grid_constant__ DecodeMaps maps, Params p, const __nv_bfloat16* __restrict__ q,
     const int32_t* __restrict__ sel, const int32_t* __restrict__ nsel,
     __nv_bfloat16* __restrict__ out, int gathered) {
@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_decode_kernel(
     const int qpos = p.q_begin;
 
     if (warp == 0) {
-        const int nb_w = build_key_blocks_warp(p, j, sel + prob * p.kg, nsel[prob], gathered != 0,
+        const int nb_w = build_key_blocks_warp(p, j, sel + prob * p.kg, nsel + prob, gathered != 0,
                                                sm.blk_row, sm.blk_pos);
         if (lane == 0) {
             sm.nb = nb_w;
@@ -162,16 +162,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_decode_kernel(
                 }
                 break;
             }
-            // S^T = K Q^T for 16 keys x 8 heads
-            float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+            // S^T = K Q^T for 16 keys x 8 heads (two accumulator chains)
+            float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sacc2[4] = {0.f, 0.f, 0.f, 0.f};
             const uint32_t kb = ptx::smem_u32(sm.u.ring.k[s]);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const int chunk = (kk & 3) * 2 + (mq >> 1);
                 uint32_t a[4];
                 ptx::ldsm_x4(kb + (kk >> 2) * 2048 + krow * 128 + ((chunk ^ (krow & 7)) << 4), a);
-                ptx::mma_16816(sacc, a, qf[kk][0], qf[kk][1]);
+                ptx::mma_16816((kk & 1) ? sacc2 : sacc, a, qf[kk][0], qf[kk][1]);
             }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[e] += sacc2[e];
             // this lane holds keys g, g+8 for heads 2t4, 2t4+1
             const int kp = sm.blk_pos[lo + i];
             const bool v0 = kp + g <= qpos, v1 = kp + g + 8 <= qpos;
@@ -320,7 +322,7 @@ int pick_cluster(const Params& p, size_t smem) {
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int units = p.B * p.Hkv;
-    int cl = sms / units;
+    int cl = 2 * sms / units;  // two CTAs per SM
     cl = cl < 1 ? 1 : (cl > kMaxCluster ? kMaxCluster : cl);
     for (; cl > 1; --cl) {
         if (max_active[cl] == 0) {

@@ -69,8 +69,8 @@ __global__ void __launch_bounds__(128) attend_simt_kernel(Params p, const T* __r
 
     if (warp == 0) {
         const int32_t* list = sel ? sel + prob * p.kg : nullptr;
-        const int n_list = sel ? nsel[prob] : 0;
-        const int nb_w = build_key_blocks_warp(p, j, list, n_list, gathered, blk_row, blk_pos);
+        const int nb_w = build_key_blocks_warp(p, j, list, sel ? nsel + prob : nullptr, gathered,
+                                               blk_row, blk_pos);
         if (lane == 0) s_nb = nb_w;
     }
     for (int x = tid; x < kRowsPerCta * D; x += blockDim.x) {

@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     if (tok0 >= span_end || tok0 + 32 <= p.q_begin) return;
 
     if (warp == 0) {
-        const int nb_w = build_key_blocks_warp(p, j, sel + prob * p.kg, nsel[prob], false,
+        const int nb_w = build_key_blocks_warp(p, j, sel + prob * p.kg, nsel + prob, false,
                                                sm.blk_row, sm.blk_pos);
         if (lane == 0) {
             sm.nb = nb_w;

@@ -19,6 +19,7 @@
 #include <set>
 
 #include "hga_kernels.h"
+#include "hga_topk.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -106,77 +107,6 @@ __device__ __forceinline__ void load_row(const float* row, int lane, float* v) {
 
 constexpr int kRowsInFlight = 8;
 
-__host__ __device__ __forceinline__ int next_pow2(int n) {
-    int m = 1;
-    while (m < n) m <<= 1;
-    return m;
-}
-
-// Whole CTA: keep the top k of keys[0..n) (key 0 = absent; a key's low word
-// holds its candidate position) and write their mapped indices idx_of(x) in
-// ascending position order to out[0..k_cap), padded with -1. keys must have
-// room for next_pow2(n) entries; flags for ceil(n / 32) words. Sorting
-// (bitonic, descending) plus a position bitmap keeps every step parallel.
-// Returns the number kept (valid in warp 0).
-template <typename IndexOf>
-__device__ int cta_topk_compact(unsigned long long* keys, unsigned* flags, int n, int k,
-                                int k_cap, int32_t* out, IndexOf idx_of) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n2 = next_pow2(n);
-    const int nwords = (n + 31) >> 5;
-    for (int i = n + tid; i < n2; i += blockDim.x) keys[i] = 0ull;
-    for (int w = tid; w < nwords; w += blockDim.x) flags[w] = 0u;
-    __syncthreads();
-    for (int kk = 2; kk <= n2; kk <<= 1) {
-        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-            for (int i = tid; i < n2; i += blockDim.x) {
-                const int ixj = i ^ jj;
-                if (ixj > i) {
-                    const unsigned long long a = keys[i], b = keys[ixj];
-                    const bool desc = (i & kk) == 0;
-                    if ((a < b) == desc) {
-                        keys[i] = b;
-                        keys[ixj] = a;
-                    }
-                }
-            }
-            __syncthreads();
-        }
-    }
-    const int top = k < n ? k : n;
-    for (int i = tid; i < top; i += blockDim.x) {
-        const unsigned long long key = keys[i];
-        if (key > 1ull) {
-            const int x = rank_key_index(key);
-            atomicOr(&flags[x >> 5], 1u << (x & 31));
-        }
-    }
-    __syncthreads();
-    int base = 0;
-    if (warp == 0) {
-        for (int w0 = 0; w0 < nwords; w0 += 32) {
-            const int w = w0 + lane;
-            unsigned f = w < nwords ? flags[w] : 0u;
-            const int c = __popc(f);
-            int incl = c;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += v;
-            }
-            int o = base + incl - c;
-            while (f) {
-                const int bit = __ffs(f) - 1;
-                f &= f - 1u;
-                out[o++] = idx_of(w * 32 + bit);
-            }
-            base += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        for (int s = base + lane; s < k_cap; s += 32) out[s] = -1;
-    }
-    return base;
-}
-
 // Level 1. Grid (CL, nQC, B*Hkv), cluster (CL, 1, 1), 256 threads.
 template <int DPL>
 __global__ void __launch_bounds__(256) route_chunks_kernel(Params p, float* __restrict__ qbar,
@@ -186,7 +116,7 @@ __global__ void __launch_bounds__(256) route_chunks_kernel(Params p, float* __re
                                                            int32_t* __restrict__ sel,
                                                            int32_t* __restrict__ nsel,
                                                            float* __restrict__ scores) {
-    extern __shared__ unsigned long long keys[];
+    extern __shared__ uint32_t keys[];     // [nC] candidate keys, then 256 histogram words
     cg::cluster_group cluster = cg::this_cluster();
     const int CL = (int)cluster.num_blocks();
     const int r = (int)cluster.block_rank();
@@ -195,7 +125,7 @@ __global__ void __launch_bounds__(256) route_chunks_kernel(Params p, float* __re
     const int j = p.j0 + jj;
     const int64_t prob = bh * p.nQC + jj;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    unsigned long long* lk = cluster.map_shared_rank(keys, 0);
+    uint32_t* lk = cluster.map_shared_rank(keys, 0);
 
     float q[DPL];
     if (fuse_qbar) {
@@ -263,7 +193,7 @@ __global__ void __launch_bounds__(256) route_chunks_kernel(Params p, float* __re
             const int c = c0 + lane;
             if (c < c_hi) {
                 const bool forced = is_forced(p, j, c);
-                lk[c] = forced ? 0ull : rank_key(s, c);
+                lk[c] = forced ? 0u : score_key32(s);
                 if (scores) scores[prob * p.nC + c] = forced ? __int_as_float(0x7fc00000) : s;
             }
         }
@@ -272,11 +202,10 @@ __global__ void __launch_bounds__(256) route_chunks_kernel(Params p, float* __re
         for (int c = j + threadIdx.x; c < p.nC; c += blockDim.x)
             scores[prob * p.nC + c] = __int_as_float(0x7fc00000);
     cluster.sync();
-    if (r != 0) return;
-    unsigned* flags = reinterpret_cast<unsigned*>(keys + next_pow2(p.nC));
-    const int kept = cta_topk_compact(keys, flags, j, p.kc, p.kc, sel + prob * p.kc,
-                                      [](int x) { return x; });
-    if (threadIdx.x == 0) nsel[prob] = kept;
+    if (r != 0 || warp != 0) return;
+    const int kept = warp_radix_topk(keys, j, p.kc, p.kc, sel + prob * p.kc, keys + p.nC,
+                                     [](int x) { return x; });
+    if (lane == 0) nsel[prob] = kept;
 }
 
 // Level 2. Grid (CL, nQC, B*Hkv), cluster (CL, 1, 1), 256 threads.
@@ -286,7 +215,7 @@ __global__ void __launch_bounds__(256) route_groups_kernel(
     const int32_t* __restrict__ sel_chunks, const int32_t* __restrict__ n_sel_chunks,
     int32_t* __restrict__ sel_groups, int32_t* __restrict__ n_sel_groups,
     float* __restrict__ scores) {
-    extern __shared__ unsigned long long keys[];
+    extern __shared__ uint32_t keys[];     // [kc*G] candidate keys, then 256 histogram words
     __shared__ int s_chunk[1024];  // validated chunk of each slot, -1 if invalid
     cg::cluster_group cluster = cg::this_cluster();
     const int CL = (int)cluster.num_blocks();
@@ -296,7 +225,7 @@ __global__ void __launch_bounds__(256) route_groups_kernel(
     const int j = p.j0 + jj;
     const int64_t prob = bh * p.nQC + jj;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    unsigned long long* lk = cluster.map_shared_rank(keys, 0);
+    uint32_t* lk = cluster.map_shared_rank(keys, 0);
 
     int n = n_sel_chunks[prob];
     if (n < 0 || n > p.kc) {
@@ -350,7 +279,7 @@ __global__ void __launch_bounds__(256) route_groups_kernel(
                 const int c = s_chunk[x / p.G];
                 // ties break on the candidate position x: candidates are in
                 // ascending global group order, so this equals breaking on gi
-                lk[x] = c < 0 ? 0ull : rank_key(s, x);
+                lk[x] = c < 0 ? 0u : score_key32(s);
                 if (scores)
                     scores[prob * p.kc * p.G + x] = c < 0 ? __int_as_float(0x7fc00000) : s;
             }
@@ -360,12 +289,12 @@ __global__ void __launch_bounds__(256) route_groups_kernel(
         for (int x = ncand + threadIdx.x; x < p.kc * p.G; x += blockDim.x)
             scores[prob * p.kc * p.G + x] = __int_as_float(0x7fc00000);
     cluster.sync();
-    if (r != 0) return;
+    if (r != 0 || warp != 0) return;
     const int G = p.G;
-    unsigned* flags = reinterpret_cast<unsigned*>(keys + next_pow2(p.kc * p.G));
-    const int kept = cta_topk_compact(keys, flags, ncand, p.kg, p.kg, sel_groups + prob * p.kg,
-                                      [&](int x) { return s_chunk[x / G] * G + x % G; });
-    if (threadIdx.x == 0) n_sel_groups[prob] = kept;
+    const int kept = warp_radix_topk(keys, ncand, p.kg, p.kg, sel_groups + prob * p.kg,
+                                     keys + p.kc * p.G,
+                                     [&](int x) { return s_chunk[x / G] * G + x % G; });
+    if (lane == 0) n_sel_groups[prob] = kept;
 }
 
 // Raise a kernel's dynamic shared-memory limit once per process (a driver
@@ -434,14 +363,13 @@ cudaError_t launch_route_chunks(const Params& p, const void* q_rot, float* qbar,
         return launch_route_chunks_tiled(p, qbar, chunk_sum, sel, n_sel, scores, st);
     int fuse = route_chunks_fuses_qbar(p) ? 1 : 0;
     const int cl = chunk_cluster(p);
-    size_t smem = (size_t)next_pow2(p.nC) * sizeof(unsigned long long) +
-                  (size_t)((p.nC + 31) / 32) * sizeof(unsigned);
+    size_t smem = ((size_t)p.nC + 256) * sizeof(uint32_t);
     dim3 grid(cl, p.nQC, p.B * p.Hkv);
     Params pp = p;
     void* args[] = {&pp, (void*)&qbar, (void*)&q_rot, &fuse, (void*)&chunk_sum, &sel, &n_sel, &scores};
     const void* fn = p.d == 128 ? (const void*)route_chunks_kernel<4>
                                 : (const void*)route_chunks_kernel<2>;
-    cudaError_t e = allow_smem(fn, kMaxChunks * (sizeof(unsigned long long) + 1));
+    cudaError_t e = allow_smem(fn, (kMaxChunks + 256) * sizeof(uint32_t));
     if (e != cudaSuccess) return e;
     return launch_cluster(fn, grid, 256, smem, cl, st, args);
 }
@@ -453,15 +381,14 @@ cudaError_t launch_route_groups(const Params& p, const float* qbar, const float*
     if (p.nQC == 0) return cudaSuccess;
     const int64_t problems = (int64_t)p.B * p.Hkv * p.nQC;
     const int cl = problems >= 1024 ? 1 : 4;
-    size_t smem = (size_t)next_pow2(p.kc * p.G) * sizeof(unsigned long long) +
-                  (size_t)((p.kc * p.G + 31) / 32) * sizeof(unsigned);
+    size_t smem = ((size_t)p.kc * p.G + 256) * sizeof(uint32_t);
     dim3 grid(cl, p.nQC, p.B * p.Hkv);
     Params pp = p;
     void* args[] = {&pp, (void*)&qbar, (void*)&group_sum, (void*)&sel_chunks,
                     (void*)&n_sel_chunks, &sel_groups, &n_sel_groups, &scores};
     const void* fn = p.d == 128 ? (const void*)route_groups_kernel<4>
                                 : (const void*)route_groups_kernel<2>;
-    cudaError_t e = allow_smem(fn, 8192 * (sizeof(unsigned long long) + 1));
+    cudaError_t e = allow_smem(fn, (8192 + 256) * sizeof(uint32_t));
     if (e != cudaSuccess) return e;
     return launch_cluster(fn, grid, 256, smem, cl, st, args);
 }

@@ -10,10 +10,11 @@
 // memory once for all of them: a register-blocked fp32 product (each thread
 // 4 query chunks x 4 table rows) writes the 16 score rows to shared memory.
 // Each warp then selects the top-k of its query chunks with a 4-pass radix
-// select (8-bit digits of the order-preserving score key, warp-private
-// histograms) and writes the winners in ascending chunk order. Ties on the
-// threshold score go to the lower chunk index; NaN ranks last.
+// select over the order-preserving score keys (hga_topk.cuh) and writes the
+// winners in ascending chunk order. Ties go to the lower chunk index; NaN
+// ranks last.
 #include "hga_kernels.h"
+#include "hga_topk.cuh"
 
 namespace hga {
 
@@ -23,15 +24,6 @@ constexpr int kQB = 16;          // query chunks per CTA
 constexpr int kCT = 256;         // table rows per tile
 constexpr int kKS = 32;          // dims per k-slice
 constexpr int kThreads = 256;
-
-// Order-preserving 32-bit key of a score: larger score -> larger key; -0 == +0;
-// NaN -> 0 (below every number).
-__device__ __forceinline__ uint32_t score_key(float s) {
-    if (s != s) return 0u;
-    s += 0.0f;
-    const uint32_t b = __float_as_uint(s);
-    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) route_chunks_tiled_kernel(
@@ -107,97 +99,20 @@ __global__ void __launch_bounds__(kThreads) route_chunks_tiled_kernel(
     for (int q = warp; q < nq; q += kThreads / 32) {
         const int jj = jj0 + q, j = p.j0 + jj;
         const int64_t prob = bh * p.nQC + jj;
-        const float* srow = sc + q * ncp;
-        auto cand = [&](int c) { return c < j && !is_forced(p, j, c); };
-        // candidates count
-        int n_cand = 0;
-        for (int c0 = 0; c0 < j; c0 += 32) {
-            const int c = c0 + lane;
-            n_cand += __popc(__ballot_sync(0xffffffffu, c < j && cand(c)));
-        }
-        const int k = p.kc < n_cand ? p.kc : n_cand;
-        uint32_t prefix = 0u, mask = 0u;
-        int need = k;
-        if (k < n_cand) {
-            for (int shift = 24; shift >= 0; shift -= 8) {
-                for (int b = lane; b < 256; b += 32) h[b] = 0u;
-                __syncwarp();
-                for (int c = lane; c < j; c += 32) {
-                    if (!cand(c)) continue;
-                    const uint32_t key = score_key(srow[c]);
-                    if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
-                }
-                __syncwarp();
-                // digits in descending order: lane L owns digits 255-8L .. 248-8L
-                uint32_t cnt[8];
-                uint32_t lsum = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    cnt[i] = h[255 - 8 * lane - i];
-                    lsum += cnt[i];
-                }
-                uint32_t incl = lsum;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
-                    if (lane >= off) incl += v;
-                }
-                const uint32_t excl = incl - lsum;
-                // the lane whose range holds the need-th largest
-                const bool here = excl < (uint32_t)need && (uint32_t)need <= incl;
-                const unsigned hm = __ballot_sync(0xffffffffu, here);
-                const int owner = hm ? __ffs(hm) - 1 : 0;
-                uint32_t digit = 0u, above = 0u;
-                if (lane == owner) {
-                    uint32_t run = excl;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        if (run + cnt[i] >= (uint32_t)need) {
-                            digit = 255u - 8u * lane - i;
-                            above = run;
-                            break;
-                        }
-                        run += cnt[i];
-                    }
-                }
-                digit = __shfl_sync(0xffffffffu, digit, owner);
-                above = __shfl_sync(0xffffffffu, above, owner);
-                need -= (int)above;
-                prefix |= digit << shift;
-                mask |= 255u << shift;
-                __syncwarp();
-            }
-        }
-        // keys > prefix are in; among keys == prefix the first `need` (by index) are in
-        int base = 0, ties = 0;
-        int32_t* out = sel + prob * p.kc;
-        for (int c0 = 0; c0 < j; c0 += 32) {
-            const int c = c0 + lane;
-            bool is = false, tie = false;
-            if (c < j && cand(c)) {
-                if (k >= n_cand) {
-                    is = true;
-                } else {
-                    const uint32_t key = score_key(srow[c]);
-                    is = key > prefix;
-                    tie = key == prefix;
-                }
-            }
-            const unsigned tm = __ballot_sync(0xffffffffu, tie);
-            const int trank = ties + __popc(tm & ((1u << lane) - 1u));
-            is = is || (tie && trank < need);
-            ties += __popc(tm);
-            const unsigned m = __ballot_sync(0xffffffffu, is);
-            if (is) out[base + __popc(m & ((1u << lane) - 1u))] = c;
-            base += __popc(m);
-        }
-        for (int s = base + lane; s < p.kc; s += 32) out[s] = -1;
-        if (lane == 0) nsel[prob] = base;
+        float* srow = sc + q * ncp;
         if (scores_out) {
             float* so = scores_out + prob * p.nC;
             for (int c = lane; c < p.nC; c += 32)
-                so[c] = cand(c) ? srow[c] : __int_as_float(0x7fc00000);
+                so[c] = (c < j && !is_forced(p, j, c)) ? srow[c] : __int_as_float(0x7fc00000);
         }
+        // the score row becomes the key row in place (0 = not a candidate)
+        uint32_t* krow = reinterpret_cast<uint32_t*>(srow);
+        for (int c = lane; c < j; c += 32)
+            krow[c] = is_forced(p, j, c) ? 0u : score_key32(srow[c]);
+        __syncwarp();
+        const int kept = warp_radix_topk(krow, j, p.kc, p.kc, sel + prob * p.kc, h,
+                                         [](int x) { return x; });
+        if (lane == 0) nsel[prob] = kept;
     }
 }
 
