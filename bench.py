@@ -27,6 +27,15 @@ sys.path.insert(0, ROOT)
 from long_context_rope_b200 import synth  # noqa: E402
 
 METRIC = "routed attn prefill tok/s & decode µs/step at 64K; % of HBM/TC roofline"
+
+# DRAM bytes (read + write) of one prefill attention launch at 64K context,
+# from an ncu capture of attend_tc_kernel at 32K context (568.6 MB: Q and O
+# once, K/V from L2) scaled x2 (one unit per query chunk). Valid for the
+# kernel as captured; set to None when attend_tc_kernel changes until it is
+# captured again.
+TC_TRAFFIC_BYTES = 2 * 568.6e6
+TC_TRAFFIC_NOTE = ("ncu dram__bytes_read+write of attend_tc_kernel at 32K context x2 "
+                   "(profiles/attend_tc_prefill_32k_ncu.md)")
 PREFILL = "prefill_64k"
 DECODES = ("decode_16x32k", "tiered_decode_4x64k")
 
@@ -299,37 +308,58 @@ def run_decode(name, args, dist):
         pipeline.fill_windows(cfg, k_host, v_host, k_win, v_win)
         cfg_w = cfg.copy(kv_layout=hga.HGA_KV_WINDOWS)
 
-        def step():
+        def step(separate=False):
             pipeline.decode(cfg_w, q_rot, cs, gs, k_win, v_win, rb, out, gathered=gat,
-                            k_src=k_host, v_src=v_host, src_is_host=True)
-        launches = 5
-        moved = int(0)
+                            k_src=k_host, v_src=v_host, src_is_host=True, separate=separate)
+        launches, launches_sep = 3, 4  # route (one launch), gather, attend
     else:
         v = x["v"].to(dev)
 
-        def step():
-            pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out)
-        launches = 4
+        def step(separate=False):
+            pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out, separate=separate)
+        launches, launches_sep = 1, 3  # one-launch decode step
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize()
-    if hga.get_device_error() != 0:
-        raise RuntimeError(f"device error word set in {name}")
-    # a decode step is launch-latency bound: capture it once, replay the graph
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, capture_error_mode="relaxed"):
-        step()
-    eager_step = step
+    K = max(args.steps, 20)
 
-    def step():
-        graph.replay()
+    def timed(separate):
+        """Median device time of one step replayed from a CUDA graph (L2
+        flushed between steps), plus the eager median for reference."""
+        for _ in range(max(3, args.warmup)):
+            step(separate)
+        torch.cuda.synchronize()
+        if hga.get_device_error() != 0:
+            raise RuntimeError(f"device error word set in {name}")
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+            step(separate)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        if hga.get_device_error() != 0:
+            raise RuntimeError(f"device error word set in {name} (graph)")
+        ev = Events(2 * K)
+        for i in range(K):
+            flush.fill_(i & 0xff)  # write a buffer larger than L2 between steps
+            ev.rec(2 * i, st)
+            graph.replay()
+            ev.rec(2 * i + 1, st)
+        torch.cuda.synchronize()
+        times = [ev.ms(2 * i, 2 * i + 1) * 1000.0 for i in range(K)]
+        ev2 = Events(2 * 5)
+        for i in range(5):
+            flush.fill_(i & 0xff)
+            ev2.rec(2 * i, st)
+            step(separate)
+            ev2.rec(2 * i + 1, st)
+        torch.cuda.synchronize()
+        eager = float(np.median([ev2.ms(2 * i, 2 * i + 1) * 1000.0 for i in range(5)]))
+        del graph
+        return times, eager
 
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize()
-    if hga.get_device_error() != 0:
-        raise RuntimeError(f"device error word set in {name} (graph)")
+    times_sep, eager_sep = timed(True)
+    times, eager_us = timed(False)
+    us = dist.max(float(np.median(times)))
+    us_sep = dist.max(float(np.median(times_sep)))
     n_sel = rb.n_sel_groups.cpu().numpy()
     moved = int(n_sel.sum()) * 16 * w.head_dim * 2 * 2  # routed K+V bytes
     # algorithmic HBM bytes of one step (each byte the step must touch, once)
@@ -339,31 +369,13 @@ def run_decode(name, args, dist):
     group_sums = int(rb.n_sel_chunks.cpu().numpy().sum()) * w.groups_per_chunk * w.head_dim * 4
     q_o = 2 * w.batch * w.n_q_heads * w.head_dim * 2
     hbm_bytes = forced_kv + chunk_sums + group_sums + q_o + (2 * moved if w.tiered else moved)
-    K = max(args.steps, 20)
-    ev = Events(2 * K)
-    for i in range(K):
-        flush.fill_(i & 0xff)  # write a buffer larger than L2 between steps
-        ev.rec(2 * i, st)
-        step()
-        ev.rec(2 * i + 1, st)
-    torch.cuda.synchronize()
-    times = [ev.ms(2 * i, 2 * i + 1) * 1000.0 for i in range(K)]
-    us = dist.max(float(np.median(times)))
-    # the same step launched eagerly (host launch overhead included), for reference
-    ev2 = Events(2 * 5)
-    for i in range(5):
-        flush.fill_(i & 0xff)
-        ev2.rec(2 * i, st)
-        eager_step()
-        ev2.rec(2 * i + 1, st)
-    torch.cuda.synchronize()
-    eager_us = float(np.median([ev2.ms(2 * i, 2 * i + 1) * 1000.0 for i in range(5)]))
-    del graph
     return dict(workload=name, us_per_step=us, us_min=float(np.min(times)), steps=K,
                 hbm_bytes_per_step=hbm_bytes, hbm_gbs=hbm_bytes / (us * 1e-6) / 1e9,
                 hbm_frac=hbm_bytes / (us * 1e-6) / 1e9 / load_peaks()["hbm"],
                 us_per_step_eager=eager_us, cuda_graph=True,
                 launches_per_step=launches, routed_kv_bytes=moved,
+                us_per_step_separate_kernels=us_sep, us_per_step_separate_eager=eager_sep,
+                launches_per_step_separate=launches_sep,
                 host_link_gbs=(moved / (us * 1e-6) / 1e9) if w.tiered else None)
 
 
@@ -493,7 +505,10 @@ def main():
             "stage_ms": pre["stage_ms"],
             "roofline": {"kernel": "hga_attend (prefill)", "bound": "tensor",
                          "achieved": ach, "peak": peaks["tc_sustained"], "unit": "TFLOP/s",
-                         "frac": ach / peaks["tc_sustained"], "traffic": None,
+                         "frac": ach / peaks["tc_sustained"],
+                         "traffic": TC_TRAFFIC_BYTES if args.workload == "prefill_64k" else None,
+                         "traffic_note": TC_TRAFFIC_NOTE if args.workload == "prefill_64k"
+                         else None,
                          "flops_per_launch": pre["flops"],
                          "peak_note": f"bf16 sustained, {peaks['src']}"},
             "gpu_launches": pre["launches_per_step"] * args.steps,

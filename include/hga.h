@@ -148,6 +148,33 @@ hga_status hga_route_groups(const hga_config* cfg, const float* qbar, const floa
                             int32_t* sel_groups, int32_t* n_sel_groups, float* scores_out,
                             void* stream);
 
+/* Both routing levels in one call ("Kernmechanisme" item 2, Niveau 1 and 2):
+ * the same q-bar and bitwise the same selections as hga_route_chunks
+ * followed by hga_route_groups on these arguments, without the score
+ * outputs. For a one-token query span (decode) in bf16 with d = 128 and
+ * top_k_chunks <= 64 this is one launch (both levels split across a
+ * thread-block cluster); otherwise the two calls' kernels run in sequence.
+ * qbar_out [B,Hkv,nQC,d] fp32, sel_chunks / n_sel_chunks, sel_groups /
+ * n_sel_groups as for the two calls; all required. */
+hga_status hga_route(const hga_config* cfg, const void* q_rot, const float* chunk_sum,
+                     const float* group_sum, float* qbar_out, int32_t* sel_chunks,
+                     int32_t* n_sel_chunks, int32_t* sel_groups, int32_t* n_sel_groups,
+                     void* stream);
+
+/* One routed attention step over a resident cache: hga_route, then
+ * hga_attend in index mode over the full store k_cache / v_cache
+ * [B, Hkv, L, d] (cfg->kv_layout must be HGA_KV_FULL; the host tier goes
+ * through hga_route, hga_gather_kv and hga_attend). Writes q-bar, both
+ * selections (as hga_route) and out [B, q_len, Hq, d]. For a one-token query
+ * span (decode) in bf16, d = 128, gq <= 8, L % 16 == 0, top_k_chunks <= 64
+ * this is a single launch: the always-visible blocks are fetched while the
+ * routing runs; the attention result equals hga_attend's within fp32
+ * summation order. Other configurations run the separate kernels. */
+hga_status hga_decode_step(const hga_config* cfg, const void* q_rot, const float* chunk_sum,
+                           const float* group_sum, const void* k_cache, const void* v_cache,
+                           float* qbar_out, int32_t* sel_chunks, int32_t* n_sel_chunks,
+                           int32_t* sel_groups, int32_t* n_sel_groups, void* out, void* stream);
+
 /* Exact-token retrieval ("Kernmechanisme" item 4; "Geheugenarchitectuur"
  * cold tier): copy the K and V rows of every selected group into compact
  * buffers k_dst, v_dst [B, Hkv, nQC, top_k_groups * g, d]; slot s holds the

@@ -112,7 +112,7 @@ static_assert(offsetof(hga_config, rope_theta) == 48, "hga_config layout is part
 
 extern "C" {
 
-int32_t hga_version(void) { return 10000; }
+int32_t hga_version(void) { return 10100; }
 
 const char* hga_status_string(hga_status s) {
     switch (s) {
@@ -201,6 +201,88 @@ hga_status hga_route_groups(const hga_config* cfg, const float* qbar, const floa
     HGA_ATTACH_ERR(p);
     return launched(launch_route_groups(p, qbar, group_sum, sel_chunks, n_sel_chunks, sel_groups,
                                         n_sel_groups, scores_out, (cudaStream_t)stream));
+}
+
+// Shared checks of hga_route / hga_decode_step (routing outputs).
+static hga_status check_route_args(const Params& p, const void* q_rot, const float* chunk_sum,
+                                   const float* group_sum, const float* qbar_out,
+                                   const int32_t* sel_chunks, const int32_t* n_sel_chunks,
+                                   const int32_t* sel_groups, const int32_t* n_sel_groups) {
+    (void)p;
+    if (!q_rot || !chunk_sum || !group_sum || !qbar_out || !sel_chunks || !n_sel_chunks ||
+        !sel_groups || !n_sel_groups)
+        return HGA_ERR_NULL;
+    if (!aligned16(q_rot) || !aligned16(chunk_sum) || !aligned16(group_sum) ||
+        !aligned16(qbar_out) || !aligned16(sel_chunks) || !aligned16(n_sel_chunks) ||
+        !aligned16(sel_groups) || !aligned16(n_sel_groups))
+        return HGA_ERR_ALIGN;
+    return HGA_OK;
+}
+
+// The two routing levels as separate kernels.
+static hga_status route_separate(const Params& p, const void* q_rot, const float* chunk_sum,
+                                 const float* group_sum, float* qbar_out, int32_t* sel_chunks,
+                                 int32_t* n_sel_chunks, int32_t* sel_groups,
+                                 int32_t* n_sel_groups, cudaStream_t st) {
+    if (!route_chunks_fuses_qbar(p) && launch_qbar(p, q_rot, qbar_out, st) != cudaSuccess)
+        return HGA_ERR_CUDA;
+    if (launch_route_chunks(p, q_rot, qbar_out, chunk_sum, sel_chunks, n_sel_chunks, nullptr,
+                            st) != cudaSuccess)
+        return HGA_ERR_CUDA;
+    return launched(launch_route_groups(p, qbar_out, group_sum, sel_chunks, n_sel_chunks,
+                                        sel_groups, n_sel_groups, nullptr, st));
+}
+
+hga_status hga_route(const hga_config* cfg, const void* q_rot, const float* chunk_sum,
+                     const float* group_sum, float* qbar_out, int32_t* sel_chunks,
+                     int32_t* n_sel_chunks, int32_t* sel_groups, int32_t* n_sel_groups,
+                     void* stream) {
+    Params p;
+    hga_status s = make_params(cfg, &p);
+    if (s != HGA_OK) return s;
+    if (p.nQC == 0) return HGA_OK;
+    s = check_route_args(p, q_rot, chunk_sum, group_sum, qbar_out, sel_chunks, n_sel_chunks,
+                         sel_groups, n_sel_groups);
+    if (s != HGA_OK) return s;
+    HGA_ATTACH_ERR(p);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (decode_step_supports(p))
+        return launched(launch_decode_step(p, q_rot, chunk_sum, group_sum, nullptr, nullptr,
+                                           qbar_out, sel_chunks, n_sel_chunks, sel_groups,
+                                           n_sel_groups, nullptr, st));
+    return route_separate(p, q_rot, chunk_sum, group_sum, qbar_out, sel_chunks, n_sel_chunks,
+                          sel_groups, n_sel_groups, st);
+}
+
+hga_status hga_decode_step(const hga_config* cfg, const void* q_rot, const float* chunk_sum,
+                           const float* group_sum, const void* k_cache, const void* v_cache,
+                           float* qbar_out, int32_t* sel_chunks, int32_t* n_sel_chunks,
+                           int32_t* sel_groups, int32_t* n_sel_groups, void* out, void* stream) {
+    Params p;
+    hga_status s = make_params(cfg, &p);
+    if (s != HGA_OK) return s;
+    if (p.nQC == 0) return HGA_OK;
+    s = check_route_args(p, q_rot, chunk_sum, group_sum, qbar_out, sel_chunks, n_sel_chunks,
+                         sel_groups, n_sel_groups);
+    if (s != HGA_OK) return s;
+    if (!k_cache || !v_cache || !out) return HGA_ERR_NULL;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return HGA_ERR_ALIGN;
+    if (p.kv_layout != HGA_KV_FULL) return HGA_ERR_UNSUPPORTED;
+    HGA_ATTACH_ERR(p);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (decode_step_supports(p))
+        return launched(launch_decode_step(p, q_rot, chunk_sum, group_sum, k_cache, v_cache,
+                                           qbar_out, sel_chunks, n_sel_chunks, sel_groups,
+                                           n_sel_groups, out, st));
+    s = route_separate(p, q_rot, chunk_sum, group_sum, qbar_out, sel_chunks, n_sel_chunks,
+                       sel_groups, n_sel_groups, st);
+    if (s != HGA_OK) return s;
+    KvSources kv{k_cache, v_cache, nullptr, nullptr};
+    if (tc_kernel_supports(p, false))
+        return launched(launch_attend_tc(p, q_rot, kv, sel_groups, n_sel_groups, out, st));
+    if (decode_kernel_supports(p))
+        return launched(launch_attend_decode(p, q_rot, kv, sel_groups, n_sel_groups, out, st));
+    return launched(launch_attend_simt(p, q_rot, kv, sel_groups, n_sel_groups, out, st));
 }
 
 static hga_status device_view(const void* ptr, bool want_host, const void** dev_ptr) {

@@ -1,0 +1,273 @@
+// hga_decode_core.cuh -- the attention half of single-token decode, shared by
+// the split-K decode attention kernel and the fused decode step.
+//
+// "Technische Samenvatting: Hierarchical Global Attention (HGA)"
+// (gist.science), "Kernmechanisme" item 4: standard softmax over the bounded
+// exact token set. One query token, gq <= 8 query heads of one KV head; the
+// heads share every key/value load (GQA).
+//
+// A CTA streams its share of the unit's 16-row key blocks through a ring of
+// shared-memory stages (TMA tile loads, 128-byte swizzle) and eight consumer
+// warps take every 8th block: S^T[16 keys x 8 heads] = K_blk Q^T and
+// O^T[128 dims x 8 heads] += V^T P^T on warp-level bf16 MMA (m16n8k16, fp32
+// accumulate) with a per-warp online softmax in fp32. Partials (max, sum, O)
+// merge first across the warps of a CTA, then across the CTAs of the cluster
+// through distributed shared memory.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "hga_common.cuh"
+#include "hga_ptx.cuh"
+
+namespace hga {
+namespace dec {
+
+namespace cg = cooperative_groups;
+
+constexpr int kD = 128;
+constexpr int kStages = 8;                       // ring of key blocks
+constexpr int kBlkBytes = kGroupRows * kD * 2;   // 4 KiB per block per tensor
+constexpr int kConsumers = 8;                    // consumer warps
+constexpr int kThreads = (kConsumers + 1) * 32;  // + one producer warp
+constexpr int kMaxCluster = 16;
+
+struct Partial {
+    float m[8], l[8];          // per head
+    float o[8][kD];            // per head, un-normalised
+};
+
+struct Ring {
+    alignas(1024) uint8_t k[kStages][kBlkBytes];
+    alignas(1024) uint8_t v[kStages][kBlkBytes];
+};
+
+// Per-warp accumulator state of the online softmax.
+struct WarpAcc {
+    float o[8][4];
+    float m[2], l[2];
+};
+
+// Q^T as MMA B fragments: lane (g, t4) holds Q[head g][16kk + 2t4 .. +1] and
+// Q[head g][16kk + 2t4 + 8 .. +9]; heads >= gq are zero.
+__device__ __forceinline__ void load_q_frags(const Params& p, const __nv_bfloat16* q, int b, int h,
+                                             uint32_t (&qf)[8][2]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
+    const bool okh = g < p.gq;
+    const __nv_bfloat16* qr =
+        q + ((int64_t)b * p.q_len * p.Hq + (int64_t)h * p.gq + (okh ? g : 0)) * kD;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        qf[kk][0] = okh ? *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 2 * t4) : 0u;
+        qf[kk][1] = okh ? *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 2 * t4 + 8) : 0u;
+    }
+}
+
+__device__ __forceinline__ void acc_init(WarpAcc& a) {
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) a.o[mt][e] = 0.f;
+    a.m[0] = a.m[1] = -INFINITY;
+    a.l[0] = a.l[1] = 0.f;
+}
+
+// Consumer warp `warp` processes local blocks warp, warp + 8, ... < nloc of
+// the ring. blk_pos[i] is the position of block i's first token. Returns
+// false (and sets *bad) if a wait gave up.
+__device__ __forceinline__ bool consume_blocks(const Params& p, const uint32_t (&qf)[8][2],
+                                               Ring& ring, uint64_t* full, uint64_t* empty,
+                                               const int* blk_pos, int nloc, int qpos,
+                                               __nv_bfloat16 (*pt)[16], WarpAcc& acc,
+                                               int* bad) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t4 = lane & 3;
+    const float sc = 1.4426950408889634f / sqrtf((float)kD);
+    const int mq = lane >> 3;
+    const int krow = (mq & 1) * 8 + (lane & 7);      // K ldmatrix row
+    const int vkey = (mq >> 1) * 8 + (lane & 7);     // V ldmatrix (trans) row
+    for (int i = warp; i < nloc; i += kConsumers) {
+        const int s = i % kStages;
+        const bool got = __all_sync(
+            0xffffffffu, ptx::mbar_wait_bounded(&full[s], (i / kStages) & 1, p.err));
+        if (!got) {
+            if (lane == 0) {
+                raise_dev_error(p, kDevErrTimeout);
+                *bad = 1;
+            }
+            return false;
+        }
+        // S^T = K Q^T for 16 keys x 8 heads (two accumulator chains)
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sacc2[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t kb = ptx::smem_u32(ring.k[s]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const int chunk = (kk & 3) * 2 + (mq >> 1);
+            uint32_t a[4];
+            ptx::ldsm_x4(kb + (kk >> 2) * 2048 + krow * 128 + ((chunk ^ (krow & 7)) << 4), a);
+            ptx::mma_16816((kk & 1) ? sacc2 : sacc, a, qf[kk][0], qf[kk][1]);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[e] += sacc2[e];
+        // this lane holds keys g, g+8 for heads 2t4, 2t4+1
+        const int kp = blk_pos[i];
+        const bool v0 = kp + g <= qpos, v1 = kp + g + 8 <= qpos;
+        const float sv[4] = {v0 ? sacc[0] * sc : -INFINITY, v0 ? sacc[1] * sc : -INFINITY,
+                             v1 ? sacc[2] * sc : -INFINITY, v1 ? sacc[3] * sc : -INFINITY};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float mb = fmaxf(sv[hh], sv[hh + 2]);
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 4));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 8));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 16));
+            const float mn = fmaxf(acc.m[hh], mb);
+            float alpha = 1.f, p0 = 0.f, p1 = 0.f;
+            if (mn != -INFINITY) {
+                alpha = acc.m[hh] == -INFINITY ? 0.f : ptx::ex2_approx(acc.m[hh] - mn);
+                p0 = ptx::ex2_approx(sv[hh] - mn);
+                p1 = ptx::ex2_approx(sv[hh + 2] - mn);
+            }
+            acc.m[hh] = mn;
+            // bf16 weights; the running sum uses the same rounded values
+            const __nv_bfloat16 b0 = __float2bfloat16_rn(p0);
+            const __nv_bfloat16 b1 = __float2bfloat16_rn(p1);
+            acc.l[hh] = acc.l[hh] * alpha + __bfloat162float(b0) + __bfloat162float(b1);
+            pt[2 * t4 + hh][g] = b0;
+            pt[2 * t4 + hh][g + 8] = b1;
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                acc.o[mt][hh] *= alpha;
+                acc.o[mt][hh + 2] *= alpha;
+            }
+        }
+        __syncwarp();
+        const uint32_t pb0 = *reinterpret_cast<const uint32_t*>(&pt[g][2 * t4]);
+        const uint32_t pb1 = *reinterpret_cast<const uint32_t*>(&pt[g][2 * t4 + 8]);
+        // O^T[16 dims x 8 heads] += V^T P^T, eight 16-dim tiles
+        const uint32_t vb = ptx::smem_u32(ring.v[s]);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            const int chunk = (mt & 3) * 2 + (mq & 1);
+            uint32_t a[4];
+            ptx::ldsm_x4_trans(vb + (mt >> 2) * 2048 + vkey * 128 + ((chunk ^ (vkey & 7)) << 4),
+                               a);
+            ptx::mma_16816(acc.o[mt], a, pb0, pb1);
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&empty[s]);
+    }
+    return true;
+}
+
+// Consumer warp writes its partial (row max, row sum, O) to wp.
+__device__ __forceinline__ void store_warp_partial(const WarpAcc& acc, Partial& wp) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
+    float lsum[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        float v = acc.l[hh];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        lsum[hh] = v;
+    }
+    if (g == 0) {
+        wp.m[2 * t4] = acc.m[0];
+        wp.m[2 * t4 + 1] = acc.m[1];
+        wp.l[2 * t4] = lsum[0];
+        wp.l[2 * t4 + 1] = lsum[1];
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+        const int d0 = mt * 16 + g;
+        wp.o[2 * t4][d0] = acc.o[mt][0];
+        wp.o[2 * t4 + 1][d0] = acc.o[mt][1];
+        wp.o[2 * t4][d0 + 8] = acc.o[mt][2];
+        wp.o[2 * t4 + 1][d0 + 8] = acc.o[mt][3];
+    }
+}
+
+// All threads of the CTA: merge the 8 warp partials into cta.
+__device__ __forceinline__ void merge_warps(const Partial* warp_part, Partial& cta) {
+    for (int x = threadIdx.x; x < 8 * kD; x += blockDim.x) {
+        const int n = x / kD, d = x % kD;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, warp_part[w].m[n]);
+        float num = 0.f, den = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kConsumers; ++w) {
+                const float mw = warp_part[w].m[n];
+                if (mw == -INFINITY) continue;
+                const float wgt = ptx::ex2_approx(mw - M);
+                num = fmaf(wgt, warp_part[w].o[n][d], num);
+                den = fmaf(wgt, warp_part[w].l[n], den);
+            }
+        }
+        cta.o[n][d] = num;
+        if (d == 0) {
+            cta.m[n] = M;
+            cta.l[n] = den;
+        }
+    }
+}
+
+// After a cluster barrier: CTA r merges the CL CTA partials of heads
+// r, r + CL, ... and writes the normalised output rows (bf16).
+__device__ __forceinline__ void merge_cluster_and_store(const Params& p, cg::cluster_group& cluster,
+                                                        Partial& cta_part, int b, int h,
+                                                        __nv_bfloat16* out) {
+    const int CL = (int)cluster.num_blocks();
+    const int r = (int)cluster.block_rank();
+    const int tid = threadIdx.x;
+    for (int n = r; n < p.gq; n += CL) {
+        if (tid < kD) {
+            float mc[kMaxCluster], lc[kMaxCluster], oc[kMaxCluster];
+#pragma unroll
+            for (int c = 0; c < kMaxCluster; ++c) {
+                if (c < CL) {
+                    const Partial* rp = cluster.map_shared_rank(&cta_part, c);
+                    mc[c] = rp->m[n];
+                    lc[c] = rp->l[n];
+                    oc[c] = rp->o[n][tid];
+                } else {
+                    mc[c] = -INFINITY;
+                    lc[c] = 0.f;
+                    oc[c] = 0.f;
+                }
+            }
+            float M = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kMaxCluster; ++c) M = fmaxf(M, mc[c]);
+            float num = 0.f, den = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int c = 0; c < kMaxCluster; ++c) {
+                    if (mc[c] == -INFINITY) continue;
+                    const float wgt = ptx::ex2_approx(mc[c] - M);
+                    num = fmaf(wgt, oc[c], num);
+                    den = fmaf(wgt, lc[c], den);
+                }
+            }
+            const float o = den > 0.f ? num / den : 0.f;
+            out[((int64_t)b * p.q_len * p.Hq + (int64_t)h * p.gq + n) * kD + tid] =
+                __float2bfloat16_rn(o);
+        }
+    }
+}
+
+// Issue the TMA loads of one 16-row block (K and V, two 64-column halves
+// each) into ring stage s.
+__device__ __forceinline__ void issue_block(Ring& ring, uint64_t* full, int s,
+                                            const CUtensorMap* mk, const CUtensorMap* mv, int row,
+                                            int outer) {
+    ptx::mbar_arrive_expect_tx(&full[s], 2 * kBlkBytes);
+    for (int hf = 0; hf < 2; ++hf) {
+        ptx::tma_load_3d(ring.k[s] + hf * 2048, mk, hf * 64, row, outer, &full[s]);
+        ptx::tma_load_3d(ring.v[s] + hf * 2048, mv, hf * 64, row, outer, &full[s]);
+    }
+}
+
+}  // namespace dec
+}  // namespace hga

@@ -75,4 +75,15 @@ cudaError_t launch_attend_decode(const Params& p, const void* q_rot, const KvSou
                                  const int32_t* sel_groups, const int32_t* n_sel_groups,
                                  void* out, cudaStream_t st);
 
+// One-launch decode step (q-bar, both routing levels, attention over the
+// full resident cache): bf16, d = 128, one query token, gq <= 8, L % 16 == 0,
+// top_k_chunks <= 64, top_k_groups <= 512, and routing tables that fit one
+// cluster's shared memory. With out == nullptr it stops after routing.
+bool decode_step_supports(const Params& p);
+cudaError_t launch_decode_step(const Params& p, const void* q_rot, const float* chunk_sum,
+                               const float* group_sum, const void* k_cache, const void* v_cache,
+                               float* qbar, int32_t* sel_chunks, int32_t* n_sel_chunks,
+                               int32_t* sel_groups, int32_t* n_sel_groups, void* out,
+                               cudaStream_t st);
+
 }  // namespace hga

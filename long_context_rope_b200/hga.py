@@ -81,6 +81,8 @@ def _load():
         "hga_route_groups": [C, P, P, P, P, P, P, P, P],
         "hga_gather_kv": [C, P, P, I32, P, P, P, P, P],
         "hga_attend": [C, P, P, P, P, P, P, P, P, P],
+        "hga_route": [C, P, P, P, P, P, P, P, P, P],
+        "hga_decode_step": [C, P, P, P, P, P, P, P, P, P, P, P, P],
         "hga_get_device_error": [P, ctypes.POINTER(I32)],
     }
     for name, args in sig.items():
@@ -198,6 +200,43 @@ def route_groups(cfg: HgaConfig, qbar, group_sum, sel_chunks, n_sel_chunks, sel_
         _ptr(n_sel_groups, "n_sel_groups", torch.int32, (B, H, nQC)),
         _ptr(scores, "scores", torch.float32, (B, H, nQC, cfg.top_k_chunks * G), nullable=True),
         _stream(stream)), "hga_route_groups")
+
+
+def _route_ptrs(cfg: HgaConfig, q_rot, chunk_sum, group_sum, qbar, sel_chunks, n_sel_chunks,
+                sel_groups, n_sel_groups):
+    B, H, d, nQC, G = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.n_qchunks, cfg.groups_per_chunk
+    return [
+        _ptr(q_rot, "q_rot", cfg.torch_dtype(), (B, cfg.q_len, cfg.n_q_heads, d)),
+        _ptr(chunk_sum, "chunk_sum", torch.float32, (B, H, cfg.n_chunks, d)),
+        _ptr(group_sum, "group_sum", torch.float32, (B, H, cfg.n_chunks * G, d)),
+        _ptr(qbar, "qbar", torch.float32, (B, H, nQC, d)),
+        _ptr(sel_chunks, "sel_chunks", torch.int32, (B, H, nQC, cfg.top_k_chunks)),
+        _ptr(n_sel_chunks, "n_sel_chunks", torch.int32, (B, H, nQC)),
+        _ptr(sel_groups, "sel_groups", torch.int32, (B, H, nQC, cfg.top_k_groups)),
+        _ptr(n_sel_groups, "n_sel_groups", torch.int32, (B, H, nQC)),
+    ]
+
+
+def route(cfg: HgaConfig, q_rot, chunk_sum, group_sum, qbar, sel_chunks, n_sel_chunks, sel_groups,
+          n_sel_groups, stream=None) -> None:
+    """Both routing levels (one launch for a one-token span)."""
+    args = _route_ptrs(cfg, q_rot, chunk_sum, group_sum, qbar, sel_chunks, n_sel_chunks,
+                       sel_groups, n_sel_groups)
+    _check(_lib.hga_route(ctypes.byref(cfg), *args, _stream(stream)), "hga_route")
+
+
+def decode_step(cfg: HgaConfig, q_rot, chunk_sum, group_sum, k_cache, v_cache, qbar, sel_chunks,
+                n_sel_chunks, sel_groups, n_sel_groups, out, stream=None) -> None:
+    """Routing plus attention over the full resident cache (one launch for decode)."""
+    B, H, L, d = cfg.batch, cfg.n_kv_heads, cfg.seq_len, cfg.head_dim
+    dt = cfg.torch_dtype()
+    r = _route_ptrs(cfg, q_rot, chunk_sum, group_sum, qbar, sel_chunks, n_sel_chunks, sel_groups,
+                    n_sel_groups)
+    _check(_lib.hga_decode_step(
+        ctypes.byref(cfg), r[0], r[1], r[2],
+        _ptr(k_cache, "k_cache", dt, (B, H, L, d)), _ptr(v_cache, "v_cache", dt, (B, H, L, d)),
+        *r[3:], _ptr(out, "out", dt, (B, cfg.q_len, cfg.n_q_heads, d)), _stream(stream)),
+        "hga_decode_step")
 
 
 def gather_kv(cfg: HgaConfig, k_src, v_src, src_is_host: bool, sel_groups, n_sel_groups, k_dst,

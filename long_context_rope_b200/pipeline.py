@@ -71,11 +71,19 @@ def summaries(cfg: hga.HgaConfig, k_raw, cs, gs, k_rot=None, stream=None):
     hga.build_summaries(cfg, k_raw, cs, gs, k_rot, 0, cfg.n_chunks, stream)
 
 
-def route(cfg: hga.HgaConfig, q_rot, cs, gs, rb: RouteBuffers, stream=None):
-    hga.route_chunks(cfg, q_rot, cs, rb.qbar, rb.sel_chunks, rb.n_sel_chunks, rb.chunk_scores,
-                     stream)
-    hga.route_groups(cfg, rb.qbar, gs, rb.sel_chunks, rb.n_sel_chunks, rb.sel_groups,
-                     rb.n_sel_groups, rb.group_scores, stream)
+def route(cfg: hga.HgaConfig, q_rot, cs, gs, rb: RouteBuffers, stream=None,
+          separate: bool = False):
+    """Both routing levels. With score buffers (or separate=True) the two
+    levels run as their own calls, which also write the scores; otherwise
+    one hga_route call (a single launch for decode)."""
+    if separate or rb.chunk_scores is not None or rb.group_scores is not None:
+        hga.route_chunks(cfg, q_rot, cs, rb.qbar, rb.sel_chunks, rb.n_sel_chunks,
+                         rb.chunk_scores, stream)
+        hga.route_groups(cfg, rb.qbar, gs, rb.sel_chunks, rb.n_sel_chunks, rb.sel_groups,
+                         rb.n_sel_groups, rb.group_scores, stream)
+    else:
+        hga.route(cfg, q_rot, cs, gs, rb.qbar, rb.sel_chunks, rb.n_sel_chunks, rb.sel_groups,
+                  rb.n_sel_groups, stream)
 
 
 def prefill(cfg: hga.HgaConfig, k_raw, v, q_rot, cs, gs, k_rot, rb: RouteBuffers, out,
@@ -87,10 +95,17 @@ def prefill(cfg: hga.HgaConfig, k_raw, v, q_rot, cs, gs, k_rot, rb: RouteBuffers
 
 
 def decode(cfg: hga.HgaConfig, q_rot, cs, gs, k_res, v_res, rb: RouteBuffers, out,
-           gathered=None, k_src=None, v_src=None, src_is_host=False, stream=None):
+           gathered=None, k_src=None, v_src=None, src_is_host=False, stream=None,
+           separate: bool = False):
     """One decode step: routing, optional gather into `gathered` (k, v) from
-    k_src/v_src, attention (forced chunks from k_res/v_res)."""
-    route(cfg, q_rot, cs, gs, rb, stream)
+    k_src/v_src, attention (forced chunks from k_res/v_res). Without a
+    gather (full resident cache) this is one hga_decode_step call unless
+    separate=True (routing and attention as their own calls)."""
+    if gathered is None and not separate and rb.chunk_scores is None and rb.group_scores is None:
+        hga.decode_step(cfg, q_rot, cs, gs, k_res, v_res, rb.qbar, rb.sel_chunks,
+                        rb.n_sel_chunks, rb.sel_groups, rb.n_sel_groups, out, stream)
+        return
+    route(cfg, q_rot, cs, gs, rb, stream, separate=separate)
     if gathered is not None:
         hga.gather_kv(cfg, k_src, v_src, src_is_host, rb.sel_groups, rb.n_sel_groups,
                       gathered[0], gathered[1], stream)

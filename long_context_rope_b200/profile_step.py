@@ -2,13 +2,20 @@
 
   python -m long_context_rope_b200.profile_step --workload prefill_64k --steps 2
   python -m long_context_rope_b200.profile_step --workload decode_16x32k --steps 2
+  python -m long_context_rope_b200.profile_step --workload prefill_64k --seq-len 32768
+
+--seq-len / --batch shrink a workload (same heads and routing) for captures
+that replay each launch many times.
 
 Setup (input draw, query rotation, and for decode the summaries/cache build)
-happens before the steps; each prefill step is summaries -> route_chunks ->
-route_groups -> attend, each decode step route_chunks -> route_groups ->
-[gather] -> attend. Kernel names: summaries_kernel, qbar_kernel,
-route_chunks_kernel, route_groups_kernel, attend_tc_kernel /
-attend_decode_kernel / attend_simt_kernel, gather_*_kernel.
+happens before the steps; each prefill step is summaries -> q-bar ->
+route_chunks -> route_groups -> attend; a decode step over the resident
+cache is one decode_step_kernel launch (--separate: route_chunks ->
+route_groups -> attend), a tiered decode step decode_step_kernel (routing
+only) -> gather -> attend. Kernel names: summaries_kernel, qbar_kernel,
+route_chunks_tiled_kernel / route_chunks_kernel, route_groups_kernel,
+attend_tc_kernel / attend_decode_kernel / attend_simt_kernel,
+decode_step_kernel, gather_*_kernel.
 """
 from __future__ import annotations
 
@@ -30,8 +37,16 @@ def main():
     ap.add_argument("--workload", default="prefill_64k")
     ap.add_argument("--steps", type=int, default=2)
     ap.add_argument("--gathered", action="store_true", help="decode: gather, then attend")
+    ap.add_argument("--separate", action="store_true",
+                    help="decode: routing levels and attention as separate launches")
+    ap.add_argument("--seq-len", type=int, default=None, help="override the context length")
+    ap.add_argument("--batch", type=int, default=None, help="override the batch")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
+    if args.seq_len is not None:
+        w = w.replace(seq_len=args.seq_len)
+    if args.batch is not None:
+        w = w.replace(batch=args.batch)
     cfg = hga.config_from(w)
     x = synth.draw(w, seed=0)
     k_raw = x["k_raw"].cuda()
@@ -61,13 +76,14 @@ def main():
             gat = pipeline.alloc_gathered(cfg)
             for _ in range(args.steps):
                 pipeline.decode(cfg_w, q_rot, cs, gs, k_win, v_win, rb, out, gathered=gat,
-                                k_src=k_host, v_src=v_host, src_is_host=True)
+                                k_src=k_host, v_src=v_host, src_is_host=True,
+                                separate=args.separate)
         else:
             v = x["v"].cuda()
             gat = pipeline.alloc_gathered(cfg) if args.gathered else None
             for _ in range(args.steps):
                 pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out, gathered=gat,
-                                k_src=k_rot, v_src=v)
+                                k_src=k_rot, v_src=v, separate=args.separate)
     torch.cuda.synchronize()
     err = hga.get_device_error()
     print(f"{args.workload}: {args.steps} steps done, device error word {err}")

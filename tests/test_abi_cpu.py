@@ -72,3 +72,12 @@ def test_host_validation_without_gpu(hga):
     assert L.hga_gather_kv(by(_cfg(hga)), P, P, 0, P, P, None, P, None) == -1
     assert L.hga_apply_rope(by(_cfg(hga)), P, P, 1, 4, 0, 0, None) == -2
     assert L.hga_apply_rope(by(_cfg(hga)), P, P, 0, 4, 1, 0, None) == 0  # nothing to do
+    # hga_route / hga_decode_step: required outputs, alignment, layout
+    assert L.hga_route(by(_cfg(hga)), P, P, P, None, P, P, P, P, None) == -1
+    assert L.hga_route(by(_cfg(hga)), P, P, P, P, P, P, P + 4, P, None) == -3
+    assert L.hga_decode_step(by(_cfg(hga)), P, P, P, P, P, P, P, P, P, P, None, None) == -1
+    assert L.hga_decode_step(by(_cfg(hga)), P, P, P, P, P + 2, P, P, P, P, P, P, None) == -3
+    assert L.hga_decode_step(by(_cfg(hga, kv_layout=1)), P, P, P, P, P, P, P, P, P, P, P,
+                             None) == -8
+    assert L.hga_decode_step(by(_cfg(hga, q_len=0)), P, P, P, P, P, P, P, P, P, P, P,
+                             None) == 0  # empty span

@@ -1,0 +1,181 @@
+"""GPU parity of the one-launch decode step (hga_decode_step) and of the
+two-level hga_route.
+
+Two bars:
+  * against the separate calls (hga_route_chunks, hga_route_groups,
+    hga_attend) on the same device inputs: q-bar and both selections
+    bitwise identical (same fp32 dot products, exact top-k on both sides);
+    outputs within 1e-2 (the two paths split the fp32 softmax sums
+    differently, then round to bf16);
+  * against the CPU oracle (where the oracle runs in seconds): selections
+    identical up to the near-tie exemption, outputs within the bf16
+    tolerance on the units whose routing agrees.
+The configurations cover the benchmark shape, contexts with no routing
+candidates or fewer candidates than top_k_chunks, a ragged current chunk,
+cluster sizes from 1 to 16, gq < 8, G = 8, and the largest top_k_chunks the
+one-launch path takes (64).
+"""
+import numpy as np
+import pytest
+import torch
+
+from long_context_rope_b200 import synth
+from oracle import hga_oracle as O
+from parity_util import OUT_TOL, assert_close, compare_selections
+
+pytestmark = pytest.mark.gpu
+
+BASE = synth.WORKLOADS["decode_16x32k"]
+
+VARIANTS = {
+    "few_candidates_2k": dict(batch=2, seq_len=2048),
+    "one_candidate": dict(batch=3, seq_len=64 * 5),
+    "no_candidate": dict(batch=2, seq_len=64),
+    "ragged_current_chunk": dict(batch=2, seq_len=64 * 200 + 48),
+    "cluster16_b1": dict(batch=1, seq_len=16384),
+    "cluster1_b40": dict(batch=40, seq_len=4096),
+    "gq2_kc64": dict(batch=2, seq_len=8192, n_q_heads=8, n_kv_heads=4, top_k_chunks=64,
+                     top_k_groups=200, n_sink=3, n_local=4),
+    "g8_c128": dict(batch=2, seq_len=16384, chunk_size=128, groups_per_chunk=8,
+                    top_k_chunks=16, top_k_groups=100),
+}
+ORACLE_VARIANTS = ["few_candidates_2k", "ragged_current_chunk", "gq2_kc64", "one_candidate"]
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy() if t.dtype != torch.int32 else t.cpu().numpy()
+
+
+def _setup(w, x, r=None):
+    """GPU summaries from the raw keys; the query and the cache are the GPU's
+    own rotations, or the oracle's bf16 ones when `r` is given."""
+    from long_context_rope_b200 import hga, pipeline
+    cfg = hga.config_from(w)
+    k_raw = x["k_raw"].cuda()
+    cs, gs = pipeline.alloc_summaries(cfg)
+    k_rot = torch.empty_like(k_raw)
+    pipeline.summaries(cfg, k_raw, cs, gs, k_rot)
+    del k_raw
+    q_rot = pipeline.rotate_queries(cfg, x["q_raw"].cuda())
+    if r is not None:
+        k_rot = torch.from_numpy(np.ascontiguousarray(r["k_rot"])).to(torch.bfloat16).cuda()
+        q_rot = torch.from_numpy(np.ascontiguousarray(r["q_rot"])).to(torch.bfloat16).cuda()
+    return cfg, cs, gs, k_rot, q_rot
+
+
+def _run_both(w, x, r=None):
+    from long_context_rope_b200 import hga, pipeline
+    cfg, cs, gs, k_rot, q_rot = _setup(w, x, r)
+    v = x["v"].cuda()
+    rb_s = pipeline.alloc_route(cfg)
+    out_s = torch.full_like(q_rot, float("nan"))
+    pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb_s, out_s, separate=True)
+    rb_f = pipeline.alloc_route(cfg)
+    for t in (rb_f.sel_chunks, rb_f.sel_groups, rb_f.n_sel_chunks, rb_f.n_sel_groups):
+        t.fill_(-7)
+    out_f = torch.full_like(q_rot, float("nan"))
+    pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb_f, out_f)
+    rb_r = pipeline.alloc_route(cfg)
+    pipeline.route(cfg, q_rot, cs, gs, rb_r)
+    torch.cuda.synchronize()
+    assert hga.get_device_error() == 0
+    for name in ("qbar", "sel_chunks", "n_sel_chunks", "sel_groups", "n_sel_groups"):
+        a, b, c = getattr(rb_s, name), getattr(rb_f, name), getattr(rb_r, name)
+        assert torch.equal(a, b), f"decode step {name} differs from the separate calls"
+        assert torch.equal(a, c), f"hga_route {name} differs from the separate calls"
+    assert torch.isfinite(out_f.float()).all()
+    diff = (out_f.float() - out_s.float()).abs().max().item()
+    assert diff <= 1e-2, f"decode step vs separate calls: max abs diff {diff}"
+    return rb_f, out_f, diff
+
+
+def _oracle_compare(w, r, rb, out):
+    kc, kg, G = w.top_k_chunks, w.top_k_groups, w.groups_per_chunk
+    assert_close("qbar", _np(rb.qbar), r["qbar"], atol=2e-5, rtol=2e-5)
+    rsc = r["chunk_scores"].reshape(-1, r["chunk_scores"].shape[-1])
+    same_c = compare_selections("chunks", _np(rb.sel_chunks), _np(rb.n_sel_chunks),
+                                r["sel_chunks"], r["n_sel_chunks"], lambda p, x: rsc[p, x])
+    rgs = r["group_scores"].reshape(-1, r["group_scores"].shape[-1])
+    rsel_c = r["sel_chunks"].reshape(-1, kc)
+    idx = np.flatnonzero(same_c)
+
+    def ref_group_score(p, gi):
+        pos = list(rsel_c[p]).index(gi // G) * G + gi % G
+        return rgs[p, pos]
+
+    gsg = _np(rb.sel_groups).reshape(-1, kg)[idx]
+    gng = _np(rb.n_sel_groups).reshape(-1)[idx]
+    same_g = compare_selections("groups", gsg, gng, r["sel_groups"].reshape(-1, kg)[idx],
+                                r["n_sel_groups"].reshape(-1)[idx],
+                                lambda p, x: ref_group_score(idx[p], x))
+    same = np.zeros_like(same_c)
+    same[idx[same_g]] = True
+    assert same.mean() >= 0.99, same.mean()
+    gq = w.n_q_heads // w.n_kv_heads
+    g_out = _np(out)
+    worst = 0.0
+    for b in range(w.batch):
+        for h in range(w.n_kv_heads):
+            if not same[b * w.n_kv_heads + h]:
+                continue
+            gg = g_out[b, 0, h * gq:(h + 1) * gq]
+            rr = r["out"][b, 0, h * gq:(h + 1) * gq]
+            worst = max(worst, float(np.abs(gg - rr).max()))
+    assert worst <= OUT_TOL[w.dtype], worst
+    return worst
+
+
+def test_decode_step_benchmark_shape_vs_oracle():
+    w = BASE
+    x = synth.draw(w, seed=4)
+    r = O.pipeline(w, x)
+    rb, out, diff = _run_both(w, x, r)
+    worst = _oracle_compare(w, r, rb, out)
+    print(f"decode_16x32k one-launch step: vs oracle {worst:.3e}, vs separate calls {diff:.3e}")
+
+
+@pytest.mark.parametrize("name", sorted(VARIANTS))
+def test_decode_step_variants(name):
+    w = BASE.replace(name=name, **VARIANTS[name])
+    x = synth.draw(w, seed=5)
+    r = O.pipeline(w, x) if name in ORACLE_VARIANTS else None
+    rb, out, diff = _run_both(w, x, r)
+    msg = f"{name}: vs separate calls {diff:.3e}"
+    if r is not None:
+        msg += f", vs oracle {_oracle_compare(w, r, rb, out):.3e}"
+    print(msg)
+
+
+def test_decode_step_repeat_and_prefill_route():
+    """Two steps in a row give identical results; hga_route on a prefill span
+    (separate kernels inside) equals the two routing calls."""
+    from long_context_rope_b200 import hga, pipeline
+    w = BASE.replace(name="repeat", batch=4, seq_len=8192)
+    x = synth.draw(w, seed=6)
+    cfg, cs, gs, k_rot, q_rot = _setup(w, x)
+    v = x["v"].cuda()
+    res = []
+    for _ in range(2):
+        rb = pipeline.alloc_route(cfg)
+        out = torch.empty_like(q_rot)
+        pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out)
+        res.append((rb, out))
+    torch.cuda.synchronize()
+    assert torch.equal(res[0][1], res[1][1])
+    assert torch.equal(res[0][0].sel_groups, res[1][0].sel_groups)
+
+    wp = synth.WORKLOADS["prefill_4k"]
+    xp = synth.draw(wp, seed=1)
+    cfgp = hga.config_from(wp)
+    k_raw = xp["k_raw"].cuda()
+    csp, gsp = pipeline.alloc_summaries(cfgp)
+    pipeline.summaries(cfgp, k_raw, csp, gsp, None)
+    qp = pipeline.rotate_queries(cfgp, xp["q_raw"].cuda())
+    rb1 = pipeline.alloc_route(cfgp)
+    pipeline.route(cfgp, qp, csp, gsp, rb1, separate=True)
+    rb2 = pipeline.alloc_route(cfgp)
+    pipeline.route(cfgp, qp, csp, gsp, rb2)
+    torch.cuda.synchronize()
+    assert hga.get_device_error() == 0
+    for name in ("qbar", "sel_chunks", "n_sel_chunks", "sel_groups", "n_sel_groups"):
+        assert torch.equal(getattr(rb1, name), getattr(rb2, name)), name
