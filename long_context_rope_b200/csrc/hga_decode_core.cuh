@@ -32,9 +32,13 @@ constexpr int kConsumers = 8;                    // consumer warps
 constexpr int kThreads = (kConsumers + 1) * 32;  // + one producer warp
 constexpr int kMaxCluster = 16;
 
+// Row stride of a partial's O: 132 floats, so the per-warp stores (lanes
+// spread over 4 heads x 8 dims) fall in 32 distinct banks.
+constexpr int kOStride = kD + 4;
+
 struct Partial {
     float m[8], l[8];          // per head
-    float o[8][kD];            // per head, un-normalised
+    float o[8][kOStride];      // per head, un-normalised (dims 0..kD-1 used)
 };
 
 struct Ring {

@@ -248,6 +248,18 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Registers filled by tcgen05.ld hold their values only after
+// tcgen05.wait::ld. An empty volatile asm that reads and writes them, placed
+// after the wait, makes every later use depend on a point after the wait (the
+// compiler cannot hoist a use above it). N is a multiple of 8.
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t* r) {
+#pragma unroll
+    for (int i = 0; i < N; i += 8)
+        asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]),
+                     "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7]));
+}
+
 // Shared-memory matrix descriptor (sm_100 format): start address, leading
 // and stride byte offsets (all >> 4), version 1 at bit 46, layout type at
 // bits 61-63 (2 = 128-byte swizzle).

@@ -123,10 +123,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     if (tok0 >= span_end || tok0 + 32 <= p.q_begin) return;
 
     if (warp == 0) {
-        const int nb_w = build_key_blocks_warp(p, j, sel + prob * p.kg, nsel + prob, false,
-                                               sm.blk_row, sm.blk_pos);
+        // barriers first, then the Q tiles (they do not depend on the key
+        // set), so the Q load overlaps the reads of the selection list
         if (lane == 0) {
-            sm.nb = nb_w;
             sm.abort = 0;
             ptx::mbar_init(&sm.bar_q, 1);
             for (int s = 0; s < 2; ++s) {
@@ -140,7 +139,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             }
             ptx::mbar_init(&sm.drain, 1);
             ptx::fence_mbar_init();
+            const int tq = tok0 - p.q_begin;
+            ptx::mbar_arrive_expect_tx(&sm.bar_q, 2 * kTile);
+            for (int x = 0; x < 2; ++x) {
+                ptx::tma_load_4d(sm.q[x], &maps.q, 0, h * 8, tq + 16 * x, b, &sm.bar_q);
+                ptx::tma_load_4d(sm.q[x] + kPanel, &maps.q, 64, h * 8, tq + 16 * x, b, &sm.bar_q);
+            }
         }
+        const int nb_w = build_key_blocks_warp(p, j, sel + prob * p.kg, nsel + prob, false,
+                                               sm.blk_row, sm.blk_pos);
+        if (lane == 0) sm.nb = nb_w;
     } else if (warp == 1) {
         ptx::tmem_alloc(&sm.tmem_base, kTmemCols);
         ptx::tmem_relinquish();
@@ -156,12 +164,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     if (warp == 0) {
         // ------------------------------------------------------ producer
         if (lane == 0 && n_tiles > 0) {
-            const int tq = tok0 - p.q_begin;
-            ptx::mbar_arrive_expect_tx(&sm.bar_q, 2 * kTile);
-            for (int x = 0; x < 2; ++x) {
-                ptx::tma_load_4d(sm.q[x], &maps.q, 0, h * 8, tq + 16 * x, b, &sm.bar_q);
-                ptx::tma_load_4d(sm.q[x] + kPanel, &maps.q, 64, h * 8, tq + 16 * x, b, &sm.bar_q);
-            }
             for (int t = 0; t < n_tiles; ++t) {
                 const int s = t & 1;
                 if (t >= 2 && !wait_bar(&sm.k_empty[s], ((t >> 1) - 1) & 1, abort, p.err)) break;
@@ -229,6 +231,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             while (!ptx::mbar_try_wait(&sm.drain, 0) &&
                    ptx::globaltimer_ns() - t0 < ptx::kWaitLimitNs) {
             }
+        } else if (lane == 0) {
+            // no key tile: still let the Q load land before the CTA exits
+            wait_bar(&sm.bar_q, 0, abort, p.err);
         }
     } else {
         // ------------------------------------------------------ softmax
@@ -257,6 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
 #pragma unroll
                 for (int c = 0; c < 4; ++c) ptx::tmem_ld32(s_addr + 32 * c, xr + 32 * c);
                 ptx::tmem_wait_ld();
+                ptx::reg_fence<kTileKeys>(xr);
             }
             // mask (causal within the current chunk; padding past the set)
             const int blk0 = t * kBlocksPerTile;
@@ -315,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                     uint32_t o[32];
                     ptx::tmem_ld32(o_addr + 32 * c, o);
                     ptx::tmem_wait_ld();
+                    ptx::reg_fence<32>(o);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
                     ptx::tmem_st32(o_addr + 32 * c, o);
@@ -338,6 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                 uint32_t o[32];
                 ptx::tmem_ld32(o_addr + 32 * c, o);
                 ptx::tmem_wait_ld();
+                ptx::reg_fence<32>(o);
                 if (row_ok) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 8) {

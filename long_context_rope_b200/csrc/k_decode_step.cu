@@ -11,18 +11,18 @@
 //
 // One cluster of CL CTAs per (sequence, KV head). The always-visible blocks
 // do not depend on routing, so the producer warp issues their TMA loads at
-// the start and they land while routing runs. Routing is split across the
-// cluster and needs no serial selection pass:
+// the start and they land while routing runs. Routing needs one cluster
+// exchange and no serial selection pass:
 //   level 1  CTA r scores a contiguous slice of the candidate chunks and
 //            ranks them locally (count of larger keys); its local top k_c
 //            (the only ones that can be in the global top k_c) go to every
 //            CTA's finalist table through distributed shared memory;
-//            cluster barrier; each CTA ranks its own finalists against the
-//            table: rank < k_c is a winner.
-//   level 2  each CTA scores the G groups of its own winning chunks, ranks
-//            them locally, publishes its local top k_g; cluster barrier;
-//            every CTA ranks the whole table and sorts the winners by
-//            group index, so every CTA holds the routed list.
+//            cluster barrier; every CTA ranks the whole table (rank < k_c
+//            wins) and sorts the winners by chunk index.
+//   level 2  every CTA scores all G groups of the selected chunks (at most
+//            G x k_c rows, shared through L2) and ranks them exactly; the
+//            candidates are already in ascending group order, so one warp
+//            compacts the winners with ballots.
 // Keys are 64-bit: the order-preserving 32-bit score key above, the index
 // below (lower index wins a tie), 0 = not a candidate, so every rank is
 // exact and unique. The scores are the same fp32 dot products, summed in the
@@ -52,13 +52,12 @@ using dec::kThreads;
 
 constexpr int kMaxSlice = 512;   // level-1 candidates per CTA
 constexpr int kMaxF1 = 512;      // level-1 finalist slots of the cluster
-constexpr int kMaxCand2 = 512;   // level-2 candidates per CTA
-constexpr int kMaxF2 = 1024;     // level-2 finalist slots of the cluster
+constexpr int kMaxCand2 = 512;   // level-2 candidates (G x k_c)
 constexpr int kMaxKc = 64;
 constexpr int kMaxKg = 512;
 constexpr int kMaxLocal = 256;   // key blocks per CTA
-constexpr int kRowsInFlight = 8;
 constexpr int kRankThreads = kConsumers * 32;
+constexpr int kL1Rows = 16;      // level-1 rows per consumer warp per batch
 
 struct StepMaps {
     CUtensorMap k, v;
@@ -74,15 +73,13 @@ struct StepSmem {
     uint64_t full[kStages], empty[kStages];
     uint64_t key1[kMaxSlice];     // own level-1 candidates
     uint64_t f1[kMaxF1];          // level-1 finalists of all CTAs
-    uint64_t key2[kMaxCand2];     // own level-2 candidates
-    uint64_t f2[kMaxF2];          // level-2 finalists of all CTAs
-    int rank[kMaxF2];             // rank scratch
-    int win1[kMaxKc];             // chunk winners by global rank (read in rank 0)
-    int own_win[kMaxKc];          // this CTA's winning chunks
-    int wl[kMaxKg];               // winning groups, unordered
-    int routed[kMaxKg];           // winning groups, ascending
+    uint64_t key2[kMaxCand2];     // level-2 candidates (all of them, every CTA)
+    int rank[kMaxSlice > kMaxCand2 ? kMaxSlice : kMaxCand2];  // rank scratch
+    int win1[kMaxKc];             // selected chunks, ascending
+    int wl[kMaxKc];               // selected chunks, unordered, as -(index + 1)
+    int routed[kMaxKg];           // selected groups, ascending
     int blk_pos[kMaxLocal];
-    int n_own_win, n_wl, n_dense, bad;
+    int n_win1, n_wl, bad;
 };
 
 __device__ __forceinline__ uint64_t rank_key(uint32_t key32, int idx) {
@@ -93,22 +90,40 @@ __device__ __forceinline__ int index_of(uint64_t k) {
 }
 
 // Consumer threads (kRankThreads): rank[x] = number of b[0..nb) larger than
-// a[x], for every present a[x] (0 = absent: not ranked, never counted).
-__device__ __forceinline__ void count_greater(const uint64_t* a, int na, const uint64_t* b, int nb,
-                                              int* rank) {
+// a[x], for every present a[x] (0 = absent: not ranked, never counted). Each
+// thread holds kR candidates and streams a 1/tpc share of b through them, so
+// one shared-memory load serves kR comparisons; the tpc partial counts of a
+// candidate are summed with warp shuffles.
+constexpr int kR = 4;
+template <typename T>
+__device__ __forceinline__ void count_greater(const T* a, int na, const T* b, int nb, int* rank) {
     const int t = threadIdx.x;
     int tpc = 1;
-    while (tpc < 32 && na * tpc * 2 <= kRankThreads) tpc <<= 1;
-    const int per_pass = kRankThreads / tpc;
-    const int sub = t % tpc;
-    for (int base = 0; base < na; base += per_pass) {
-        const int x = base + t / tpc;
-        const uint64_t ax = x < na ? a[x] : 0ull;
-        int cnt = 0;
-        if (ax != 0ull)
-            for (int y = sub; y < nb; y += tpc) cnt += b[y] > ax ? 1 : 0;
-        for (int off = 1; off < tpc; off <<= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-        if (sub == 0 && x < na && ax != 0ull) rank[x] = cnt;
+    while (tpc < 32 && tpc * 2 * na <= kRankThreads * kR) tpc <<= 1;
+    const int groups = kRankThreads / tpc;
+    const int sub = t % tpc, gid = t / tpc;
+    for (int base = 0; base < na; base += groups * kR) {
+        T ax[kR];
+        int cnt[kR];
+#pragma unroll
+        for (int k = 0; k < kR; ++k) {
+            const int x = base + gid + k * groups;
+            ax[k] = x < na ? a[x] : T(0);
+            cnt[k] = 0;
+        }
+#pragma unroll 4
+        for (int y = sub; y < nb; y += tpc) {
+            const T by = b[y];
+#pragma unroll
+            for (int k = 0; k < kR; ++k) cnt[k] += by > ax[k] ? 1 : 0;
+        }
+#pragma unroll
+        for (int k = 0; k < kR; ++k) {
+            for (int off = 1; off < tpc; off <<= 1)
+                cnt[k] += __shfl_xor_sync(0xffffffffu, cnt[k], off);
+            const int x = base + gid + k * groups;
+            if (sub == 0 && x < na && ax[k] != T(0)) rank[x] = cnt[k];
+        }
     }
 }
 
@@ -127,7 +142,7 @@ __device__ __forceinline__ int forced_below_in(const Params& p, int j, int lo, i
 
 // Score rows [0, n) of a summary table for this warp's share and hand each
 // (row, fp32 score) to emit. Same arithmetic and order as the routing kernels.
-template <typename RowOf, typename Emit>
+template <int kRowsInFlight, typename RowOf, typename Emit>
 __device__ __forceinline__ void score_rows(const float* q, int n, RowOf row_of, Emit emit) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int x0 = warp * kRowsInFlight; x0 < n; x0 += kConsumers * kRowsInFlight) {
@@ -186,9 +201,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     nf_loc = nf_loc < 0 ? 0 : nf_loc;
     if (tid == 0) {
         sm.bad = 0;
-        sm.n_own_win = 0;
+        sm.n_win1 = 0;
         sm.n_wl = 0;
-        sm.n_dense = 0;
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(&sm.full[s], 1);
             ptx::mbar_init(&sm.empty[s], 1);
@@ -206,15 +220,42 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
         for (int i = 0; i < n_pre; ++i)
             dec::issue_block(sm.u.ring, sm.full, i, &maps.k, &maps.v, sm.blk_pos[i], (int)bh);
 
+    // ---- level-1 slice: the first batch of this warp's chunk-summary rows is
+    // requested before q-bar, so the two memory latencies overlap
+    const int per1 = (j + CL - 1) / CL;
+    const int c_lo = r * per1;
+    const int c_hi = c_lo + per1 < j ? c_lo + per1 : j;
+    const int ns = c_hi > c_lo ? c_hi - c_lo : 0;
+    const float* ctab = cs + bh * (int64_t)p.nC * kD;
+    float4 first[kL1Rows];
+    if (consumer) {
+#pragma unroll
+        for (int u = 0; u < kL1Rows; ++u) {
+            const int x = warp * kL1Rows + u;
+            first[u] = x < ns ? __ldg(reinterpret_cast<const float4*>(ctab + (int64_t)(c_lo + x) * kD) + lane)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+
     // ---- q-bar of the new token over the KV head's gq query heads
     float qv[4] = {0.f, 0.f, 0.f, 0.f};
     {
         const int64_t row0 = ((int64_t)b * p.q_len * p.Hq + (int64_t)h * p.gq) * kD;
-#pragma unroll 8
-        for (int r2 = 0; r2 < p.gq; ++r2) {
-            const __nv_bfloat16* qp = q + row0 + (int64_t)r2 * kD + lane * 4;
+        uint2 raw[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) qv[e] += __bfloat162float(qp[e]);
+        for (int r2 = 0; r2 < 8; ++r2)
+            raw[r2] = r2 < p.gq ? *reinterpret_cast<const uint2*>(q + row0 + (int64_t)r2 * kD + lane * 4)
+                                : make_uint2(0u, 0u);
+#pragma unroll
+        for (int r2 = 0; r2 < 8; ++r2) {
+            if (r2 < p.gq) {
+                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[r2]);
+                const float2 lo = __bfloat1622float2(h2[0]), hi = __bfloat1622float2(h2[1]);
+                qv[0] += lo.x;
+                qv[1] += lo.y;
+                qv[2] += hi.x;
+                qv[3] += hi.y;
+            }
         }
         const float inv_n = 1.0f / (float)p.gq;
 #pragma unroll
@@ -226,18 +267,37 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     }
 
     // ---- level 1: own slice of the candidate chunks [0, j)
-    const int per1 = (j + CL - 1) / CL;
-    const int c_lo = r * per1;
-    const int c_hi = c_lo + per1 < j ? c_lo + per1 : j;
-    const int ns = c_hi > c_lo ? c_hi - c_lo : 0;
     const int cap1 = p.kc < per1 ? p.kc : per1;
-    const float* ctab = cs + bh * (int64_t)p.nC * kD;
-    if (consumer)
-        score_rows(qv, ns, [&](int x) { return ctab + (int64_t)(c_lo + x) * kD; },
-                   [&](int x, float s) {
-                       const int c = c_lo + x;
-                       sm.key1[x] = is_forced(p, j, c) ? 0ull : rank_key(score_key32(s), c);
-                   });
+    if (consumer) {
+        auto emit1 = [&](int x, float s) {
+            const int c = c_lo + x;
+            sm.key1[x] = is_forced(p, j, c) ? 0ull : rank_key(score_key32(s), c);
+        };
+        // the prefetched first batch (same dot products and order as score_rows)
+        float sc[kL1Rows];
+#pragma unroll
+        for (int u = 0; u < kL1Rows; ++u) {
+            float s = 0.f;
+            s = fmaf(qv[0], first[u].x, s);
+            s = fmaf(qv[1], first[u].y, s);
+            s = fmaf(qv[2], first[u].z, s);
+            s = fmaf(qv[3], first[u].w, s);
+            sc[u] = warp_sum(s);
+        }
+        if (lane < kL1Rows) {
+            float s = sc[0];
+#pragma unroll
+            for (int u = 1; u < kL1Rows; ++u)
+                if (lane == u) s = sc[u];
+            if (warp * kL1Rows + lane < ns) emit1(warp * kL1Rows + lane, s);
+        }
+        // rows beyond the first batch (slices longer than 8 x kL1Rows)
+        const int rest0 = kConsumers * kL1Rows;
+        if (ns > rest0)
+            score_rows<kL1Rows>(qv, ns - rest0,
+                                [&](int x) { return ctab + (int64_t)(c_lo + rest0 + x) * kD; },
+                                [&](int x, float s) { emit1(rest0 + x, s); });
+    }
     __syncthreads();
     if (consumer) count_greater(sm.key1, ns, sm.key1, ns, sm.rank);
     __syncthreads();
@@ -255,86 +315,56 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     }
     cluster.sync();
 
-    // own finalists against all finalists: the global top k_c
+    // ---- every CTA ranks the whole finalist table: the global top k_c
     const int nF1 = CL * cap1;
-    if (consumer) count_greater(sm.f1 + r * cap1, cap1, sm.f1, nF1, sm.rank);
+    if (consumer) count_greater(sm.f1, nF1, sm.f1, nF1, sm.rank);
     __syncthreads();
-    {
-        int* win1_0 = cluster.map_shared_rank(sm.win1, 0);
-        for (int x = tid; x < cap1; x += blockDim.x) {
-            const uint64_t k = sm.f1[r * cap1 + x];
-            if (k != 0ull && sm.rank[x] < p.kc) {
-                const int c = index_of(k);
-                win1_0[sm.rank[x]] = c;
-                sm.own_win[atomicAdd(&sm.n_own_win, 1)] = c;
-            }
-        }
+    for (int x = tid; x < nF1; x += blockDim.x) {
+        const uint64_t k = sm.f1[x];
+        if (k != 0ull && sm.rank[x] < p.kc) sm.wl[atomicAdd(&sm.n_win1, 1)] = -index_of(k) - 1;
     }
     __syncthreads();
+    // chunk winners in ascending order: wl holds -(index + 1), so the count of
+    // larger entries is the count of smaller indices
+    const int nsel1 = sm.n_win1;  // min(k_c, number of candidates)
+    if (consumer) count_greater(sm.wl, nsel1, sm.wl, nsel1, sm.rank);
+    __syncthreads();
+    for (int i = tid; i < nsel1; i += blockDim.x) sm.win1[sm.rank[i]] = -sm.wl[i] - 1;
+    __syncthreads();
+    if (r == 0) {
+        for (int i = tid; i < p.kc; i += blockDim.x) sel_c[prob * p.kc + i] = i < nsel1 ? sm.win1[i] : -1;
+        if (tid == 0) nsel_c[prob] = nsel1;
+    }
 
-    // ---- level 2: the G groups of this CTA's winning chunks
-    const int n2 = sm.n_own_win * p.G;
-    const int cap2_raw = p.G * (p.kc < cap1 ? p.kc : cap1);
-    const int cap2 = p.kg < cap2_raw ? p.kg : cap2_raw;
+    // ---- level 2: every CTA scores all G groups of the selected chunks
+    // (candidate x = group x % G of the (x / G)-th chunk: ascending group
+    // index) and ranks them exactly; no second cluster exchange is needed
+    const int n2 = nsel1 * p.G;
     const float* gtab = gs + bh * (int64_t)p.nC * p.G * kD;
     if (consumer)
-        score_rows(qv, n2,
-                   [&](int x) {
-                       return gtab + ((int64_t)sm.own_win[x / p.G] * p.G + x % p.G) * kD;
-                   },
-                   [&](int x, float s) {
-                       sm.key2[x] = rank_key(score_key32(s), sm.own_win[x / p.G] * p.G + x % p.G);
-                   });
+        score_rows<16>(qv, n2,
+                       [&](int x) { return gtab + ((int64_t)sm.win1[x / p.G] * p.G + x % p.G) * kD; },
+                       [&](int x, float s) {
+                           sm.key2[x] = rank_key(score_key32(s), sm.win1[x / p.G] * p.G + x % p.G);
+                       });
     __syncthreads();
     if (consumer) count_greater(sm.key2, n2, sm.key2, n2, sm.rank);
     __syncthreads();
-    {
-        const int filled = n2 < cap2 ? n2 : cap2;
-        for (int x = tid; x < n2; x += blockDim.x)
-            if (sm.rank[x] < cap2)
-                for (int t = 0; t < CL; ++t)
-                    cluster.map_shared_rank(sm.f2, t)[r * cap2 + sm.rank[x]] = sm.key2[x];
-        for (int x = filled + tid; x < cap2; x += blockDim.x)
-            for (int t = 0; t < CL; ++t) cluster.map_shared_rank(sm.f2, t)[r * cap2 + x] = 0ull;
-    }
-    cluster.sync();
-
-    // ---- selections
-    const int n_cand1 = j - forced_below_in(p, j, 0, j);
-    const int nsel1 = p.kc < n_cand1 ? p.kc : n_cand1;
-    if (r == 0 && warp == 0) {
-        int32_t* so = sel_c + prob * p.kc;
-        for (int i = lane; i < p.kc; i += 32) {
-            if (i < nsel1) {
-                const int c = sm.win1[i];
-                int pos = 0;
-                for (int t = 0; t < nsel1; ++t) pos += sm.win1[t] < c ? 1 : 0;
-                so[pos] = c;
-            }
-            if (i >= nsel1) so[i] = -1;
+    // winners (rank < k_g) in candidate order = ascending group index: one
+    // warp compacts them with ballots
+    if (warp == 0) {
+        int base = 0;
+        for (int x0 = 0; x0 < n2; x0 += 32) {
+            const int x = x0 + lane;
+            const bool win = x < n2 && sm.rank[x] < p.kg;
+            const unsigned m = __ballot_sync(0xffffffffu, win);
+            if (win) sm.routed[base + __popc(m & ((1u << lane) - 1u))] = index_of(sm.key2[x]);
+            base += __popc(m);
         }
-        if (lane == 0) nsel_c[prob] = nsel1;
+        if (lane == 0) sm.n_wl = base;
     }
-    // the table's present entries (at most G * k_c) are packed into key2,
-    // then ranked among themselves
-    const int nF2 = CL * cap2;
-    for (int x = tid; x < nF2; x += blockDim.x)
-        if (sm.f2[x] != 0ull) sm.key2[atomicAdd(&sm.n_dense, 1)] = sm.f2[x];
-    __syncthreads();
-    const int n_dense = sm.n_dense;
-    if (consumer) count_greater(sm.key2, n_dense, sm.key2, n_dense, sm.rank);
-    __syncthreads();
-    for (int x = tid; x < n_dense; x += blockDim.x)
-        if (sm.rank[x] < p.kg) sm.wl[atomicAdd(&sm.n_wl, 1)] = index_of(sm.key2[x]);
     __syncthreads();
     const int nw = sm.n_wl;
-    for (int i = tid; i < nw; i += blockDim.x) {
-        const int gi = sm.wl[i];
-        int pos = 0;
-        for (int t = 0; t < nw; ++t) pos += sm.wl[t] < gi ? 1 : 0;
-        sm.routed[pos] = gi;
-    }
-    __syncthreads();
     if (r == 0) {
         for (int i = tid; i < p.kg; i += blockDim.x) sel_g[prob * p.kg + i] = i < nw ? sm.routed[i] : -1;
         if (tid == 0) nsel_g[prob] = nw;
@@ -386,11 +416,10 @@ bool step_fits(const Params& p, int cl) {
     const int j = p.j0;
     const int per1 = (j + cl - 1) / cl;
     const int cap1 = p.kc < per1 ? p.kc : per1;
-    const int cap2_raw = p.G * (p.kc < cap1 ? p.kc : cap1);
-    const int cap2 = p.kg < cap2_raw ? p.kg : cap2_raw;
     const int n_fb_max = (p.n_sink + p.n_local + 1) * p.G;
-    return per1 <= kMaxSlice && cl * cap1 <= kMaxF1 && cap2_raw <= kMaxCand2 &&
-           cl * cap2 <= kMaxF2 && (n_fb_max + cl - 1) / cl + (p.kg + cl - 1) / cl <= kMaxLocal;
+    return per1 <= kMaxSlice && cl * cap1 <= kMaxF1 && cl * cap1 <= kMaxSlice &&
+           p.G * p.kc <= kMaxCand2 &&
+           (n_fb_max + cl - 1) / cl + (p.kg + cl - 1) / cl <= kMaxLocal;
 }
 
 std::mutex g_step_mu;

@@ -49,9 +49,12 @@ struct QVec<float> {
 };
 
 // q-bar of every (b, KV head, query chunk): mean of the rotated queries over
-// the chunk's query tokens and the KV head's gq query heads. Grid (nQC, B).
+// the chunk's query tokens and the KV head's gq query heads. Grid (nQC, B);
+// 128 threads, so one wave holds the whole grid (64K context: 1024 CTAs, ~7
+// per SM at 48 registers) and no partial second wave trails the stream.
+constexpr int kQbarThreads = 128;
 template <typename T>
-__global__ void __launch_bounds__(256) qbar_kernel(Params p, const T* __restrict__ q,
+__global__ void __launch_bounds__(kQbarThreads) qbar_kernel(Params p, const T* __restrict__ q,
                                                    float* __restrict__ qbar) {
     constexpr int V = QVec<T>::N;
     extern __shared__ float red[];
@@ -332,17 +335,17 @@ cudaError_t launch_qbar(const Params& p, const void* q_rot, float* qbar, cudaStr
     if (p.nQC == 0) return cudaSuccess;
     const int V = p.dtype == HGA_BF16 ? 8 : 4;
     const int ncol = p.Hkv * (p.d / V);
-    const int TL = ncol >= 256 ? 1 : 256 / ncol;
+    const int TL = ncol >= kQbarThreads ? 1 : kQbarThreads / ncol;
     size_t smem = (size_t)TL * ncol * V * sizeof(float);
     dim3 grid(p.nQC, p.B);
     if (p.dtype == HGA_BF16) {
         auto fn = qbar_kernel<__nv_bfloat16>;
         if (smem > 48 * 1024) cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        fn<<<grid, 256, smem, st>>>(p, (const __nv_bfloat16*)q_rot, qbar);
+        fn<<<grid, kQbarThreads, smem, st>>>(p, (const __nv_bfloat16*)q_rot, qbar);
     } else {
         auto fn = qbar_kernel<float>;
         if (smem > 48 * 1024) cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        fn<<<grid, 256, smem, st>>>(p, (const float*)q_rot, qbar);
+        fn<<<grid, kQbarThreads, smem, st>>>(p, (const float*)q_rot, qbar);
     }
     return cudaGetLastError();
 }
