@@ -340,20 +340,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             const float inv = l > 0.f ? 1.0f / l : 0.f;
             __nv_bfloat16* orow =
                 out + (((int64_t)b * p.q_len + (qpos - p.q_begin)) * p.Hq + (int64_t)h * 8 + head) * kD;
+            // all of O in one round trip
+            uint32_t o[kD];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t o[32];
-                ptx::tmem_ld32(o_addr + 32 * c, o);
-                ptx::tmem_wait_ld();
-                ptx::reg_fence<32>(o);
-                if (row_ok) {
+            for (int c = 0; c < 4; ++c) ptx::tmem_ld32(o_addr + 32 * c, o + 32 * c);
+            ptx::tmem_wait_ld();
+            ptx::reg_fence<kD>(o);
+            if (row_ok) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        float f[8];
+                for (int e = 0; e < kD; e += 8) {
+                    float f[8];
 #pragma unroll
-                        for (int z = 0; z < 8; ++z) f[z] = __uint_as_float(o[e + z]) * inv;
-                        *reinterpret_cast<uint4*>(orow + 32 * c + e) = f32x8_to_bf16(f);
-                    }
+                    for (int z = 0; z < 8; ++z) f[z] = __uint_as_float(o[e + z]) * inv;
+                    *reinterpret_cast<uint4*>(orow + e) = f32x8_to_bf16(f);
                 }
             }
         } else if (row_ok) {

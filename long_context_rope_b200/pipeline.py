@@ -131,3 +131,31 @@ def fill_windows(cfg: hga.HgaConfig, k_full, v_full, k_win, v_win):
         hi = min((c + 1) * C, cfg.seq_len)
         k_win[:, :, w * C: w * C + hi - c * C].copy_(k_full[:, :, c * C: hi], non_blocking=True)
         v_win[:, :, w * C: w * C + hi - c * C].copy_(v_full[:, :, c * C: hi], non_blocking=True)
+
+
+def decode_append(cfg_cap: hga.HgaConfig, pos: int, k_new_raw, v_new, q_rot_new, k_raw_cache,
+                  k_rot_cache, v_cache, cs, gs, rb: RouteBuffers, out, stream=None):
+    """One step of a decode loop over caches of fixed capacity cfg_cap.seq_len
+    ([B, Hkv, capacity, d]) at token position `pos`.
+
+    Appends the new token (k_new_raw, v_new: [B, Hkv, d]) to the caches,
+    rotates its key into the rotated cache (hga_apply_rope at position pos),
+    and when the token completes its chunk, finalises that chunk's summaries
+    and rotated keys (hga_build_summaries on that one chunk). Then routes and
+    attends for the query q_rot_new [B, 1, Hq, d] at position pos
+    (hga_decode_step with q_begin = pos, q_len = 1): routing reads only the
+    summaries of chunks before the query's chunk, and attention masks keys
+    after pos, so cache rows past pos are never used."""
+    B, H, d = cfg_cap.batch, cfg_cap.n_kv_heads, cfg_cap.head_dim
+    k_new_raw = k_new_raw.contiguous()
+    k_raw_cache[:, :, pos].copy_(k_new_raw, non_blocking=True)
+    v_cache[:, :, pos].copy_(v_new, non_blocking=True)
+    rot = torch.empty_like(k_new_raw)
+    hga.apply_rope(cfg_cap, k_new_raw, rot, B * H, 1, 1, pos, stream)
+    k_rot_cache[:, :, pos].copy_(rot, non_blocking=True)
+    if (pos + 1) % cfg_cap.chunk_size == 0:
+        c = pos // cfg_cap.chunk_size
+        hga.build_summaries(cfg_cap, k_raw_cache, cs, gs, k_rot_cache, c, c + 1, stream)
+    cfg_q = cfg_cap.copy(q_begin=pos, q_len=1)
+    hga.decode_step(cfg_q, q_rot_new, cs, gs, k_rot_cache, v_cache, rb.qbar, rb.sel_chunks,
+                    rb.n_sel_chunks, rb.sel_groups, rb.n_sel_groups, out, stream)

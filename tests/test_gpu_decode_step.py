@@ -179,3 +179,53 @@ def test_decode_step_repeat_and_prefill_route():
     assert hga.get_device_error() == 0
     for name in ("qbar", "sel_chunks", "n_sel_chunks", "sel_groups", "n_sel_groups"):
         assert torch.equal(getattr(rb1, name), getattr(rb2, name)), name
+
+
+def test_decode_loop_appends_and_finalises_chunks():
+    """A decode loop over caches of fixed capacity (pipeline.decode_append):
+    each step appends a token, rotates its key into the cache, finalises the
+    summaries of the chunk it completes, and routes + attends at its position
+    with the one-launch step. Checked against the oracle run from scratch on
+    the prefix up to that position, at steps around two chunk ends; with no
+    local window, the chunk finished at position 1343 is a routing candidate
+    at position 1344, so its freshly built summary is used."""
+    from long_context_rope_b200 import hga, pipeline
+    cap = 64 * 24
+    wp = BASE.replace(name="loop", batch=2, seq_len=cap, mode="prefill", n_local=0,
+                      plant_every=1, plant_count=2)
+    x = synth.draw(wp, seed=7)  # keys, values and queries at every position
+    cfg_cap = hga.config_from(wp)
+    L0 = 64 * 20 - 3
+    B, H, d = wp.batch, wp.n_kv_heads, wp.head_dim
+    k_raw_cache = torch.zeros(B, H, cap, d, dtype=torch.bfloat16, device="cuda")
+    v_cache = torch.zeros_like(k_raw_cache)
+    k_raw_cache[:, :, :L0] = x["k_raw"][:, :, :L0].cuda()
+    v_cache[:, :, :L0] = x["v"][:, :, :L0].cuda()
+    k_rot_cache = torch.zeros_like(k_raw_cache)
+    cs, gs = pipeline.alloc_summaries(cfg_cap)
+    hga.build_summaries(cfg_cap, k_raw_cache, cs, gs, k_rot_cache, 0, L0 // 64 + 1)
+    check = {L0, 64 * 20 - 1, 64 * 20, 64 * 20 + 1, 64 * 21 - 1, 64 * 21, 64 * 21 + 1}
+    n_checked = 0
+    for pos in range(L0, 64 * 21 + 2):
+        cfg_q = cfg_cap.copy(q_begin=pos, q_len=1)
+        r = None
+        if pos in check:
+            w_pos = wp.replace(seq_len=pos + 1, mode="decode")
+            r = O.pipeline(w_pos, {"k_raw": x["k_raw"][:, :, :pos + 1], "v": x["v"][:, :, :pos + 1],
+                                   "q_raw": x["q_raw"][:, pos:pos + 1]})
+            q_rot = torch.from_numpy(np.ascontiguousarray(r["q_rot"])).to(torch.bfloat16).cuda()
+        else:
+            q_rot = pipeline.rotate_queries(cfg_q, x["q_raw"][:, pos:pos + 1].cuda())
+        rb = pipeline.alloc_route(cfg_q)
+        out = torch.full_like(q_rot, float("nan"))
+        pipeline.decode_append(cfg_cap, pos, x["k_raw"][:, :, pos].cuda(), x["v"][:, :, pos].cuda(),
+                               q_rot, k_raw_cache, k_rot_cache, v_cache, cs, gs, rb, out)
+        if r is not None:
+            torch.cuda.synchronize()
+            assert hga.get_device_error() == 0
+            w_pos = wp.replace(seq_len=pos + 1, mode="decode")
+            worst = _oracle_compare(w_pos, r, rb, out)
+            n_checked += 1
+            print(f"pos {pos}: chunks {int(rb.n_sel_chunks[0, 0, 0])} groups "
+                  f"{int(rb.n_sel_groups[0, 0, 0])} max abs error {worst:.3e}")
+    assert n_checked == len(check)
