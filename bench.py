@@ -308,30 +308,34 @@ def run_decode(name, args, dist):
         pipeline.fill_windows(cfg, k_host, v_host, k_win, v_win)
         cfg_w = cfg.copy(kv_layout=hga.HGA_KV_WINDOWS)
 
-        def step(separate=False):
+        # warm tier: a VRAM pool of 4 x top_k_groups groups per (sequence, KV head)
+        pool = pipeline.alloc_warm_pool(cfg, 4 * cfg.top_k_groups, dev)
+
+        def step(separate=False, warm=False):
             pipeline.decode(cfg_w, q_rot, cs, gs, k_win, v_win, rb, out, gathered=gat,
-                            k_src=k_host, v_src=v_host, src_is_host=True, separate=separate)
+                            k_src=k_host, v_src=v_host, src_is_host=True, separate=separate,
+                            warm=pool if warm else None)
         launches, launches_sep = 3, 4  # route (one launch), gather, attend
     else:
         v = x["v"].to(dev)
 
-        def step(separate=False):
+        def step(separate=False, warm=False):
             pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out, separate=separate)
         launches, launches_sep = 1, 3  # one-launch decode step
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     K = max(args.steps, 20)
 
-    def timed(separate):
+    def timed(separate, warm=False):
         """Median device time of one step replayed from a CUDA graph (L2
         flushed between steps), plus the eager median for reference."""
         for _ in range(max(3, args.warmup)):
-            step(separate)
+            step(separate, warm)
         torch.cuda.synchronize()
         if hga.get_device_error() != 0:
             raise RuntimeError(f"device error word set in {name}")
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, capture_error_mode="relaxed"):
-            step(separate)
+            step(separate, warm)
         for _ in range(3):
             graph.replay()
         torch.cuda.synchronize()
@@ -349,7 +353,7 @@ def run_decode(name, args, dist):
         for i in range(5):
             flush.fill_(i & 0xff)
             ev2.rec(2 * i, st)
-            step(separate)
+            step(separate, warm)
             ev2.rec(2 * i + 1, st)
         torch.cuda.synchronize()
         eager = float(np.median([ev2.ms(2 * i, 2 * i + 1) * 1000.0 for i in range(5)]))
@@ -360,6 +364,17 @@ def run_decode(name, args, dist):
     times, eager_us = timed(False)
     us = dist.max(float(np.median(times)))
     us_sep = dist.max(float(np.median(times_sep)))
+    warm_info = None
+    if w.tiered:
+        # steady state of the warm tier for this (fixed) query: its routed groups
+        # stay in the pool, so no group crosses the host link after the first step
+        times_warm, _ = timed(False, warm=True)
+        hits_misses = pool.stats.cpu().numpy().reshape(-1, 2).sum(0)
+        warm_info = dict(us_per_step=dist.max(float(np.median(times_warm))),
+                         pool_slots=int(pool.tag.shape[-1]),
+                         hit_rate=float(hits_misses[0] / max(1, hits_misses.sum())),
+                         host_bytes_per_step=int(hits_misses[1]) * 16 * w.head_dim * 2 * 2,
+                         note="fixed query: the all-hits steady state of the warm tier")
     n_sel = rb.n_sel_groups.cpu().numpy()
     moved = int(n_sel.sum()) * 16 * w.head_dim * 2 * 2  # routed K+V bytes
     # algorithmic HBM bytes of one step (each byte the step must touch, once)
@@ -375,7 +390,7 @@ def run_decode(name, args, dist):
                 us_per_step_eager=eager_us, cuda_graph=True,
                 launches_per_step=launches, routed_kv_bytes=moved,
                 us_per_step_separate_kernels=us_sep, us_per_step_separate_eager=eager_sep,
-                launches_per_step_separate=launches_sep,
+                launches_per_step_separate=launches_sep, warm_tier=warm_info,
                 host_link_gbs=(moved / (us * 1e-6) / 1e9) if w.tiered else None)
 
 

@@ -187,6 +187,35 @@ hga_status hga_gather_kv(const hga_config* cfg, const void* k_src, const void* v
                          int32_t src_is_host, const int32_t* sel_groups,
                          const int32_t* n_sel_groups, void* k_dst, void* v_dst, void* stream);
 
+/* Warm tier ("Geheugenarchitectuur": a bounded LRU cache in VRAM keeps
+ * recently routed groups between the cold host store and attention). Same
+ * result in k_dst / v_dst as hga_gather_kv with src_is_host = 1 for a
+ * one-token query span (decode): every selected group's K and V rows. A group
+ * already in the caller's VRAM pool is copied from there; a missing group is
+ * read once over the host link and also stored in the pool slot whose last
+ * use is oldest among the slots this call does not hit (ties: lower slot;
+ * empty slots first), so only misses cross the host link.
+ *   k_host, v_host     full store [B, Hkv, L, d] in mapped page-locked host
+ *                      memory (as for hga_gather_kv).
+ *   pool_k, pool_v     [B, Hkv, n_slots, g, d] device memory, cfg->dtype.
+ *   pool_tag           [B, Hkv, n_slots] int32: group index held, -1 = empty.
+ *   pool_last          [B, Hkv, n_slots] int32: step of last use, -1 = never.
+ *                      Initialise both to -1 once; the call updates them.
+ *   n_slots            top_k_groups <= n_slots <= 4096.
+ *   step               this call's step number, increasing over calls.
+ *   src_out            [B, Hkv, top_k_groups] int32, written: the source of
+ *                      each selected group (pool slot for a hit, -2 - slot for
+ *                      a miss that filled that slot, -1 for an unused entry).
+ *   stats_out          NULL or [B, Hkv, 2] int32: hits, misses.
+ * Calls on one pool must not overlap (each reads and updates its tags).
+ * HGA_ERR_UNSUPPORTED unless q_len == 1; HGA_ERR_MEMORY if a host pointer
+ * is not mapped. */
+hga_status hga_gather_kv_warm(const hga_config* cfg, const void* k_host, const void* v_host,
+                              const int32_t* sel_groups, const int32_t* n_sel_groups,
+                              void* pool_k, void* pool_v, int32_t* pool_tag, int32_t* pool_last,
+                              int32_t n_slots, int32_t step, int32_t* src_out,
+                              int32_t* stats_out, void* k_dst, void* v_dst, void* stream);
+
 /* Exact softmax attention over the bounded set ("Kernmechanisme" item 4):
  * for each query token at position p in chunk j and each query head, softmax
  * (scale 1/sqrt(d), fp32 accumulation) over the keys at positions <= p of

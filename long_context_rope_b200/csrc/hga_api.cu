@@ -112,7 +112,7 @@ static_assert(offsetof(hga_config, rope_theta) == 48, "hga_config layout is part
 
 extern "C" {
 
-int32_t hga_version(void) { return 10100; }
+int32_t hga_version(void) { return 10200; }
 
 const char* hga_status_string(hga_status s) {
     switch (s) {
@@ -319,6 +319,36 @@ hga_status hga_gather_kv(const hga_config* cfg, const void* k_src, const void* v
     if ((s = device_view(v_src, src_is_host != 0, &vd)) != HGA_OK) return s;
     return launched(launch_gather(p, kd, vd, src_is_host != 0, sel_groups, n_sel_groups, k_dst,
                                   v_dst, (cudaStream_t)stream));
+}
+
+hga_status hga_gather_kv_warm(const hga_config* cfg, const void* k_host, const void* v_host,
+                              const int32_t* sel_groups, const int32_t* n_sel_groups,
+                              void* pool_k, void* pool_v, int32_t* pool_tag, int32_t* pool_last,
+                              int32_t n_slots, int32_t step, int32_t* src_out,
+                              int32_t* stats_out, void* k_dst, void* v_dst, void* stream) {
+    Params p;
+    hga_status s = make_params(cfg, &p);
+    if (s != HGA_OK) return s;
+    if (p.nQC == 0) return HGA_OK;
+    if (!k_host || !v_host || !sel_groups || !n_sel_groups || !pool_k || !pool_v || !pool_tag ||
+        !pool_last || !src_out || !k_dst || !v_dst)
+        return HGA_ERR_NULL;
+    if (!aligned16(k_host) || !aligned16(v_host) || !aligned16(sel_groups) ||
+        !aligned16(n_sel_groups) || !aligned16(pool_k) || !aligned16(pool_v) ||
+        !aligned16(pool_tag) || !aligned16(pool_last) || !aligned16(src_out) ||
+        !aligned16(k_dst) || !aligned16(v_dst) || (stats_out && !aligned16(stats_out)))
+        return HGA_ERR_ALIGN;
+    if (p.q_len != 1) return HGA_ERR_UNSUPPORTED;
+    if (n_slots < p.kg || step < 0) return HGA_ERR_SHAPE;
+    if (!gather_warm_supports(p, n_slots)) return HGA_ERR_UNSUPPORTED;
+    HGA_ATTACH_ERR(p);
+    const void* kd = nullptr;
+    const void* vd = nullptr;
+    if ((s = device_view(k_host, true, &kd)) != HGA_OK) return s;
+    if ((s = device_view(v_host, true, &vd)) != HGA_OK) return s;
+    return launched(launch_gather_warm(p, kd, vd, sel_groups, n_sel_groups, pool_k, pool_v,
+                                       pool_tag, pool_last, n_slots, step, src_out, stats_out,
+                                       k_dst, v_dst, (cudaStream_t)stream));
 }
 
 hga_status hga_attend(const hga_config* cfg, const void* q_rot, const void* k_res,

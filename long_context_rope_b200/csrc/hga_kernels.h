@@ -47,6 +47,17 @@ cudaError_t launch_gather(const Params& p, const void* k_src, const void* v_src,
                           const int32_t* sel_groups, const int32_t* n_sel_groups, void* k_dst,
                           void* v_dst, cudaStream_t st);
 
+// Warm tier for one-token decode: the selected groups into k_dst / v_dst,
+// from a VRAM pool of n_slots groups per (sequence, KV head) where present,
+// else from the mapped host store (also filling the least recently used
+// pool slot). Needs nQC == 1 and top_k_groups <= n_slots <= 4096.
+bool gather_warm_supports(const Params& p, int n_slots);
+cudaError_t launch_gather_warm(const Params& p, const void* k_host, const void* v_host,
+                               const int32_t* sel_groups, const int32_t* n_sel_groups,
+                               void* pool_k, void* pool_v, int32_t* pool_tag, int32_t* pool_last,
+                               int n_slots, int step, int32_t* src_out, int32_t* stats_out,
+                               void* k_dst, void* v_dst, cudaStream_t st);
+
 // Where an attention unit finds its keys.
 struct KvSources {
     const void* k_res;  // full store [B,Hkv,L,d] or forced windows [B,Hkv,W*C,d]

@@ -14,6 +14,7 @@
 #include "hga_blocks.cuh"
 #include "hga_kernels.h"
 #include "hga_ptx.cuh"
+#include "hga_topk.cuh"
 
 namespace hga {
 
@@ -133,7 +134,196 @@ __global__ void __launch_bounds__(256) gather_host_kernel(Params p, const uint4*
     }
 }
 
+// ------------------------------------------------------------ warm tier
+// "Geheugenarchitectuur": between the cold store in host RAM and attention,
+// a bounded cache in VRAM keeps recently routed groups (least recently used
+// out). Per (sequence, KV head) the caller owns n_slots pool slots of one
+// group each, with the group index held (tag, -1 = empty) and the step of
+// last use (last, -1 = never).
+
+// Plan: one CTA per (sequence, KV head). Hits are found by a binary search
+// of every slot's tag in the (ascending) selection list; the misses take the
+// slots with the oldest last use that this step does not hit (ties to the
+// lower slot), chosen exactly by the warp radix select. Writes the source of
+// every selected group to src (slot for a hit, -2 - slot for a miss that
+// fills that slot, -1 for an invalid entry) and updates tag / last.
+constexpr int kMaxWarmSlots = 4096;
+
+__global__ void __launch_bounds__(256) warm_plan_kernel(Params p, const int32_t* __restrict__ sel,
+                                                        const int32_t* __restrict__ nsel,
+                                                        int32_t* __restrict__ tag,
+                                                        int32_t* __restrict__ last, int n_slots,
+                                                        int step, int32_t* __restrict__ src,
+                                                        int32_t* __restrict__ stats) {
+    extern __shared__ uint32_t wsm[];
+    uint32_t* key = wsm;                           // [n_slots] victim keys (0 = taken this step)
+    uint32_t* hist = key + n_slots;                // [256]
+    int* gi = reinterpret_cast<int*>(hist + 256);  // [kg] validated selection, -1 invalid
+    int* hit = gi + p.kg;                          // [kg] slot holding the group, -1 none
+    int* victim = hit + p.kg;                      // [kg] victim slots, ascending
+    int* lst = victim + p.kg;                      // [kg] the list as given
+    __shared__ int n_miss, n_valid;
+    const int64_t bh = blockIdx.x;
+    const int j = p.j0;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t prob = bh * p.nQC;
+    const int n = checked_count(p, nsel, prob);
+    const int32_t* list = sel + prob * p.kg;
+    for (int s = tid; s < p.kg; s += blockDim.x) {
+        gi[s] = s < n ? checked_group_entry(p, j, list, s) : -1;
+        lst[s] = s < n ? list[s] : -1;
+        hit[s] = -1;
+    }
+    __syncthreads();
+    int32_t* utag = tag + bh * n_slots;
+    int32_t* ulast = last + bh * n_slots;
+    for (int t = tid; t < n_slots; t += blockDim.x) {
+        const int g = utag[t];
+        int found = -1;
+        if (g >= 0) {  // binary search in the ascending list (valid entries ascend)
+            int lo = 0, hi = n - 1;
+            while (lo <= hi) {
+                const int mid = (lo + hi) >> 1;
+                const int v = lst[mid];
+                if (v == g) {
+                    found = mid;
+                    break;
+                }
+                if (v < g) lo = mid + 1; else hi = mid - 1;
+            }
+            if (found >= 0 && gi[found] < 0) found = -1;
+        }
+        if (found >= 0) hit[found] = t;
+        // older last use -> larger key; never used -> largest; hit -> 0 (not a victim)
+        key[t] = found >= 0 ? 0u : 0xffffffffu - (uint32_t)(ulast[t] + 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int m = 0, nv = 0;
+        for (int s0 = 0; s0 < n; s0 += 32) {
+            const int s = s0 + lane;
+            m += __popc(__ballot_sync(0xffffffffu, s < n && gi[s] >= 0 && hit[s] < 0));
+            nv += __popc(__ballot_sync(0xffffffffu, s < n && gi[s] >= 0));
+        }
+        warp_radix_topk(key, n_slots, m, m, victim, hist, [](int x) { return x; });
+        if (lane == 0) {
+            n_miss = m;
+            n_valid = nv;
+        }
+    }
+    __syncthreads();
+    // the i-th miss in list order takes the i-th victim
+    if (warp == 0) {
+        int base = 0;
+        for (int s0 = 0; s0 < p.kg; s0 += 32) {
+            const int s = s0 + lane;
+            const bool valid = s < n && gi[s] >= 0;
+            const bool miss = valid && hit[s] < 0;
+            const unsigned mm = __ballot_sync(0xffffffffu, miss);
+            int out = -1;
+            if (valid) out = miss ? -2 - victim[base + __popc(mm & ((1u << lane) - 1u))] : hit[s];
+            if (s < p.kg) src[prob * p.kg + s] = out;
+            if (valid) {
+                const int slot = miss ? victim[base + __popc(mm & ((1u << lane) - 1u))] : hit[s];
+                if (miss) utag[slot] = gi[s];
+                ulast[slot] = step;
+            }
+            base += __popc(mm);
+        }
+        if (lane == 0 && stats) {
+            stats[2 * bh] = n_valid - n_miss;  // hits (invalid entries count as neither)
+            stats[2 * bh + 1] = n_miss;
+        }
+    }
+}
+
+// Copy: grid (ceil(kg / kHostSlots), 1, B*Hkv), 256 threads. A hit copies
+// pool slot -> k_dst / v_dst (VRAM); a miss reads the mapped host store once
+// and writes both k_dst / v_dst and its pool slot.
+__global__ void __launch_bounds__(256) warm_copy_kernel(Params p, const uint4* __restrict__ k_host,
+                                                        const uint4* __restrict__ v_host,
+                                                        const int32_t* __restrict__ sel,
+                                                        const int32_t* __restrict__ src,
+                                                        uint4* __restrict__ pool_k,
+                                                        uint4* __restrict__ pool_v, int n_slots,
+                                                        uint4* __restrict__ k_dst,
+                                                        uint4* __restrict__ v_dst) {
+    __shared__ int s_src[kHostSlots], s_gi[kHostSlots];
+    const int64_t bh = blockIdx.z;
+    const int64_t prob = bh * p.nQC;
+    const int es = p.dtype == HGA_BF16 ? 2 : 4;
+    const int vec_per_blk = kGroupRows * p.d * es / 16;
+    const int s_lo = blockIdx.x * kHostSlots;
+    if (threadIdx.x < kHostSlots) {
+        const int s = s_lo + threadIdx.x;
+        s_src[threadIdx.x] = s < p.kg ? src[prob * p.kg + s] : -1;
+        s_gi[threadIdx.x] = s < p.kg ? sel[prob * p.kg + s] : -1;
+    }
+    __syncthreads();
+    const int64_t host_base = bh * (int64_t)p.L * p.d * es / 16;
+    const int64_t pool_base = bh * (int64_t)n_slots * vec_per_blk;
+    const int64_t dst_base = prob * (int64_t)p.kg * vec_per_blk;
+    for (int v0 = threadIdx.x; v0 < vec_per_blk; v0 += blockDim.x) {
+        uint4 kk[kHostSlots], vv[kHostSlots];
+#pragma unroll
+        for (int u = 0; u < kHostSlots; ++u) {
+            const int sr = s_src[u];
+            if (sr >= 0) {
+                const int64_t off = pool_base + (int64_t)sr * vec_per_blk + v0;
+                kk[u] = pool_k[off];
+                vv[u] = pool_v[off];
+            } else if (sr <= -2) {
+                const int64_t off = host_base + (int64_t)s_gi[u] * vec_per_blk + v0;
+                kk[u] = k_host[off];
+                vv[u] = v_host[off];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kHostSlots; ++u) {
+            const int sr = s_src[u];
+            if (sr == -1) continue;
+            const int64_t off = dst_base + (int64_t)(s_lo + u) * vec_per_blk + v0;
+            k_dst[off] = kk[u];
+            v_dst[off] = vv[u];
+            if (sr <= -2) {
+                const int64_t po = pool_base + (int64_t)(-2 - sr) * vec_per_blk + v0;
+                pool_k[po] = kk[u];
+                pool_v[po] = vv[u];
+            }
+        }
+    }
+}
+
 }  // namespace
+
+bool gather_warm_supports(const Params& p, int n_slots) {
+    return p.nQC == 1 && n_slots >= p.kg && n_slots <= kMaxWarmSlots;
+}
+
+cudaError_t launch_gather_warm(const Params& p, const void* k_host, const void* v_host,
+                               const int32_t* sel_groups, const int32_t* n_sel_groups,
+                               void* pool_k, void* pool_v, int32_t* pool_tag, int32_t* pool_last,
+                               int n_slots, int step, int32_t* src_out, int32_t* stats_out,
+                               void* k_dst, void* v_dst, cudaStream_t st) {
+    const size_t smem = (size_t)(n_slots + 256) * sizeof(uint32_t) + (size_t)4 * p.kg * sizeof(int);
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(warm_plan_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)((kMaxWarmSlots + 256) * 4 + 4 * kMaxBlocks * 4));
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    warm_plan_kernel<<<p.B * p.Hkv, 256, smem, st>>>(p, sel_groups, n_sel_groups, pool_tag,
+                                                     pool_last, n_slots, step, src_out, stats_out);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    dim3 grid((p.kg + kHostSlots - 1) / kHostSlots, 1, p.B * p.Hkv);
+    warm_copy_kernel<<<grid, 256, 0, st>>>(p, (const uint4*)k_host, (const uint4*)v_host,
+                                           sel_groups, src_out, (uint4*)pool_k, (uint4*)pool_v,
+                                           n_slots, (uint4*)k_dst, (uint4*)v_dst);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_gather(const Params& p, const void* k_src, const void* v_src, bool from_host,
                           const int32_t* sel_groups, const int32_t* n_sel_groups, void* k_dst,

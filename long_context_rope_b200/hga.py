@@ -83,6 +83,7 @@ def _load():
         "hga_attend": [C, P, P, P, P, P, P, P, P, P],
         "hga_route": [C, P, P, P, P, P, P, P, P, P],
         "hga_decode_step": [C, P, P, P, P, P, P, P, P, P, P, P, P],
+        "hga_gather_kv_warm": [C, P, P, P, P, P, P, P, P, I32, I32, P, P, P, P, P],
         "hga_get_device_error": [P, ctypes.POINTER(I32)],
     }
     for name, args in sig.items():
@@ -251,6 +252,30 @@ def gather_kv(cfg: HgaConfig, k_src, v_src, src_is_host: bool, sel_groups, n_sel
         _ptr(n_sel_groups, "n_sel_groups", torch.int32, (B, H, nQC)),
         _ptr(k_dst, "k_dst", dt, dst_shape), _ptr(v_dst, "v_dst", dt, dst_shape),
         _stream(stream)), "hga_gather_kv")
+
+
+def gather_kv_warm(cfg: HgaConfig, k_host, v_host, sel_groups, n_sel_groups, pool_k, pool_v,
+                   pool_tag, pool_last, step: int, src_out, k_dst, v_dst, stats=None,
+                   stream=None) -> None:
+    """Warm-tier gather for a one-token query span (see hga_gather_kv_warm)."""
+    B, H, d, kg, g = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.top_k_groups, cfg.group_size
+    dt = cfg.torch_dtype()
+    n_slots = pool_tag.shape[-1]
+    store = (B, H, cfg.seq_len, d)
+    gat_shape = (B, H, cfg.n_qchunks, kg * g, d)
+    _check(_lib.hga_gather_kv_warm(
+        ctypes.byref(cfg), _ptr(k_host, "k_host", dt, store, device=False),
+        _ptr(v_host, "v_host", dt, store, device=False),
+        _ptr(sel_groups, "sel_groups", torch.int32, (B, H, cfg.n_qchunks, kg)),
+        _ptr(n_sel_groups, "n_sel_groups", torch.int32, (B, H, cfg.n_qchunks)),
+        _ptr(pool_k, "pool_k", dt, (B, H, n_slots, g, d)),
+        _ptr(pool_v, "pool_v", dt, (B, H, n_slots, g, d)),
+        _ptr(pool_tag, "pool_tag", torch.int32, (B, H, n_slots)),
+        _ptr(pool_last, "pool_last", torch.int32, (B, H, n_slots)), n_slots, step,
+        _ptr(src_out, "src_out", torch.int32, (B, H, kg)),
+        _ptr(stats, "stats", torch.int32, (B, H, 2), nullable=True),
+        _ptr(k_dst, "k_dst", dt, gat_shape), _ptr(v_dst, "v_dst", dt, gat_shape),
+        _stream(stream)), "hga_gather_kv_warm")
 
 
 def window_slots(cfg: HgaConfig) -> int:

@@ -31,6 +31,29 @@ class RouteBuffers:
     group_scores: Optional[torch.Tensor] = None
 
 
+@dataclasses.dataclass
+class WarmPool:
+    """Warm tier: a VRAM pool of n_slots routed groups per (sequence, KV
+    head), their tags and last-use steps, and per-call outputs."""
+    k: torch.Tensor
+    v: torch.Tensor
+    tag: torch.Tensor
+    last: torch.Tensor
+    src: torch.Tensor
+    stats: torch.Tensor
+    step: int = 0
+
+
+def alloc_warm_pool(cfg: hga.HgaConfig, n_slots: int, device="cuda") -> WarmPool:
+    B, H, d, g = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.group_size
+    i32 = dict(dtype=torch.int32, device=device)
+    return WarmPool(
+        k=torch.zeros(B, H, n_slots, g, d, dtype=cfg.torch_dtype(), device=device),
+        v=torch.zeros(B, H, n_slots, g, d, dtype=cfg.torch_dtype(), device=device),
+        tag=torch.full((B, H, n_slots), -1, **i32), last=torch.full((B, H, n_slots), -1, **i32),
+        src=torch.empty(B, H, cfg.top_k_groups, **i32), stats=torch.zeros(B, H, 2, **i32))
+
+
 def alloc_summaries(cfg: hga.HgaConfig, device="cuda"):
     B, H, d, nC, G = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.n_chunks, cfg.groups_per_chunk
     cs = torch.empty(B, H, nC, d, dtype=torch.float32, device=device)
@@ -96,7 +119,7 @@ def prefill(cfg: hga.HgaConfig, k_raw, v, q_rot, cs, gs, k_rot, rb: RouteBuffers
 
 def decode(cfg: hga.HgaConfig, q_rot, cs, gs, k_res, v_res, rb: RouteBuffers, out,
            gathered=None, k_src=None, v_src=None, src_is_host=False, stream=None,
-           separate: bool = False):
+           separate: bool = False, warm: Optional[WarmPool] = None):
     """One decode step: routing, optional gather into `gathered` (k, v) from
     k_src/v_src, attention (forced chunks from k_res/v_res). Without a
     gather (full resident cache) this is one hga_decode_step call unless
@@ -106,7 +129,15 @@ def decode(cfg: hga.HgaConfig, q_rot, cs, gs, k_res, v_res, rb: RouteBuffers, ou
                         rb.n_sel_chunks, rb.sel_groups, rb.n_sel_groups, out, stream)
         return
     route(cfg, q_rot, cs, gs, rb, stream, separate=separate)
-    if gathered is not None:
+    if gathered is not None and warm is not None:
+        # host store behind the VRAM warm tier: only pool misses cross the link
+        hga.gather_kv_warm(cfg, k_src, v_src, rb.sel_groups, rb.n_sel_groups, warm.k, warm.v,
+                           warm.tag, warm.last, warm.step, warm.src, gathered[0], gathered[1],
+                           warm.stats, stream)
+        warm.step += 1
+        hga.attend(cfg, q_rot, k_res, v_res, rb.sel_groups, rb.n_sel_groups, out,
+                   k_gat=gathered[0], v_gat=gathered[1], stream=stream)
+    elif gathered is not None:
         hga.gather_kv(cfg, k_src, v_src, src_is_host, rb.sel_groups, rb.n_sel_groups,
                       gathered[0], gathered[1], stream)
         hga.attend(cfg, q_rot, k_res, v_res, rb.sel_groups, rb.n_sel_groups, out,

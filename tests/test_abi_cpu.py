@@ -81,3 +81,13 @@ def test_host_validation_without_gpu(hga):
                              None) == -8
     assert L.hga_decode_step(by(_cfg(hga, q_len=0)), P, P, P, P, P, P, P, P, P, P, P,
                              None) == 0  # empty span
+    # hga_gather_kv_warm: decode only, pool at least top_k_groups slots
+    dec = _cfg(hga, q_begin=4095, q_len=1)
+    assert L.hga_gather_kv_warm(by(dec), P, P, P, P, P, P, P, None, 128, 0, P, None, P, P,
+                                None) == -1
+    assert L.hga_gather_kv_warm(by(_cfg(hga)), P, P, P, P, P, P, P, P, 128, 0, P, None, P, P,
+                                None) == -8
+    assert L.hga_gather_kv_warm(by(dec), P, P, P, P, P, P, P, P, 64, 0, P, None, P, P,
+                                None) == -2
+    assert L.hga_gather_kv_warm(by(dec), P, P, P, P, P, P, P, P, 128, 0, P, P + 4, P, P,
+                                None) == -3
