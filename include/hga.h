@@ -68,7 +68,8 @@ typedef enum {
     HGA_ERR_DEVICE_INDEX = -6, /* a kernel met an invalid entry in a caller-supplied list */
     HGA_ERR_TIMEOUT = -7,      /* a bounded device-side wait gave up */
     HGA_ERR_UNSUPPORTED = -8,  /* valid arguments, combination not implemented */
-    HGA_ERR_MEMORY = -9        /* a pointer is not in the memory space the call needs */
+    HGA_ERR_MEMORY = -9,       /* a pointer is not in the memory space the call needs */
+    HGA_ERR_SCRATCH_LIMIT = -10 /* larger than the library's fixed scratch array */
 } hga_status;
 
 typedef enum { HGA_BF16 = 0, HGA_F32 = 1 } hga_dtype;
@@ -215,6 +216,33 @@ hga_status hga_gather_kv_warm(const hga_config* cfg, const void* k_host, const v
                               void* pool_k, void* pool_v, int32_t* pool_tag, int32_t* pool_last,
                               int32_t n_slots, int32_t step, int32_t* src_out,
                               int32_t* stats_out, void* k_dst, void* v_dst, void* stream);
+
+/* hga_gather_kv_warm without a caller scratch buffer. The pages have no
+ * counterpart of this call: it exists for callers that may not allocate
+ * device memory, e.g. a serving engine that reserves nearly all of HBM for
+ * its KV pools at start-up and hands out only fixed buffers, or a decode loop
+ * that cannot afford the device-wide synchronisation cudaFree implies. Same
+ * arguments and results as hga_gather_kv_warm minus src_out: the per-selection
+ * source list that the plan kernel hands to the copy kernel lives in a static
+ * device array of 65536 int32 (256 KiB) inside the library, which every GPU
+ * that loads the library holds until the process exits. The call allocates
+ * nothing (no cudaMalloc, no allocating library routine).
+ *   - HGA_ERR_SCRATCH_LIMIT if batch * n_kv_heads * top_k_groups > 65536.
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress (that device current) before enqueueing anything;
+ *     make that first call before any stream capture.
+ *   - Nothing in the array needs a starting value: each call writes every
+ *     entry it reads before reading it. The array keeps the last call's
+ *     contents.
+ *   - All calls on a device share the one array: calls that overlap on the
+ *     GPU (unordered streams, or several host threads) race and corrupt each
+ *     other's results. Order them, e.g. on one stream. */
+hga_status hga_gather_kv_warm_noalloc(const hga_config* cfg, const void* k_host,
+                                      const void* v_host, const int32_t* sel_groups,
+                                      const int32_t* n_sel_groups, void* pool_k, void* pool_v,
+                                      int32_t* pool_tag, int32_t* pool_last, int32_t n_slots,
+                                      int32_t step, int32_t* stats_out, void* k_dst, void* v_dst,
+                                      void* stream);
 
 /* Exact softmax attention over the bounded set ("Kernmechanisme" item 4):
  * for each query token at position p in chunk j and each query head, softmax

@@ -34,6 +34,33 @@ hga_status error_word(int** out) {
     return HGA_OK;
 }
 
+// Scratch of hga_gather_kv_warm_noalloc: the source list that the warm
+// tier's plan kernel writes and its copy kernel reads, one int32 per
+// (sequence, KV head, selection slot). 65536 entries (256 KiB), held by every
+// GPU that loads the library until exit. Each call writes every entry it
+// reads first, so nothing here needs a starting value. In host code the name
+// g_warm_scratch is only a handle for the runtime, never a pointer to give a
+// kernel: warm_scratch() returns the device address.
+constexpr int64_t kWarmScratchEntries = 65536;
+static __device__ __align__(256) int32_t g_warm_scratch[kWarmScratchEntries];
+int32_t* g_warm_scratch_addr[kMaxDevices] = {};
+std::mutex g_scratch_mutex;
+
+// Device address of g_warm_scratch on the current device (looked up once per
+// device, with that device current).
+hga_status warm_scratch(int32_t** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HGA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_warm_scratch_addr[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_warm_scratch) != cudaSuccess) return HGA_ERR_CUDA;
+        g_warm_scratch_addr[dev] = static_cast<int32_t*>(ptr);
+    }
+    *out = g_warm_scratch_addr[dev];
+    return HGA_OK;
+}
+
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
 // Checks shared by every call; fills p.
@@ -127,6 +154,8 @@ const char* hga_status_string(hga_status s) {
         case HGA_ERR_TIMEOUT: return "HGA_ERR_TIMEOUT: a bounded device wait gave up";
         case HGA_ERR_UNSUPPORTED: return "HGA_ERR_UNSUPPORTED: combination not implemented";
         case HGA_ERR_MEMORY: return "HGA_ERR_MEMORY: pointer not in the required memory space";
+        case HGA_ERR_SCRATCH_LIMIT:
+            return "HGA_ERR_SCRATCH_LIMIT: larger than the library's fixed scratch array";
     }
     return "HGA_ERR_UNKNOWN";
 }
@@ -349,6 +378,40 @@ hga_status hga_gather_kv_warm(const hga_config* cfg, const void* k_host, const v
     return launched(launch_gather_warm(p, kd, vd, sel_groups, n_sel_groups, pool_k, pool_v,
                                        pool_tag, pool_last, n_slots, step, src_out, stats_out,
                                        k_dst, v_dst, (cudaStream_t)stream));
+}
+
+hga_status hga_gather_kv_warm_noalloc(const hga_config* cfg, const void* k_host,
+                                      const void* v_host, const int32_t* sel_groups,
+                                      const int32_t* n_sel_groups, void* pool_k, void* pool_v,
+                                      int32_t* pool_tag, int32_t* pool_last, int32_t n_slots,
+                                      int32_t step, int32_t* stats_out, void* k_dst, void* v_dst,
+                                      void* stream) {
+    Params p;
+    hga_status s = make_params(cfg, &p);
+    if (s != HGA_OK) return s;
+    if (p.nQC == 0) return HGA_OK;
+    if (!k_host || !v_host || !sel_groups || !n_sel_groups || !pool_k || !pool_v || !pool_tag ||
+        !pool_last || !k_dst || !v_dst)
+        return HGA_ERR_NULL;
+    if (!aligned16(k_host) || !aligned16(v_host) || !aligned16(sel_groups) ||
+        !aligned16(n_sel_groups) || !aligned16(pool_k) || !aligned16(pool_v) ||
+        !aligned16(pool_tag) || !aligned16(pool_last) || !aligned16(k_dst) ||
+        !aligned16(v_dst) || (stats_out && !aligned16(stats_out)))
+        return HGA_ERR_ALIGN;
+    if (p.q_len != 1) return HGA_ERR_UNSUPPORTED;
+    if (n_slots < p.kg || step < 0) return HGA_ERR_SHAPE;
+    if (!gather_warm_supports(p, n_slots)) return HGA_ERR_UNSUPPORTED;
+    if ((int64_t)p.B * p.Hkv * p.kg > kWarmScratchEntries) return HGA_ERR_SCRATCH_LIMIT;
+    int32_t* src = nullptr;
+    if ((s = warm_scratch(&src)) != HGA_OK) return s;
+    HGA_ATTACH_ERR(p);
+    const void* kd = nullptr;
+    const void* vd = nullptr;
+    if ((s = device_view(k_host, true, &kd)) != HGA_OK) return s;
+    if ((s = device_view(v_host, true, &vd)) != HGA_OK) return s;
+    return launched(launch_gather_warm(p, kd, vd, sel_groups, n_sel_groups, pool_k, pool_v,
+                                       pool_tag, pool_last, n_slots, step, src, stats_out, k_dst,
+                                       v_dst, (cudaStream_t)stream));
 }
 
 hga_status hga_attend(const hga_config* cfg, const void* q_rot, const void* k_res,

@@ -24,7 +24,8 @@ HGA_BF16, HGA_F32 = 0, 1
 HGA_KV_FULL, HGA_KV_WINDOWS = 0, 1
 STATUS = {0: "HGA_OK", -1: "HGA_ERR_NULL", -2: "HGA_ERR_SHAPE", -3: "HGA_ERR_ALIGN",
           -4: "HGA_ERR_CONFIG", -5: "HGA_ERR_CUDA", -6: "HGA_ERR_DEVICE_INDEX",
-          -7: "HGA_ERR_TIMEOUT", -8: "HGA_ERR_UNSUPPORTED", -9: "HGA_ERR_MEMORY"}
+          -7: "HGA_ERR_TIMEOUT", -8: "HGA_ERR_UNSUPPORTED", -9: "HGA_ERR_MEMORY",
+          -10: "HGA_ERR_SCRATCH_LIMIT"}
 
 
 class HgaError(RuntimeError):
@@ -84,6 +85,7 @@ def _load():
         "hga_route": [C, P, P, P, P, P, P, P, P, P],
         "hga_decode_step": [C, P, P, P, P, P, P, P, P, P, P, P, P],
         "hga_gather_kv_warm": [C, P, P, P, P, P, P, P, P, I32, I32, P, P, P, P, P],
+        "hga_gather_kv_warm_noalloc": [C, P, P, P, P, P, P, P, P, I32, I32, P, P, P, P],
         "hga_get_device_error": [P, ctypes.POINTER(I32)],
     }
     for name, args in sig.items():
@@ -276,6 +278,31 @@ def gather_kv_warm(cfg: HgaConfig, k_host, v_host, sel_groups, n_sel_groups, poo
         _ptr(stats, "stats", torch.int32, (B, H, 2), nullable=True),
         _ptr(k_dst, "k_dst", dt, gat_shape), _ptr(v_dst, "v_dst", dt, gat_shape),
         _stream(stream)), "hga_gather_kv_warm")
+
+
+def gather_kv_warm_noalloc(cfg: HgaConfig, k_host, v_host, sel_groups, n_sel_groups, pool_k,
+                           pool_v, pool_tag, pool_last, step: int, k_dst, v_dst, stats=None,
+                           stream=None) -> None:
+    """gather_kv_warm for callers that may not allocate device memory: the
+    plan-to-copy source list lives in the library's fixed scratch array
+    (see hga_gather_kv_warm_noalloc). Allocates nothing itself either."""
+    B, H, d, kg, g = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.top_k_groups, cfg.group_size
+    dt = cfg.torch_dtype()
+    n_slots = pool_tag.shape[-1]
+    store = (B, H, cfg.seq_len, d)
+    gat_shape = (B, H, cfg.n_qchunks, kg * g, d)
+    _check(_lib.hga_gather_kv_warm_noalloc(
+        ctypes.byref(cfg), _ptr(k_host, "k_host", dt, store, device=False),
+        _ptr(v_host, "v_host", dt, store, device=False),
+        _ptr(sel_groups, "sel_groups", torch.int32, (B, H, cfg.n_qchunks, kg)),
+        _ptr(n_sel_groups, "n_sel_groups", torch.int32, (B, H, cfg.n_qchunks)),
+        _ptr(pool_k, "pool_k", dt, (B, H, n_slots, g, d)),
+        _ptr(pool_v, "pool_v", dt, (B, H, n_slots, g, d)),
+        _ptr(pool_tag, "pool_tag", torch.int32, (B, H, n_slots)),
+        _ptr(pool_last, "pool_last", torch.int32, (B, H, n_slots)), n_slots, step,
+        _ptr(stats, "stats", torch.int32, (B, H, 2), nullable=True),
+        _ptr(k_dst, "k_dst", dt, gat_shape), _ptr(v_dst, "v_dst", dt, gat_shape),
+        _stream(stream)), "hga_gather_kv_warm_noalloc")
 
 
 def window_slots(cfg: HgaConfig) -> int:
