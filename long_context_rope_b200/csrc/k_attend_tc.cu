@@ -259,8 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             float sx[kTileKeys];
             {
                 uint32_t* xr = reinterpret_cast<uint32_t*>(sx);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) ptx::tmem_ld32(s_addr + 32 * c, xr + 32 * c);
+                ptx::tmem_ld64(s_addr, xr);
+                ptx::tmem_ld64(s_addr + 64, xr + 64);
                 ptx::tmem_wait_ld();
                 ptx::reg_fence<kTileKeys>(xr);
             }
@@ -283,8 +283,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                     }
                 }
             } else {
+                // four independent three-input chains
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int c = 0; c < kTileKeys; ++c) mraw = fmaxf(mraw, sx[c]);
+                for (int c = 0; c < kTileKeys; c += 8) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) m4[u] = ptx::fmax3(m4[u], sx[c + 2 * u], sx[c + 2 * u + 1]);
+                }
+                mraw = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             }
             const float m_new = fmaxf(m_used, mraw * sc);
             bool rescale = false;
@@ -300,17 +306,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             }
             // P = 2^(S*sc - m), rounded to bf16; the row sum uses the rounded values
             uint32_t pk[kTileKeys / 2];
-            float lsum = 0.f;
+            float lsum0 = 0.f, lsum1 = 0.f;
             const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
 #pragma unroll
             for (int c = 0; c < kTileKeys; c += 2) {
-                const float p0 = ptx::ex2_approx(fmaf(sx[c], sc, neg_m));
-                const float p1 = ptx::ex2_approx(fmaf(sx[c + 1], sc, neg_m));
+                float a0, a1;
+                ptx::fma2_bc(sx[c], sx[c + 1], sc, neg_m, a0, a1);
+                const float p0 = ptx::ex2_approx(a0);
+                const float p1 = ptx::ex2_approx(a1);
                 __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-                const float2 f2 = __bfloat1622float2(b2);
-                lsum += f2.x + f2.y;
                 pk[c / 2] = *reinterpret_cast<uint32_t*>(&b2);
+                ptx::add_bf16x2_f32(pk[c / 2], lsum0, lsum1);
             }
+            const float lsum = lsum0 + lsum1;
             // tcgen05.ld/st are warp-collective: the whole warp rescales its
             // rows when any row needs it (rows that do not use alpha = 1).
             // PV of the previous tile has completed: S of this tile was issued
