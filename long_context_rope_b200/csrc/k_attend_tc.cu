@@ -63,6 +63,7 @@ struct TcSmem {
     int abort;
     int blk_row[kMaxBlocks];
     int blk_pos[kMaxBlocks];
+    int tile_last[kMaxBlocks / kBlocksPerTile];  // last key position of a tile, INT_MAX if partial
 };
 
 // Bounded wait shared by the roles of one CTA: gives up after the time limit,
@@ -149,6 +150,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         const int nb_w = build_key_blocks_warp(p, j, sel + prob * p.kg, nsel + prob, false,
                                                sm.blk_row, sm.blk_pos);
         if (lane == 0) sm.nb = nb_w;
+        __syncwarp();
+        for (int t = lane; t * kBlocksPerTile < nb_w; t += 32) {
+            int last = 0;
+#pragma unroll
+            for (int i = 0; i < kBlocksPerTile; ++i) {
+                const int blk = t * kBlocksPerTile + i;
+                last = blk < nb_w ? max(last, sm.blk_pos[blk] + kGroupRows - 1) : INT_MAX;
+            }
+            sm.tile_last[t] = last;
+        }
     } else if (warp == 1) {
         ptx::tmem_alloc(&sm.tmem_base, kTmemCols);
         ptx::tmem_relinquish();
@@ -266,10 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             }
             // mask (causal within the current chunk; padding past the set)
             const int blk0 = t * kBlocksPerTile;
-            bool need_mask = blk0 + kBlocksPerTile > nb;
-#pragma unroll
-            for (int i = 0; i < kBlocksPerTile; ++i)
-                need_mask |= (blk0 + i < nb) && (sm.blk_pos[blk0 + i] + kGroupRows - 1 > tokx);
+            const bool need_mask = sm.tile_last[t] > tokx;
             float mraw = -INFINITY;
             if (need_mask) {
 #pragma unroll

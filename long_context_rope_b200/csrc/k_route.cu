@@ -300,6 +300,86 @@ __global__ void __launch_bounds__(256) route_groups_kernel(
     if (lane == 0) n_sel_groups[prob] = kept;
 }
 
+// Level 2 when every query chunk has at most 256 candidate groups
+// (top_k_chunks * G <= 256): grid (nQC, B*Hkv), 128 threads. A warp takes
+// one selected chunk at a time and reads its G group rows (contiguous in the
+// table) with coalesced 16-byte loads; lane L holds dims L*DPL.. of every
+// row, so each score is the same per-lane partial dot product and butterfly
+// sum as in route_groups_kernel and the decode step (bitwise identical
+// scores and selections). Warp 0 then selects.
+template <int DPL>
+__global__ void __launch_bounds__(128) route_groups_small_kernel(
+    Params p, const float* __restrict__ qbar, const float* __restrict__ gs,
+    const int32_t* __restrict__ sel_chunks, const int32_t* __restrict__ n_sel_chunks,
+    int32_t* __restrict__ sel_groups, int32_t* __restrict__ n_sel_groups,
+    float* __restrict__ scores) {
+    constexpr int kMaxCand = 256;
+    __shared__ uint32_t keys[kMaxCand];
+    __shared__ uint32_t hist[256];
+    __shared__ int s_chunk[kMaxCand];
+    const int jj = blockIdx.x;
+    const int64_t bh = blockIdx.y;
+    const int j = p.j0 + jj;
+    const int64_t prob = bh * p.nQC + jj;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+
+    int n = n_sel_chunks[prob];
+    if (n < 0 || n > p.kc) {
+        if (t == 0) raise_dev_error(p, kDevErrCount);
+        n = n < 0 ? 0 : p.kc;
+    }
+    const int32_t* sc_in = sel_chunks + prob * p.kc;
+    for (int s = t; s < n; s += blockDim.x) {
+        const int c = sc_in[s];
+        const bool ok = c >= 0 && c < j && !is_forced(p, j, c) && (s == 0 || c > sc_in[s - 1]);
+        s_chunk[s] = ok ? c : -1;
+        if (!ok) raise_dev_error(p, kDevErrChunkIndex);
+    }
+    float q[DPL];
+    {
+        const float* qr = qbar + prob * p.d;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) q[e] = qr[lane * DPL + e];
+    }
+    __syncthreads();
+
+    const int G = p.G;
+    const float* table = gs + bh * (int64_t)p.nC * G * p.d;
+    for (int s = warp; s < n; s += 4) {
+        const int c = s_chunk[s];
+        const float* rows = table + (int64_t)(c < 0 ? 0 : c) * G * p.d;
+        float v[8][DPL];
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+            if (g < G) load_row<DPL>(rows + (int64_t)g * p.d, lane, v[g]);
+        float sc = 0.f;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            if (g < G) {
+                float a = 0.f;
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) a = fmaf(q[e], v[g][e], a);
+                a = warp_sum(a);
+                if (lane == g) sc = a;
+            }
+        }
+        if (lane < G) {
+            const int x = s * G + lane;
+            keys[x] = c < 0 ? 0u : score_key32(sc);
+            if (scores) scores[prob * p.kc * G + x] = c < 0 ? __int_as_float(0x7fc00000) : sc;
+        }
+    }
+    const int ncand = n * G;
+    if (scores)
+        for (int x = ncand + t; x < p.kc * G; x += blockDim.x)
+            scores[prob * p.kc * G + x] = __int_as_float(0x7fc00000);
+    __syncthreads();
+    if (warp != 0) return;
+    const int kept = warp_radix_topk(keys, ncand, p.kg, p.kg, sel_groups + prob * p.kg, hist,
+                                     [&](int x) { return s_chunk[x / G] * G + x % G; });
+    if (lane == 0) n_sel_groups[prob] = kept;
+}
+
 // Raise a kernel's dynamic shared-memory limit once per process (a driver
 // call per launch would add host latency to every decode step).
 cudaError_t allow_smem(const void* fn, size_t bytes) {
@@ -382,6 +462,16 @@ cudaError_t launch_route_groups(const Params& p, const float* qbar, const float*
                                 int32_t* sel_groups, int32_t* n_sel_groups, float* scores,
                                 cudaStream_t st) {
     if (p.nQC == 0) return cudaSuccess;
+    if (p.kc * p.G <= 256) {
+        const dim3 grid(p.nQC, p.B * p.Hkv);
+        if (p.d == 128)
+            route_groups_small_kernel<4><<<grid, 128, 0, st>>>(
+                p, qbar, group_sum, sel_chunks, n_sel_chunks, sel_groups, n_sel_groups, scores);
+        else
+            route_groups_small_kernel<2><<<grid, 128, 0, st>>>(
+                p, qbar, group_sum, sel_chunks, n_sel_chunks, sel_groups, n_sel_groups, scores);
+        return cudaGetLastError();
+    }
     const int64_t problems = (int64_t)p.B * p.Hkv * p.nQC;
     const int cl = problems >= 1024 ? 1 : 4;
     size_t smem = ((size_t)p.kc * p.G + 256) * sizeof(uint32_t);

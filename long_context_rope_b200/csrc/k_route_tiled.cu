@@ -6,13 +6,16 @@
 // top-k; sink, local and current chunks are always visible and never routed.
 //
 // In prefill all query chunks of one (sequence, KV head) score the same
-// table, so a CTA takes 16 query chunks and streams the table through shared
-// memory once for all of them: a register-blocked fp32 product (each thread
-// 4 query chunks x 4 table rows) writes the 16 score rows to shared memory.
-// Each warp then selects the top-k of its query chunks with a 4-pass radix
-// select over the order-preserving score keys (hga_topk.cuh) and writes the
-// winners in ascending chunk order. Ties go to the lower chunk index; NaN
-// ranks last.
+// table, so a CTA takes 8 query chunks and streams the table through shared
+// memory once for all of them: a register-blocked fp32 product (each of 256
+// threads 4 query chunks x 2 table rows), with the next table slice loaded
+// into registers while the current one is multiplied, writes the 8 score
+// rows to shared memory. Each of the 8 warps then selects the top-k of one
+// query chunk with a 4-pass radix select over the order-preserving score
+// keys (hga_topk.cuh) and writes the winners in ascending chunk order. Ties
+// go to the lower chunk index; NaN ranks last. Work grows with the query
+// chunk index (more earlier chunks to score), so CTAs take the last query
+// chunks first and the block scheduler fills in with the short ones.
 #include "hga_kernels.h"
 #include "hga_topk.cuh"
 
@@ -20,13 +23,17 @@ namespace hga {
 
 namespace {
 
-constexpr int kQB = 16;          // query chunks per CTA
+constexpr int kQB = 8;           // query chunks per CTA (one selecting warp each)
 constexpr int kCT = 256;         // table rows per tile
 constexpr int kKS = 32;          // dims per k-slice
 constexpr int kThreads = 256;
+constexpr int kRowV = kKS / 4;   // float4 per thread per slice (one row)
+static_assert(kThreads == kCT, "one loading thread per tile row");
+static_assert(kThreads / 32 == kQB, "one warp per query chunk");
+static_assert(kThreads / 32 * 256 <= kKS * kCT, "histograms fit in the tile buffer");
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) route_chunks_tiled_kernel(
+__global__ void __launch_bounds__(kThreads, 3) route_chunks_tiled_kernel(
     Params p, const float* __restrict__ qbar, const float* __restrict__ cs,
     int32_t* __restrict__ sel, int32_t* __restrict__ nsel, float* __restrict__ scores_out) {
     extern __shared__ __align__(16) float smem_f[];
@@ -34,11 +41,11 @@ __global__ void __launch_bounds__(kThreads) route_chunks_tiled_kernel(
     float* tile = qT + D * kQB;                 // [kKS][kCT] transposed table slice
     float* sc = tile + kKS * kCT;               // [kQB][ncp] scores
     const int ncp = (p.nC + 3) & ~3;
-    uint32_t* hist = reinterpret_cast<uint32_t*>(sc + kQB * ncp);  // [8 warps][256]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(tile);  // [8 warps][256], after the products
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t bh = blockIdx.y;
-    const int jj0 = blockIdx.x * kQB;
+    const int jj0 = (gridDim.x - 1 - blockIdx.x) * kQB;  // longest first
     const int nq = p.nQC - jj0 < kQB ? p.nQC - jj0 : kQB;
     const int j_hi = p.j0 + jj0 + nq;           // chunks [0, j_hi - 1) are candidates at most
 
@@ -47,56 +54,67 @@ __global__ void __launch_bounds__(kThreads) route_chunks_tiled_kernel(
         qT[x] = q < nq ? qbar[((bh * p.nQC) + jj0 + q) * D + k] : 0.f;
     }
     const float* table = cs + bh * (int64_t)p.nC * D;
-    const int qg = tid & 3;                     // query group: queries 4*qg .. 4*qg+3
-    const int cg = tid >> 2;                    // table group: rows 4*cg .. 4*cg+3 of the tile
-    for (int c0 = 0; c0 < j_hi - 1; c0 += kCT) {
-        float acc[4][4];
+    const int qg = tid & 1;                     // query group: queries 4*qg .. 4*qg+3
+    const int cg = tid >> 1;                    // rows 2*cg, 2*cg+1 of the tile
+    const int lr = tid;                         // loader: tile row
+    constexpr int kSlices = D / kKS;
+    const int n_steps = ((j_hi - 1 + kCT - 1) / kCT) * kSlices;
+    float4 pf[kRowV];
+    auto load = [&](int step) {
+        const int c = (step / kSlices) * kCT + lr;
+        const int k0 = (step % kSlices) * kKS;
+        const bool in = c < p.nC;
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int v = 0; v < kRowV; ++v)
+            pf[v] = in ? __ldg(reinterpret_cast<const float4*>(table + (int64_t)c * D + k0) + v)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    if (n_steps > 0) load(0);
+    float acc[4][2];
+    for (int step = 0; step < n_steps; ++step) {
+        const int ks = step % kSlices;
+        const int c0 = (step / kSlices) * kCT, k0 = ks * kKS;
+        if (ks == 0) {
 #pragma unroll
-            for (int bb = 0; bb < 4; ++bb) acc[a][bb] = 0.f;
-        for (int k0 = 0; k0 < D; k0 += kKS) {
-            __syncthreads();
-            {
-                // row c0 + tid of the table, dims k0 .. k0 + kKS, written transposed
-                const int c = c0 + tid;
-                const bool in = c < p.nC;
+            for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = 0.f;
+        }
+        __syncthreads();  // the previous slice is no longer read
 #pragma unroll
-                for (int v = 0; v < kKS / 4; ++v) {
-                    float4 t = in ? __ldg(reinterpret_cast<const float4*>(table + (int64_t)c * D + k0) + v)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-                    tile[(4 * v + 0) * kCT + tid] = t.x;
-                    tile[(4 * v + 1) * kCT + tid] = t.y;
-                    tile[(4 * v + 2) * kCT + tid] = t.z;
-                    tile[(4 * v + 3) * kCT + tid] = t.w;
-                }
-            }
-            __syncthreads();
+        for (int v = 0; v < kRowV; ++v) {
+            const int kr = 4 * v;
+            tile[(kr + 0) * kCT + lr] = pf[v].x;
+            tile[(kr + 1) * kCT + lr] = pf[v].y;
+            tile[(kr + 2) * kCT + lr] = pf[v].z;
+            tile[(kr + 3) * kCT + lr] = pf[v].w;
+        }
+        __syncthreads();
+        if (step + 1 < n_steps) load(step + 1);  // lands while this slice is multiplied
 #pragma unroll 8
-            for (int k = 0; k < kKS; ++k) {
-                const float4 qv = *reinterpret_cast<const float4*>(qT + (k0 + k) * kQB + 4 * qg);
-                const float4 tv = *reinterpret_cast<const float4*>(tile + k * kCT + 4 * cg);
-                const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
-                const float ta[4] = {tv.x, tv.y, tv.z, tv.w};
+        for (int k = 0; k < kKS; ++k) {
+            const float4 qv = *reinterpret_cast<const float4*>(qT + (k0 + k) * kQB + 4 * qg);
+            const float2 tv = *reinterpret_cast<const float2*>(tile + k * kCT + 2 * cg);
+            const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
-                for (int a = 0; a < 4; ++a)
-#pragma unroll
-                    for (int bb = 0; bb < 4; ++bb) acc[a][bb] = fmaf(qa[a], ta[bb], acc[a][bb]);
+            for (int a = 0; a < 4; ++a) {
+                acc[a][0] = fmaf(qa[a], tv.x, acc[a][0]);
+                acc[a][1] = fmaf(qa[a], tv.y, acc[a][1]);
             }
         }
+        if (ks == kSlices - 1) {
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < 4; ++a)
 #pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                const int c = c0 + 4 * cg + bb;
-                if (c < ncp) sc[(4 * qg + a) * ncp + c] = acc[a][bb];
-            }
+                for (int bb = 0; bb < 2; ++bb) {
+                    const int c = c0 + 2 * cg + bb;
+                    if (c < ncp) sc[(4 * qg + a) * ncp + c] = acc[a][bb];
+                }
+        }
     }
     __syncthreads();
 
     // ---- per query chunk: radix top-k over its candidates (one warp each)
     uint32_t* h = hist + warp * 256;
-    for (int q = warp; q < nq; q += kThreads / 32) {
+    for (int q = warp; q < nq; q += kThreads / 32) {  // one pass: a warp per query chunk
         const int jj = jj0 + q, j = p.j0 + jj;
         const int64_t prob = bh * p.nQC + jj;
         float* srow = sc + q * ncp;
@@ -126,15 +144,13 @@ cudaError_t launch_route_chunks_tiled(const Params& p, const float* qbar, const 
                                       int32_t* sel, int32_t* n_sel, float* scores,
                                       cudaStream_t st) {
     const int ncp = (p.nC + 3) & ~3;
-    const size_t smem = (size_t)(p.d * kQB + kKS * kCT + kQB * ncp) * sizeof(float) +
-                        (size_t)(kThreads / 32) * 256 * sizeof(uint32_t);
+    const size_t smem = (size_t)(p.d * kQB + kKS * kCT + kQB * ncp) * sizeof(float);
     dim3 grid((p.nQC + kQB - 1) / kQB, p.B * p.Hkv);
     const void* fn = p.d == 128 ? (const void*)route_chunks_tiled_kernel<128>
                                 : (const void*)route_chunks_tiled_kernel<64>;
     static bool attr = false;
     if (!attr) {
-        const size_t max_smem = (size_t)(128 * kQB + kKS * kCT + kQB * 2048) * sizeof(float) +
-                                (size_t)(kThreads / 32) * 256 * sizeof(uint32_t);
+        const size_t max_smem = (size_t)(128 * kQB + kKS * kCT + kQB * 2048) * sizeof(float);
         cudaError_t e = cudaFuncSetAttribute(route_chunks_tiled_kernel<128>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)max_smem);

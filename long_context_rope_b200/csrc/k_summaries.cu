@@ -20,6 +20,11 @@ struct Vec;
 template <>
 struct Vec<__nv_bfloat16> {
     static constexpr int N = 8;
+    using Raw = uint4;  // one 16-byte vector as loaded
+    static __device__ __forceinline__ Raw load_raw(const __nv_bfloat16* p) {
+        return __ldg(reinterpret_cast<const uint4*>(p));
+    }
+    static __device__ __forceinline__ void unpack(const Raw& r, float* f) { bf16x8_to_f32(r, f); }
     static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* f) {
         bf16x8_to_f32(*reinterpret_cast<const uint4*>(p), f);
     }
@@ -30,6 +35,13 @@ struct Vec<__nv_bfloat16> {
 template <>
 struct Vec<float> {
     static constexpr int N = 4;
+    using Raw = float4;
+    static __device__ __forceinline__ Raw load_raw(const float* p) {
+        return __ldg(reinterpret_cast<const float4*>(p));
+    }
+    static __device__ __forceinline__ void unpack(const Raw& r, float* f) {
+        f[0] = r.x; f[1] = r.y; f[2] = r.z; f[3] = r.w;
+    }
     static __device__ __forceinline__ void load(const float* p, float* f) {
         float4 v = *reinterpret_cast<const float4*>(p);
         f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
@@ -91,14 +103,24 @@ __global__ void summaries_kernel(Params p, const T* __restrict__ k_raw, float* _
 #pragma unroll
     for (int e = 0; e < V; ++e) acc0[e] = acc1[e] = 0.f;
 
+    // every row load of this thread is issued before any arithmetic
+    typename Vec<T>::Raw raw_a[4], raw_b[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int64_t t = c0 + 16 * k + 4 * s + m;
+        if (t < p.L) {
+            const T* row = base + t * p.d;
+            raw_a[m] = Vec<T>::load_raw(row + u * V);
+            raw_b[m] = Vec<T>::load_raw(row + half + u * V);
+        }
+    }
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
         int64_t t = c0 + 16 * k + 4 * s + m;
         if (t < p.L) {
             float a[V], b[V], ra[V], rb[V];
-            const T* row = base + t * p.d;
-            Vec<T>::load(row + u * V, a);
-            Vec<T>::load(row + half + u * V, b);
+            Vec<T>::unpack(raw_a[m], a);
+            Vec<T>::unpack(raw_b[m], b);
 #pragma unroll
             for (int e = 0; e < V; ++e) {
                 const int i = u * V + e;
