@@ -27,8 +27,8 @@ constexpr int kQB = 8;           // query chunks per CTA (one selecting warp eac
 constexpr int kCT = 256;         // table rows per tile
 constexpr int kKS = 32;          // dims per k-slice
 constexpr int kThreads = 256;
-constexpr int kRowV = kKS / 4;   // float4 per thread per slice (one row)
-static_assert(kThreads == kCT, "one loading thread per tile row");
+constexpr int kPerThread = kCT * kKS / 4 / kThreads;  // float4 per thread per slice
+static_assert(kKS == 32 && kCT % 32 == 0, "a slice row is 8 float4, rows come in warps of 4");
 static_assert(kThreads / 32 == kQB, "one warp per query chunk");
 static_assert(kThreads / 32 * 256 <= kKS * kCT, "histograms fit in the tile buffer");
 
@@ -56,18 +56,24 @@ __global__ void __launch_bounds__(kThreads, 3) route_chunks_tiled_kernel(
     const float* table = cs + bh * (int64_t)p.nC * D;
     const int qg = tid & 1;                     // query group: queries 4*qg .. 4*qg+3
     const int cg = tid >> 1;                    // rows 2*cg, 2*cg+1 of the tile
-    const int lr = tid;                         // loader: tile row
+    // Loader: float4 e = tid + kThreads * v of the slice is row e / 8, dims
+    // 4 * (e % 8) ..; a warp reads 4 whole 128-byte slice rows. The
+    // transposed tile stores row r of dim kk at column r ^ (4 * (kk / 4 % 8)),
+    // so those stores hit 32 distinct banks; the XOR keeps 2 * cg and
+    // 2 * cg + 1 adjacent for the float2 reads of the product.
     constexpr int kSlices = D / kKS;
     const int n_steps = ((j_hi - 1 + kCT - 1) / kCT) * kSlices;
-    float4 pf[kRowV];
+    float4 pf[kPerThread];
     auto load = [&](int step) {
-        const int c = (step / kSlices) * kCT + lr;
         const int k0 = (step % kSlices) * kKS;
-        const bool in = c < p.nC;
 #pragma unroll
-        for (int v = 0; v < kRowV; ++v)
-            pf[v] = in ? __ldg(reinterpret_cast<const float4*>(table + (int64_t)c * D + k0) + v)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int v = 0; v < kPerThread; ++v) {
+            const int e = tid + kThreads * v;
+            const int c = (step / kSlices) * kCT + (e >> 3);
+            pf[v] = c < p.nC ? __ldg(reinterpret_cast<const float4*>(table + (int64_t)c * D + k0) +
+                                     (e & 7))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     };
     if (n_steps > 0) load(0);
     float acc[4][2];
@@ -80,19 +86,21 @@ __global__ void __launch_bounds__(kThreads, 3) route_chunks_tiled_kernel(
         }
         __syncthreads();  // the previous slice is no longer read
 #pragma unroll
-        for (int v = 0; v < kRowV; ++v) {
-            const int kr = 4 * v;
-            tile[(kr + 0) * kCT + lr] = pf[v].x;
-            tile[(kr + 1) * kCT + lr] = pf[v].y;
-            tile[(kr + 2) * kCT + lr] = pf[v].z;
-            tile[(kr + 3) * kCT + lr] = pf[v].w;
+        for (int v = 0; v < kPerThread; ++v) {
+            const int e = tid + kThreads * v;
+            const int ch = e & 7, col = (e >> 3) ^ (ch << 2);
+            tile[(4 * ch + 0) * kCT + col] = pf[v].x;
+            tile[(4 * ch + 1) * kCT + col] = pf[v].y;
+            tile[(4 * ch + 2) * kCT + col] = pf[v].z;
+            tile[(4 * ch + 3) * kCT + col] = pf[v].w;
         }
         __syncthreads();
         if (step + 1 < n_steps) load(step + 1);  // lands while this slice is multiplied
 #pragma unroll 8
         for (int k = 0; k < kKS; ++k) {
             const float4 qv = *reinterpret_cast<const float4*>(qT + (k0 + k) * kQB + 4 * qg);
-            const float2 tv = *reinterpret_cast<const float2*>(tile + k * kCT + 2 * cg);
+            const float2 tv =
+                *reinterpret_cast<const float2*>(tile + k * kCT + ((2 * cg) ^ (((k >> 2) & 7) << 2)));
             const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
