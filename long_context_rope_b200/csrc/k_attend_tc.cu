@@ -19,7 +19,8 @@
 //               masks (causal / padding), keeps a lazily rescaled running max
 //               (O is rescaled in TMEM only when the max grows by > 2^8),
 //               writes P = 2^(S - max) as bf16 back into TMEM over its S row,
-//               and at the end normalises O and stores the output.
+//               and at the end normalises O and writes the output rows into
+//               the tile's (then idle) Q buffer, from where TMA stores them.
 // TMEM: S_A | S_B | O_A | O_B (128 columns each); P_X lives in the first 64
 // columns of S_X and feeds the PV MMA directly from TMEM. The key set comes
 // in arbitrary group order (forced chunks, then routed groups), so each
@@ -49,7 +50,7 @@ __host__ __device__ constexpr uint32_t col_s(int x) { return (uint32_t)(x * 128)
 __host__ __device__ constexpr uint32_t col_o(int x) { return (uint32_t)(256 + x * 128); }
 
 struct TcMaps {
-    CUtensorMap q, k, v;
+    CUtensorMap q, k, v, o;  // o: the output, same geometry as q
 };
 
 struct TcSmem {
@@ -57,7 +58,7 @@ struct TcSmem {
     alignas(1024) uint8_t k[2][kTile];
     alignas(1024) uint8_t v[2][kTile];
     uint64_t bar_q, k_full[2], k_empty[2], v_full[2], v_empty[2];
-    uint64_t s_full[2], p_full[2], o_done[2], drain;
+    uint64_t s_full[2], p_full[2], o_done[2], st_ready[2], drain;
     uint32_t tmem_base;
     int nb;
     int abort;
@@ -137,6 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                 ptx::mbar_init(&sm.s_full[s], 1);
                 ptx::mbar_init(&sm.p_full[s], 4);
                 ptx::mbar_init(&sm.o_done[s], 1);
+                ptx::mbar_init(&sm.st_ready[s], 4);
             }
             ptx::mbar_init(&sm.drain, 1);
             ptx::fence_mbar_init();
@@ -362,7 +364,34 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             for (int c = 0; c < 4; ++c) ptx::tmem_ld32(o_addr + 32 * c, o + 32 * c);
             ptx::tmem_wait_ld();
             ptx::reg_fence<kD>(o);
-            if (row_ok) {
+            if (tokx >= p.q_begin && tokx + 16 <= span_end) {
+                // Whole M tile in the span: the rows go to the Q buffer of this
+                // tile (its last QK completed before o_done) in the Q map's
+                // swizzled layout, then two TMA stores write them out.
+                uint8_t* stage = sm.q[x];
+#pragma unroll
+                for (int pnl = 0; pnl < 2; ++pnl) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        float f[8];
+#pragma unroll
+                        for (int z = 0; z < 8; ++z) f[z] = __uint_as_float(o[64 * pnl + 8 * c + z]) * inv;
+                        *reinterpret_cast<uint4*>(stage + pnl * kPanel + r * 128 + ((c ^ (r & 7)) << 4)) =
+                            f32x8_to_bf16(f);
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&sm.st_ready[x]);
+                if (q4 == 2 && lane == 0 &&  // one warp of the four issues the stores
+                    wait_bar(&sm.st_ready[x], 0, abort, p.err)) {
+                    const int tq = tokx - p.q_begin;
+                    ptx::tma_store_4d(&maps.o, stage, 0, h * 8, tq, b);
+                    ptx::tma_store_4d(&maps.o, stage + kPanel, 64, h * 8, tq, b);
+                    ptx::bulk_commit();
+                    ptx::bulk_wait_read_all();
+                }
+            } else if (row_ok) {
 #pragma unroll
                 for (int e = 0; e < kD; e += 8) {
                     float f[8];
@@ -401,7 +430,8 @@ cudaError_t launch_attend_tc(const Params& p, const void* q_rot, const KvSources
     const int64_t BH = (int64_t)p.B * p.Hkv;
     bool ok = make_query_map(&maps.q, q_rot, p.B, p.q_len, p.Hq, kD, 8, 16) &&
               make_rows_map(&maps.k, kv.k_res, BH, p.L, kD, kGroupRows) &&
-              make_rows_map(&maps.v, kv.v_res, BH, p.L, kD, kGroupRows);
+              make_rows_map(&maps.v, kv.v_res, BH, p.L, kD, kGroupRows) &&
+              make_query_map(&maps.o, out, p.B, p.q_len, p.Hq, kD, 8, 16);
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = sizeof(TcSmem) + 1024;
     static bool attr_set = false;
