@@ -7,20 +7,27 @@
 // heads per KV head, one (sequence, KV head, query chunk) unit is a real
 // dense contraction: 512 query rows against up to ~1.8K keys.
 //
-// CTA = two M tiles (A, B) of 128 query rows each (16 tokens x 8 heads),
-// sharing every K/V tile; 10 warps:
-//   warp 0      TMA producer: both Q tiles once, then K and V tiles of 128 keys
-//               assembled from 16-row group boxes (two stages each);
+// A persistent CTA per SM walks the units (query-token pair, query chunk,
+// sequence x KV head) u = blockIdx.x, blockIdx.x + gridDim.x, ... Each unit
+// is two M tiles (A, B) of 128 query rows (16 tokens x 8 heads) that share
+// every K/V tile; 11 warps:
+//   warp 10     builds the key-block list of the CTA's next units (double
+//               buffered), so no unit waits for its selection list;
+//   warp 0      TMA producer: a unit's Q tiles as soon as the previous unit's
+//               last QK has completed, then K and V tiles of 128 keys
+//               assembled from 16-row group boxes (two stages each; stages
+//               and barrier phases follow a per-CTA tile counter across units);
 //   warp 1      TMEM owner and MMA issuer. Issue order per key tile t:
 //               PV_A(t), QK_A(t+1), PV_B(t), QK_B(t+1), so the tensor core
-//               works on one M tile while the other's softmax runs;
+//               works on one M tile while the other's softmax runs; the next
+//               unit's first QKs follow the last PVs on the same queue;
 //   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B: each thread
 //               owns one query row (its TMEM lane); it loads its S row,
 //               masks (causal / padding), keeps a lazily rescaled running max
 //               (O is rescaled in TMEM only when the max grows by > 2^8),
 //               writes P = 2^(S - max) as bf16 back into TMEM over its S row,
-//               and at the end normalises O and writes the output rows into
-//               the tile's (then idle) Q buffer, from where TMA stores them.
+//               and at the end of a unit normalises O and writes it out
+//               through a small per-warp staging area as coalesced rows.
 // TMEM: S_A | S_B | O_A | O_B (128 columns each); P_X lives in the first 64
 // columns of S_X and feeds the PV MMA directly from TMEM. The key set comes
 // in arbitrary group order (forced chunks, then routed groups), so each
@@ -42,7 +49,7 @@ constexpr int kTileKeys = 128;             // keys per tile
 constexpr int kBlocksPerTile = kTileKeys / kGroupRows;
 constexpr int kPanel = 128 * 128;          // 128 rows x 128 bytes (64 bf16)
 constexpr int kTile = 2 * kPanel;          // 128 x 128 bf16
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;  // 11 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -50,22 +57,45 @@ __host__ __device__ constexpr uint32_t col_s(int x) { return (uint32_t)(x * 128)
 __host__ __device__ constexpr uint32_t col_o(int x) { return (uint32_t)(256 + x * 128); }
 
 struct TcMaps {
-    CUtensorMap q, k, v, o;  // o: the output, same geometry as q
+    CUtensorMap q, k, v;
 };
 
 struct TcSmem {
     alignas(1024) uint8_t q[2][kTile];
     alignas(1024) uint8_t k[2][kTile];
     alignas(1024) uint8_t v[2][kTile];
-    uint64_t bar_q, k_full[2], k_empty[2], v_full[2], v_empty[2];
-    uint64_t s_full[2], p_full[2], o_done[2], st_ready[2], drain;
+    uint64_t bar_q, q_empty, k_full[2], k_empty[2], v_full[2], v_empty[2];
+    uint64_t s_full[2], p_full[2], o_done[2], list_full[2], list_empty[2], drain;
     uint32_t tmem_base;
-    int nb;
     int abort;
-    int blk_row[kMaxBlocks];
-    int blk_pos[kMaxBlocks];
-    int tile_last[kMaxBlocks / kBlocksPerTile];  // last key position of a tile, INT_MAX if partial
+    int nb[2];                                        // per list buffer
+    int blk_row[2][kMaxBlocks];
+    int blk_pos[2][kMaxBlocks];
+    int tile_last[2][kMaxBlocks / kBlocksPerTile];    // last key position of a tile, INT_MAX if partial
+    alignas(16) uint8_t stage[8][32 * 64];            // per softmax warp: 32 rows x 32 output dims
 };
+
+static_assert(sizeof(TcSmem) + 1024 <= 227 * 1024, "shared memory of one CTA");
+
+// One unit = (query-token pair of M tiles, query chunk, sequence x KV head);
+// false for a pair with no token in the query span.
+struct Unit {
+    int pair, jj, b, h, j, tok0;
+    int64_t bh;
+};
+
+__device__ __forceinline__ bool unit_at(const Params& p, int u, Unit& un) {
+    const int pairs = p.C / 32;
+    un.pair = u % pairs;
+    const int rest = u / pairs;
+    un.jj = rest % p.nQC;
+    un.bh = rest / p.nQC;
+    un.b = (int)(un.bh / p.Hkv);
+    un.h = (int)(un.bh % p.Hkv);
+    un.j = p.j0 + un.jj;
+    un.tok0 = un.j * p.C + un.pair * 32;
+    return un.tok0 < p.q_begin + p.q_len && un.tok0 + 32 > p.q_begin;
+}
 
 // Bounded wait shared by the roles of one CTA: gives up after the time limit,
 // when another role of this CTA gave up (*abort), or when any CTA of the grid
@@ -110,26 +140,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                                                                Params p,
                                                                const int32_t* __restrict__ sel,
                                                                const int32_t* __restrict__ nsel,
-                                                               __nv_bfloat16* __restrict__ out) {
+                                                               __nv_bfloat16* __restrict__ out,
+                                                               int n_units) {
     extern __shared__ uint8_t smem_raw[];
     TcSmem& sm = *reinterpret_cast<TcSmem*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int pair = blockIdx.x, jj = blockIdx.y;
-    const int64_t bh = blockIdx.z;
-    const int b = (int)(bh / p.Hkv), h = (int)(bh % p.Hkv);
-    const int j = p.j0 + jj;
-    const int64_t prob = bh * p.nQC + jj;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int span_end = p.q_begin + p.q_len;
-    const int tok0 = j * p.C + pair * 32;  // first token position of M tile A
-    if (tok0 >= span_end || tok0 + 32 <= p.q_begin) return;
 
     if (warp == 0) {
-        // barriers first, then the Q tiles (they do not depend on the key
-        // set), so the Q load overlaps the reads of the selection list
         if (lane == 0) {
             sm.abort = 0;
             ptx::mbar_init(&sm.bar_q, 1);
+            ptx::mbar_init(&sm.q_empty, 1);
             for (int s = 0; s < 2; ++s) {
                 ptx::mbar_init(&sm.k_full[s], 1);
                 ptx::mbar_init(&sm.k_empty[s], 1);
@@ -138,29 +161,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                 ptx::mbar_init(&sm.s_full[s], 1);
                 ptx::mbar_init(&sm.p_full[s], 4);
                 ptx::mbar_init(&sm.o_done[s], 1);
-                ptx::mbar_init(&sm.st_ready[s], 4);
+                ptx::mbar_init(&sm.list_full[s], 1);
+                ptx::mbar_init(&sm.list_empty[s], 9);  // the producer and the 8 softmax warps
             }
             ptx::mbar_init(&sm.drain, 1);
             ptx::fence_mbar_init();
-            const int tq = tok0 - p.q_begin;
-            ptx::mbar_arrive_expect_tx(&sm.bar_q, 2 * kTile);
-            for (int x = 0; x < 2; ++x) {
-                ptx::tma_load_4d(sm.q[x], &maps.q, 0, h * 8, tq + 16 * x, b, &sm.bar_q);
-                ptx::tma_load_4d(sm.q[x] + kPanel, &maps.q, 64, h * 8, tq + 16 * x, b, &sm.bar_q);
-            }
-        }
-        const int nb_w = build_key_blocks_warp(p, j, sel + prob * p.kg, nsel + prob, false,
-                                               sm.blk_row, sm.blk_pos);
-        if (lane == 0) sm.nb = nb_w;
-        __syncwarp();
-        for (int t = lane; t * kBlocksPerTile < nb_w; t += 32) {
-            int last = 0;
-#pragma unroll
-            for (int i = 0; i < kBlocksPerTile; ++i) {
-                const int blk = t * kBlocksPerTile + i;
-                last = blk < nb_w ? max(last, sm.blk_pos[blk] + kGroupRows - 1) : INT_MAX;
-            }
-            sm.tile_last[t] = last;
         }
     } else if (warp == 1) {
         ptx::tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -170,73 +175,154 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const int nb = sm.nb;
-    const int n_tiles = (nb + kBlocksPerTile - 1) / kBlocksPerTile;
     volatile int* abort = &sm.abort;
+    auto n_tiles_of = [](int nb) { return (nb + kBlocksPerTile - 1) / kBlocksPerTile; };
 
-    if (warp == 0) {
+    if (warp == 10) {
+        // ------------------------------------------------------ block lists
+        // builds the key-block list of this CTA's next units into a double buffer
+        int k = 0;
+        Unit un;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            if (!unit_at(p, u, un)) continue;
+            const int bf = k & 1;
+            if (k >= 2 &&
+                !__all_sync(0xffffffffu, wait_bar(&sm.list_empty[bf], ((k >> 1) - 1) & 1, abort, p.err)))
+                break;
+            const int64_t prob = un.bh * p.nQC + un.jj;
+            const int nb = build_key_blocks_warp(p, un.j, sel + prob * p.kg, nsel + prob, false,
+                                                 sm.blk_row[bf], sm.blk_pos[bf]);
+            __syncwarp();
+            for (int t = lane; t * kBlocksPerTile < nb; t += 32) {
+                int last = 0;
+#pragma unroll
+                for (int i = 0; i < kBlocksPerTile; ++i) {
+                    const int blk = t * kBlocksPerTile + i;
+                    last = blk < nb ? max(last, sm.blk_pos[bf][blk] + kGroupRows - 1) : INT_MAX;
+                }
+                sm.tile_last[bf][t] = last;
+            }
+            __syncwarp();
+            if (lane == 0) {
+                sm.nb[bf] = nb;
+                ptx::mbar_arrive(&sm.list_full[bf]);
+            }
+            ++k;
+        }
+    } else if (warp == 0) {
         // ------------------------------------------------------ producer
-        if (lane == 0 && n_tiles > 0) {
-            for (int t = 0; t < n_tiles; ++t) {
-                const int s = t & 1;
-                if (t >= 2 && !wait_bar(&sm.k_empty[s], ((t >> 1) - 1) & 1, abort, p.err)) break;
-                ptx::mbar_arrive_expect_tx(&sm.k_full[s], kTile);
-                for (int i = 0; i < kBlocksPerTile; ++i) {
-                    const int blk = t * kBlocksPerTile + i;
-                    const int row = blk < nb ? sm.blk_row[blk] : p.L;  // past the end: zero fill
-                    ptx::tma_load_3d(sm.k[s] + i * 2048, &maps.k, 0, row, (int)bh, &sm.k_full[s]);
-                    ptx::tma_load_3d(sm.k[s] + kPanel + i * 2048, &maps.k, 64, row, (int)bh,
-                                     &sm.k_full[s]);
+        if (lane == 0) {
+            int k = 0, g0 = 0;
+            Unit un;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+                if (!unit_at(p, u, un)) continue;
+                const int bf = k & 1;
+                if (!wait_bar(&sm.list_full[bf], (k >> 1) & 1, abort, p.err)) break;
+                const int nb = sm.nb[bf];
+                const int n = n_tiles_of(nb);
+                if (k >= 1 && !wait_bar(&sm.q_empty, (k - 1) & 1, abort, p.err)) break;
+                const int tq = un.tok0 - p.q_begin;
+                ptx::mbar_arrive_expect_tx(&sm.bar_q, 2 * kTile);
+                for (int x = 0; x < 2; ++x) {
+                    ptx::tma_load_4d(sm.q[x], &maps.q, 0, un.h * 8, tq + 16 * x, un.b, &sm.bar_q);
+                    ptx::tma_load_4d(sm.q[x] + kPanel, &maps.q, 64, un.h * 8, tq + 16 * x, un.b,
+                                     &sm.bar_q);
                 }
-                if (t >= 2 && !wait_bar(&sm.v_empty[s], ((t >> 1) - 1) & 1, abort, p.err)) break;
-                ptx::mbar_arrive_expect_tx(&sm.v_full[s], kTile);
-                for (int i = 0; i < kBlocksPerTile; ++i) {
-                    const int blk = t * kBlocksPerTile + i;
-                    const int row = blk < nb ? sm.blk_row[blk] : p.L;
-                    ptx::tma_load_3d(sm.v[s] + i * 2048, &maps.v, 0, row, (int)bh, &sm.v_full[s]);
-                    ptx::tma_load_3d(sm.v[s] + kPanel + i * 2048, &maps.v, 64, row, (int)bh,
-                                     &sm.v_full[s]);
+                for (int t = 0; t < n; ++t) {
+                    const int g = g0 + t, s = g & 1;
+                    if (g >= 2 && !wait_bar(&sm.k_empty[s], ((g >> 1) - 1) & 1, abort, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::mbar_arrive_expect_tx(&sm.k_full[s], kTile);
+                    for (int i = 0; i < kBlocksPerTile; ++i) {
+                        const int blk = t * kBlocksPerTile + i;
+                        const int row = blk < nb ? sm.blk_row[bf][blk] : p.L;  // past the end: zero fill
+                        ptx::tma_load_3d(sm.k[s] + i * 2048, &maps.k, 0, row, (int)un.bh, &sm.k_full[s]);
+                        ptx::tma_load_3d(sm.k[s] + kPanel + i * 2048, &maps.k, 64, row, (int)un.bh,
+                                         &sm.k_full[s]);
+                    }
+                    if (g >= 2 && !wait_bar(&sm.v_empty[s], ((g >> 1) - 1) & 1, abort, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::mbar_arrive_expect_tx(&sm.v_full[s], kTile);
+                    for (int i = 0; i < kBlocksPerTile; ++i) {
+                        const int blk = t * kBlocksPerTile + i;
+                        const int row = blk < nb ? sm.blk_row[bf][blk] : p.L;
+                        ptx::tma_load_3d(sm.v[s] + i * 2048, &maps.v, 0, row, (int)un.bh, &sm.v_full[s]);
+                        ptx::tma_load_3d(sm.v[s] + kPanel + i * 2048, &maps.v, 64, row, (int)un.bh,
+                                         &sm.v_full[s]);
+                    }
                 }
+                if (!ok) break;
+                ptx::mbar_arrive(&sm.list_empty[bf]);
+                g0 += n;
+                ++k;
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
-        if (lane == 0 && n_tiles > 0) {
+        if (lane == 0) {
             const uint32_t q_s[2] = {ptx::smem_u32(sm.q[0]), ptx::smem_u32(sm.q[1])};
-            bool ok = wait_bar(&sm.bar_q, 0, abort, p.err) && wait_bar(&sm.k_full[0], 0, abort, p.err);
-            if (ok) {
+            int k = 0, g0 = 0;
+            Unit un;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+                if (!unit_at(p, u, un)) continue;
+                const int bf = k & 1;
+                ok = wait_bar(&sm.list_full[bf], (k >> 1) & 1, abort, p.err);
+                if (!ok) break;
+                const int n = n_tiles_of(sm.nb[bf]);
+                const int s0 = g0 & 1;
+                ok = wait_bar(&sm.bar_q, k & 1, abort, p.err) &&
+                     wait_bar(&sm.k_full[s0], (g0 >> 1) & 1, abort, p.err);
+                if (!ok) break;
                 ptx::tc_fence_after();
-                const uint32_t k0 = ptx::smem_u32(sm.k[0]);
+                // S_x of the previous unit was read and its P consumed by the PV
+                // issued before on this in-order queue
+                const uint32_t k0 = ptx::smem_u32(sm.k[s0]);
                 issue_qk(tmem + col_s(0), q_s[0], k0);
                 ptx::umma_commit(&sm.s_full[0]);
                 issue_qk(tmem + col_s(1), q_s[1], k0);
                 ptx::umma_commit(&sm.s_full[1]);
-                ptx::umma_commit(&sm.k_empty[0]);
-            }
-            for (int t = 0; ok && t < n_tiles; ++t) {
-                const int s = t & 1, s1 = (t + 1) & 1;
-                const bool more = t + 1 < n_tiles;
-                if (!wait_bar(&sm.v_full[s], (t >> 1) & 1, abort, p.err)) break;
-                if (more && !wait_bar(&sm.k_full[s1], ((t + 1) >> 1) & 1, abort, p.err)) break;
-                const uint32_t v_s = ptx::smem_u32(sm.v[s]);
-                const uint32_t k_s1 = ptx::smem_u32(sm.k[s1]);
-                for (int x = 0; x < 2; ++x) {
-                    if (!wait_bar(&sm.p_full[x], t & 1, abort, p.err)) {
+                if (n == 1) ptx::umma_commit(&sm.q_empty);
+                ptx::umma_commit(&sm.k_empty[s0]);
+                for (int t = 0; ok && t < n; ++t) {
+                    const int g = g0 + t, s = g & 1, s1 = (g + 1) & 1;
+                    const bool more = t + 1 < n;
+                    if (!wait_bar(&sm.v_full[s], (g >> 1) & 1, abort, p.err)) { ok = false; break; }
+                    if (more && !wait_bar(&sm.k_full[s1], ((g + 1) >> 1) & 1, abort, p.err)) {
                         ok = false;
                         break;
                     }
-                    ptx::tc_fence_after();
-                    issue_pv(tmem + col_o(x), tmem + col_s(x), v_s, t > 0);
-                    if (more) {
-                        issue_qk(tmem + col_s(x), q_s[x], k_s1);
-                        ptx::umma_commit(&sm.s_full[x]);
-                    } else {
-                        ptx::umma_commit(&sm.o_done[x]);
+                    const uint32_t v_s = ptx::smem_u32(sm.v[s]);
+                    const uint32_t k_s1 = ptx::smem_u32(sm.k[s1]);
+                    for (int x = 0; x < 2; ++x) {
+                        // P_x of this tile; for t == 0 this also orders the
+                        // PV that overwrites O_x after the same warps' epilogue
+                        // of the previous unit read it
+                        if (!wait_bar(&sm.p_full[x], g & 1, abort, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        issue_pv(tmem + col_o(x), tmem + col_s(x), v_s, t > 0);
+                        if (more) {
+                            issue_qk(tmem + col_s(x), q_s[x], k_s1);
+                            ptx::umma_commit(&sm.s_full[x]);
+                        } else {
+                            ptx::umma_commit(&sm.o_done[x]);
+                        }
                     }
+                    if (!ok) break;
+                    if (more && t + 2 == n) ptx::umma_commit(&sm.q_empty);  // last QK issued
+                    ptx::umma_commit(&sm.v_empty[s]);
+                    if (more) ptx::umma_commit(&sm.k_empty[s1]);
                 }
-                if (!ok) break;
-                ptx::umma_commit(&sm.v_empty[s]);
-                if (more) ptx::umma_commit(&sm.k_empty[s1]);
+                g0 += n;
+                ++k;
             }
             // drain: every MMA issued above has completed before TMEM is freed
             ptx::umma_commit(&sm.drain);
@@ -244,9 +330,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             while (!ptx::mbar_try_wait(&sm.drain, 0) &&
                    ptx::globaltimer_ns() - t0 < ptx::kWaitLimitNs) {
             }
-        } else if (lane == 0) {
-            // no key tile: still let the Q load land before the CTA exits
-            wait_bar(&sm.bar_q, 0, abort, p.err);
         }
     } else {
         // ------------------------------------------------------ softmax
@@ -254,156 +337,165 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         const int q4 = warp & 3;                        // TMEM lane quarter
         const int r = q4 * 32 + lane;                   // row = TMEM lane
         const int head = r & 7;
-        const int tokx = tok0 + 16 * x;
-        const int qpos = tokx + (r >> 3);
-        const bool row_ok = qpos >= p.q_begin && qpos < span_end;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + col_s(x);
         const uint32_t o_addr = tmem + lane_off + col_o(x);
         const float sc = 1.4426950408889634f / sqrtf((float)kD);
-        float m_used = -INFINITY, l = 0.f;
-        bool ok = n_tiles > 0;
-        for (int t = 0; ok && t < n_tiles; ++t) {
-            if (!__all_sync(0xffffffffu, wait_bar(&sm.s_full[x], t & 1, abort, p.err))) {
+        int k = 0, g0 = 0;
+        Unit un;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+            if (!unit_at(p, u, un)) continue;
+            const int bf = k & 1;
+            if (!__all_sync(0xffffffffu, wait_bar(&sm.list_full[bf], (k >> 1) & 1, abort, p.err))) {
+                ok = false;
+                break;
+            }
+            const int nb = sm.nb[bf];
+            const int n = n_tiles_of(nb);
+            const int tokx = un.tok0 + 16 * x;
+            const int qpos = tokx + (r >> 3);
+            const bool row_ok = qpos >= p.q_begin && qpos < span_end;
+            float m_used = -INFINITY, l = 0.f;
+            for (int t = 0; t < n; ++t) {
+                const int g = g0 + t;
+                if (!__all_sync(0xffffffffu, wait_bar(&sm.s_full[x], g & 1, abort, p.err))) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                float sx[kTileKeys];
+                {
+                    uint32_t* xr = reinterpret_cast<uint32_t*>(sx);
+                    ptx::tmem_ld64(s_addr, xr);
+                    ptx::tmem_ld64(s_addr + 64, xr + 64);
+                    ptx::tmem_wait_ld();
+                    ptx::reg_fence<kTileKeys>(xr);
+                }
+                // mask (causal within the current chunk; padding past the set)
+                const int blk0 = t * kBlocksPerTile;
+                const bool need_mask = sm.tile_last[bf][t] > tokx;
+                float mraw = -INFINITY;
+                if (need_mask) {
+#pragma unroll
+                    for (int i = 0; i < kBlocksPerTile; ++i) {
+                        const int kp = blk0 + i < nb ? sm.blk_pos[bf][blk0 + i] : 0x7fffffff - 64;
+#pragma unroll
+                        for (int e = 0; e < kGroupRows; ++e) {
+                            const int c = i * kGroupRows + e;
+                            sx[c] = (kp + e <= qpos) ? sx[c] : -INFINITY;
+                            mraw = fmaxf(mraw, sx[c]);
+                        }
+                    }
+                } else {
+                    // four independent three-input chains
+                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int c = 0; c < kTileKeys; c += 8) {
+#pragma unroll
+                        for (int uu = 0; uu < 4; ++uu)
+                            m4[uu] = ptx::fmax3(m4[uu], sx[c + 2 * uu], sx[c + 2 * uu + 1]);
+                    }
+                    mraw = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                }
+                const float m_new = fmaxf(m_used, mraw * sc);
+                bool rescale = false;
+                float alpha = 1.f;
+                if (m_new != -INFINITY) {
+                    if (m_used == -INFINITY) {
+                        m_used = m_new;
+                    } else if (m_new > m_used + kRescaleLog2) {
+                        alpha = ptx::ex2_approx(m_used - m_new);
+                        m_used = m_new;
+                        rescale = true;
+                    }
+                }
+                // P = 2^(S*sc - m), rounded to bf16; the row sum uses the rounded values
+                uint32_t pk[kTileKeys / 2];
+                float lsum0 = 0.f, lsum1 = 0.f;
+                const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+#pragma unroll
+                for (int c = 0; c < kTileKeys; c += 2) {
+                    float a0, a1;
+                    ptx::fma2_bc(sx[c], sx[c + 1], sc, neg_m, a0, a1);
+                    const float p0 = ptx::ex2_approx(a0);
+                    const float p1 = ptx::ex2_approx(a1);
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+                    pk[c / 2] = *reinterpret_cast<uint32_t*>(&b2);
+                    ptx::add_bf16x2_f32(pk[c / 2], lsum0, lsum1);
+                }
+                const float lsum = lsum0 + lsum1;
+                // tcgen05.ld/st are warp-collective: the whole warp rescales its
+                // rows when any row needs it (rows that do not use alpha = 1).
+                // PV of the previous tile has completed: S of this tile was issued
+                // after it on the same (in-order) tensor-core queue.
+                if (__any_sync(0xffffffffu, rescale && t >= 1)) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t o[32];
+                        ptx::tmem_ld32(o_addr + 32 * c, o);
+                        ptx::tmem_wait_ld();
+                        ptx::reg_fence<32>(o);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        ptx::tmem_st32(o_addr + 32 * c, o);
+                    }
+                }
+                l = l * alpha + lsum;
+                ptx::tmem_st32(s_addr, pk);
+                ptx::tmem_st32(s_addr + 32, pk + 32);
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&sm.p_full[x]);
+            }
+            if (!ok) break;
+            if (lane == 0) ptx::mbar_arrive(&sm.list_empty[bf]);
+            if (!__all_sync(0xffffffffu, wait_bar(&sm.o_done[x], k & 1, abort, p.err))) {
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
-            float sx[kTileKeys];
-            {
-                uint32_t* xr = reinterpret_cast<uint32_t*>(sx);
-                ptx::tmem_ld64(s_addr, xr);
-                ptx::tmem_ld64(s_addr + 64, xr + 64);
-                ptx::tmem_wait_ld();
-                ptx::reg_fence<kTileKeys>(xr);
-            }
-            // mask (causal within the current chunk; padding past the set)
-            const int blk0 = t * kBlocksPerTile;
-            const bool need_mask = sm.tile_last[t] > tokx;
-            float mraw = -INFINITY;
-            if (need_mask) {
-#pragma unroll
-                for (int i = 0; i < kBlocksPerTile; ++i) {
-                    const int kp = blk0 + i < nb ? sm.blk_pos[blk0 + i] : 0x7fffffff - 64;
-#pragma unroll
-                    for (int e = 0; e < kGroupRows; ++e) {
-                        const int c = i * kGroupRows + e;
-                        sx[c] = (kp + e <= qpos) ? sx[c] : -INFINITY;
-                        mraw = fmaxf(mraw, sx[c]);
-                    }
-                }
-            } else {
-                // four independent three-input chains
-                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int c = 0; c < kTileKeys; c += 8) {
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) m4[u] = ptx::fmax3(m4[u], sx[c + 2 * u], sx[c + 2 * u + 1]);
-                }
-                mraw = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            }
-            const float m_new = fmaxf(m_used, mraw * sc);
-            bool rescale = false;
-            float alpha = 1.f;
-            if (m_new != -INFINITY) {
-                if (m_used == -INFINITY) {
-                    m_used = m_new;
-                } else if (m_new > m_used + kRescaleLog2) {
-                    alpha = ptx::ex2_approx(m_used - m_new);
-                    m_used = m_new;
-                    rescale = true;
-                }
-            }
-            // P = 2^(S*sc - m), rounded to bf16; the row sum uses the rounded values
-            uint32_t pk[kTileKeys / 2];
-            float lsum0 = 0.f, lsum1 = 0.f;
-            const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-#pragma unroll
-            for (int c = 0; c < kTileKeys; c += 2) {
-                float a0, a1;
-                ptx::fma2_bc(sx[c], sx[c + 1], sc, neg_m, a0, a1);
-                const float p0 = ptx::ex2_approx(a0);
-                const float p1 = ptx::ex2_approx(a1);
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-                pk[c / 2] = *reinterpret_cast<uint32_t*>(&b2);
-                ptx::add_bf16x2_f32(pk[c / 2], lsum0, lsum1);
-            }
-            const float lsum = lsum0 + lsum1;
-            // tcgen05.ld/st are warp-collective: the whole warp rescales its
-            // rows when any row needs it (rows that do not use alpha = 1).
-            // PV of the previous tile has completed: S of this tile was issued
-            // after it on the same (in-order) tensor-core queue.
-            if (__any_sync(0xffffffffu, rescale && t >= 1)) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t o[32];
-                    ptx::tmem_ld32(o_addr + 32 * c, o);
-                    ptx::tmem_wait_ld();
-                    ptx::reg_fence<32>(o);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    ptx::tmem_st32(o_addr + 32 * c, o);
-                }
-            }
-            l = l * alpha + lsum;
-            ptx::tmem_st32(s_addr, pk);
-            ptx::tmem_st32(s_addr + 32, pk + 32);
-            ptx::tmem_wait_st();
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&sm.p_full[x]);
-        }
-        if (ok && __all_sync(0xffffffffu, wait_bar(&sm.o_done[x], 0, abort, p.err))) {
-            ptx::tc_fence_after();
             const float inv = l > 0.f ? 1.0f / l : 0.f;
-            __nv_bfloat16* orow =
-                out + (((int64_t)b * p.q_len + (qpos - p.q_begin)) * p.Hq + (int64_t)h * 8 + head) * kD;
             // all of O in one round trip
             uint32_t o[kD];
 #pragma unroll
             for (int c = 0; c < 4; ++c) ptx::tmem_ld32(o_addr + 32 * c, o + 32 * c);
             ptx::tmem_wait_ld();
             ptx::reg_fence<kD>(o);
-            if (tokx >= p.q_begin && tokx + 16 <= span_end) {
-                // Whole M tile in the span: the rows go to the Q buffer of this
-                // tile (its last QK completed before o_done) in the Q map's
-                // swizzled layout, then two TMA stores write them out.
-                uint8_t* stage = sm.q[x];
+            ptx::tc_fence_before();
+            // Coalesced output: four rounds of 32 dims; each row's 64 bytes go
+            // through this warp's staging area (16-byte chunks XOR-swizzled by
+            // (row / 2) % 4) and come back as 8 rows x 4 chunks per store.
+            uint8_t* stg = sm.stage[warp - 2];
+            const int rr = lane >> 2, cc = lane & 3;   // read-back: row within 8, chunk
 #pragma unroll
-                for (int pnl = 0; pnl < 2; ++pnl) {
+            for (int qd = 0; qd < 4; ++qd) {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        float f[8];
-#pragma unroll
-                        for (int z = 0; z < 8; ++z) f[z] = __uint_as_float(o[64 * pnl + 8 * c + z]) * inv;
-                        *reinterpret_cast<uint4*>(stage + pnl * kPanel + r * 128 + ((c ^ (r & 7)) << 4)) =
-                            f32x8_to_bf16(f);
-                    }
-                }
-                ptx::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&sm.st_ready[x]);
-                if (q4 == 2 && lane == 0 &&  // one warp of the four issues the stores
-                    wait_bar(&sm.st_ready[x], 0, abort, p.err)) {
-                    const int tq = tokx - p.q_begin;
-                    ptx::tma_store_4d(&maps.o, stage, 0, h * 8, tq, b);
-                    ptx::tma_store_4d(&maps.o, stage + kPanel, 64, h * 8, tq, b);
-                    ptx::bulk_commit();
-                    ptx::bulk_wait_read_all();
-                }
-            } else if (row_ok) {
-#pragma unroll
-                for (int e = 0; e < kD; e += 8) {
+                for (int c = 0; c < 4; ++c) {
                     float f[8];
 #pragma unroll
-                    for (int z = 0; z < 8; ++z) f[z] = __uint_as_float(o[e + z]) * inv;
-                    *reinterpret_cast<uint4*>(orow + e) = f32x8_to_bf16(f);
+                    for (int z = 0; z < 8; ++z) f[z] = __uint_as_float(o[32 * qd + 8 * c + z]) * inv;
+                    *reinterpret_cast<uint4*>(stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+                        f32x8_to_bf16(f);
                 }
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int R = 8 * i + rr;                       // row within the warp
+                    const int rq = q4 * 32 + R;                     // row of the M tile
+                    const int qp = tokx + (rq >> 3);
+                    const uint4 v = *reinterpret_cast<const uint4*>(stg + R * 64 + ((cc ^ ((R >> 1) & 3)) << 4));
+                    if (qp >= p.q_begin && qp < span_end) {
+                        __nv_bfloat16* dst = out + (((int64_t)un.b * p.q_len + (qp - p.q_begin)) * p.Hq +
+                                                    (int64_t)un.h * 8 + (rq & 7)) * kD + 32 * qd + 8 * cc;
+                        *reinterpret_cast<uint4*>(dst) = v;
+                    }
+                }
+                __syncwarp();
             }
-        } else if (row_ok) {
-            __nv_bfloat16* orow =
-                out + (((int64_t)b * p.q_len + (qpos - p.q_begin)) * p.Hq + (int64_t)h * 8 + head) * kD;
-            for (int e = 0; e < kD; ++e) orow[e] = __float2bfloat16_rn(0.f);
+            g0 += n;
+            ++k;
         }
         ptx::tc_fence_before();
     }
@@ -430,8 +522,7 @@ cudaError_t launch_attend_tc(const Params& p, const void* q_rot, const KvSources
     const int64_t BH = (int64_t)p.B * p.Hkv;
     bool ok = make_query_map(&maps.q, q_rot, p.B, p.q_len, p.Hq, kD, 8, 16) &&
               make_rows_map(&maps.k, kv.k_res, BH, p.L, kD, kGroupRows) &&
-              make_rows_map(&maps.v, kv.v_res, BH, p.L, kD, kGroupRows) &&
-              make_query_map(&maps.o, out, p.B, p.q_len, p.Hq, kD, 8, 16);
+              make_rows_map(&maps.v, kv.v_res, BH, p.L, kD, kGroupRows);
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = sizeof(TcSmem) + 1024;
     static bool attr_set = false;
@@ -441,9 +532,14 @@ cudaError_t launch_attend_tc(const Params& p, const void* q_rot, const KvSources
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    dim3 grid(p.C / 32, p.nQC, (unsigned)BH);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return cudaErrorInvalidValue;
+    const int64_t n_units = (int64_t)(p.C / 32) * p.nQC * BH;
+    const int grid = (int)(n_units < sms ? n_units : sms);
     attend_tc_kernel<<<grid, kThreads, smem, st>>>(maps, p, sel_groups, n_sel_groups,
-                                                   (__nv_bfloat16*)out);
+                                                   (__nv_bfloat16*)out, (int)n_units);
     return cudaGetLastError();
 }
 
