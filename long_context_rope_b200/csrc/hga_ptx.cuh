@@ -120,23 +120,6 @@ __device__ __forceinline__ void tma_load_4d(void* dst_smem, const CUtensorMap* m
         : "memory");
 }
 
-// 4-D tiled store from this CTA's shared memory (laid out as the map's box,
-// swizzle included), tracked by the bulk async-group of the issuing thread.
-// No coordinate may be negative.
-__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src_smem, int c0,
-                                             int c1, int c2, int c3) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
-        ::"l"(map), "r"(smem_u32(src_smem)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-        : "memory");
-}
-
-// Wait until every bulk copy this thread committed has finished reading its
-// shared-memory source.
-__device__ __forceinline__ void bulk_wait_read_all() {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
