@@ -51,6 +51,10 @@ class Workload:
     plant_every: int  # prefill: plant into query chunks j>0 with j % plant_every == 0
     plant_count: int  # prefill: earlier chunks planted per query chunk (clamped to j)
     tiered: bool = False  # decode only: token K/V lives in pinned host memory
+    # prefill only: an explicit query span [span_begin, span_begin + span_len)
+    # (a chunked prefill); -1 = the whole context
+    span_begin: int = -1
+    span_len: int = -1
 
     @property
     def n_chunks(self) -> int:
@@ -62,11 +66,15 @@ class Workload:
 
     @property
     def q_begin(self) -> int:
-        return 0 if self.mode == "prefill" else self.seq_len - 1
+        if self.mode != "prefill":
+            return self.seq_len - 1
+        return 0 if self.span_begin < 0 else self.span_begin
 
     @property
     def q_len(self) -> int:
-        return self.seq_len if self.mode == "prefill" else 1
+        if self.mode != "prefill":
+            return 1
+        return self.seq_len if self.span_begin < 0 else self.span_len
 
     def torch_dtype(self) -> torch.dtype:
         return torch.bfloat16 if self.dtype == "bf16" else torch.float32
@@ -150,7 +158,10 @@ def draw(w: Workload, seed: int = 0, with_kv: bool = True) -> Dict[str, object]:
                     src = torch.randperm(j, generator=g)[:n_src].tolist()
                     add = topics[b, :, src].sum(dim=1)  # [Hkv, d]
                     add = add.repeat_interleave(gq, dim=0)  # [Hq, d]
-                    q_raw[b, j * C: min((j + 1) * C, L)] += add
+                    lo = max(j * C, w.q_begin)
+                    hi = min((j + 1) * C, L, w.q_begin + w.q_len)
+                    if hi > lo:
+                        q_raw[b, lo - w.q_begin: hi - w.q_begin] += add
                 per_b.append(src)
             planted.append(per_b)
     else:

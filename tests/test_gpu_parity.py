@@ -197,6 +197,19 @@ def test_prefill_parity_ragged_small(L, F, dtype):
     compare_prefill(w, x)
 
 
+def test_prefill_parity_chunked_span():
+    """A prefill span that starts and ends inside chunks (a chunked prefill,
+    tokens [170, 860) of 1000): the attention kernel skips the 32-token query
+    pairs that lie wholly before or after the span and masks the rows of the
+    partial M tiles at both ends; routing starts at query chunk 2."""
+    w = synth.WORKLOADS["prefill_4k"].replace(
+        name="span", seq_len=1000, n_q_heads=8, n_kv_heads=2, top_k_chunks=5, top_k_groups=13,
+        n_local=1, n_sink=2, span_begin=170, span_len=690)
+    assert (w.q_begin, w.q_len) == (170, 690)
+    x = synth.draw(w, seed=4)
+    compare_prefill(w, x)
+
+
 def test_prefill_64k_sampled():
     """The 64K-context workload at full size: every rotation, summary, score
     and selection, and the outputs of 64 sampled (KV head, query chunk) units."""
