@@ -6,7 +6,9 @@
 // file-scope __device__ int whose address is looked up once per device).
 #include <math.h>
 #include <stddef.h>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "hga.h"
 #include "hga_kernels.h"
@@ -130,6 +132,30 @@ hga_status launched(cudaError_t e) { return e == cudaSuccess ? HGA_OK : HGA_ERR_
     } while (0)
 
 }  // namespace
+}  // namespace hga
+
+namespace hga {
+
+cudaError_t current_device_index(int* dev) {
+    if (cudaGetDevice(dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    return (*dev >= 0 && *dev < kMaxDevicesPerProcess) ? cudaSuccess : cudaErrorInvalidDevice;
+}
+
+cudaError_t set_func_attr_once(const void* fn, cudaFuncAttribute attr, int value) {
+    static std::mutex mu;
+    static std::map<std::tuple<int, const void*, int>, int> done;
+    int dev = 0;
+    cudaError_t e = current_device_index(&dev);
+    if (e != cudaSuccess) return e;
+    const auto key = std::make_tuple(dev, fn, (int)attr);
+    std::lock_guard<std::mutex> lock(mu);
+    const auto it = done.find(key);
+    if (it != done.end() && it->second == value) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, attr, value);
+    if (e == cudaSuccess) done[key] = value;
+    return e;
+}
+
 }  // namespace hga
 
 using namespace hga;

@@ -13,6 +13,16 @@ namespace hga {
 constexpr int kMaxBlocks = 512;
 // Largest number of chunks the routing kernels keep in shared memory.
 constexpr int kMaxChunks = 16384;
+// Devices a process may drive (per-device caches of the launchers).
+constexpr int kMaxDevicesPerProcess = 64;
+
+// Set attribute `attr` of kernel `fn` to `value` on the current device, once
+// per (device, kernel, attribute, value): kernel attributes belong to the
+// kernel as loaded on each device, and a driver call on every launch would
+// add host latency to every decode step.
+cudaError_t set_func_attr_once(const void* fn, cudaFuncAttribute attr, int value);
+// Current device as an index into per-device caches (< kMaxDevicesPerProcess).
+cudaError_t current_device_index(int* dev);
 
 cudaError_t launch_rope(const Params& p, const void* x, void* y, int64_t n_outer,
                         int64_t n_tokens, int n_heads, int64_t pos0, cudaStream_t st);

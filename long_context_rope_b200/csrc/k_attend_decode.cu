@@ -187,14 +187,19 @@ cudaError_t launch_attend_decode(const Params& p, const void* q_rot, const KvSou
     }
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = sizeof(DecodeSmem) + 1024;
-    static int max_cluster = -1;
-    if (max_cluster < 0) {
-        cudaError_t e = cudaFuncSetAttribute(attend_decode_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(attend_decode_kernel,
-                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
+    // largest cluster that co-schedules, per device (queried once)
+    static int max_cluster_of[kMaxDevicesPerProcess];  // 0 = not yet queried
+    int dev = 0;
+    cudaError_t e = current_device_index(&dev);
+    if (e != cudaSuccess) return e;
+    e = set_func_attr_once((const void*)attend_decode_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+        e = set_func_attr_once((const void*)attend_decode_kernel,
+                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    int& max_cluster = max_cluster_of[dev];
+    if (max_cluster <= 0) {
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(kMaxCluster, 1, 1);
         q.blockDim = dim3(kThreads);

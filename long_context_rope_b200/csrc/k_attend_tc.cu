@@ -525,13 +525,9 @@ cudaError_t launch_attend_tc(const Params& p, const void* q_rot, const KvSources
               make_rows_map(&maps.v, kv.v_res, BH, p.L, kD, kGroupRows);
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = sizeof(TcSmem) + 1024;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t e = set_func_attr_once((const void*)attend_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)

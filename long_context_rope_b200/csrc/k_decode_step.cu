@@ -423,24 +423,25 @@ bool step_fits(const Params& p, int cl) {
 }
 
 std::mutex g_step_mu;
-int g_max_active[kMaxCluster + 1] = {};
-bool g_attr_done = false;
+int g_max_active[kMaxDevicesPerProcess][kMaxCluster + 1] = {};  // per device, 0 = not queried
 
 cudaError_t step_prepare(size_t smem) {
-    std::lock_guard<std::mutex> lock(g_step_mu);
-    if (g_attr_done) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(decode_step_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_func_attr_once((const void*)decode_step_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(decode_step_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,
-                                 1);
-    if (e == cudaSuccess) g_attr_done = true;
+        e = set_func_attr_once((const void*)decode_step_kernel,
+                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return e;
 }
 
+// Clusters of `cl` CTAs that can be resident at once on the current device
+// (-1 if the query fails).
 int active_clusters(int cl, size_t smem) {
+    int dev = 0;
+    if (current_device_index(&dev) != cudaSuccess) return -1;
     std::lock_guard<std::mutex> lock(g_step_mu);
-    if (g_max_active[cl] == 0) {
+    int& slot = g_max_active[dev][cl];
+    if (slot == 0) {
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(cl, 1, 1);
         q.blockDim = dim3(kThreads);
@@ -457,9 +458,9 @@ int active_clusters(int cl, size_t smem) {
             cudaGetLastError();
             n = -1;
         }
-        g_max_active[cl] = n;
+        slot = n;
     }
-    return g_max_active[cl];
+    return slot;
 }
 
 // Cluster size: two CTAs per SM over the whole grid if the tables fit and the

@@ -306,13 +306,11 @@ cudaError_t launch_gather_warm(const Params& p, const void* k_host, const void* 
                                int n_slots, int step, int32_t* src_out, int32_t* stats_out,
                                void* k_dst, void* v_dst, cudaStream_t st) {
     const size_t smem = (size_t)(n_slots + 256) * sizeof(uint32_t) + (size_t)4 * p.kg * sizeof(int);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(warm_plan_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)((kMaxWarmSlots + 256) * 4 + 4 * kMaxBlocks * 4));
+    {
+        cudaError_t e = set_func_attr_once((const void*)warm_plan_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)((kMaxWarmSlots + 256) * 4 + 4 * kMaxBlocks * 4));
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     warm_plan_kernel<<<p.B * p.Hkv, 256, smem, st>>>(p, sel_groups, n_sel_groups, pool_tag,
                                                      pool_last, n_slots, step, src_out, stats_out);
@@ -337,13 +335,9 @@ cudaError_t launch_gather(const Params& p, const void* k_src, const void* v_src,
                                                  (uint4*)v_dst);
     } else {
         const size_t smem = (size_t)kSlotsPerCta * 2 * kGroupRows * p.d * es;
-        static bool attr_set = false;
-        if (!attr_set) {
-            cudaError_t e = cudaFuncSetAttribute(
-                gather_hbm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
-            if (e != cudaSuccess) return e;
-            attr_set = true;
-        }
+        cudaError_t e = set_func_attr_once((const void*)gather_hbm_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+        if (e != cudaSuccess) return e;
         dim3 grid((p.kg + kSlotsPerCta - 1) / kSlotsPerCta, p.nQC, p.B * p.Hkv);
         gather_hbm_kernel<<<grid, 32, smem, st>>>(p, (const char*)k_src, (const char*)v_src,
                                                   sel_groups, n_sel_groups, (char*)k_dst,

@@ -15,8 +15,6 @@
 // top-k by repeated warp arg-max and compacts the winners in ascending order.
 #include <cooperative_groups.h>
 
-#include <mutex>
-#include <set>
 
 #include "hga_kernels.h"
 #include "hga_topk.cuh"
@@ -380,16 +378,9 @@ __global__ void __launch_bounds__(128) route_groups_small_kernel(
     if (lane == 0) n_sel_groups[prob] = kept;
 }
 
-// Raise a kernel's dynamic shared-memory limit once per process (a driver
-// call per launch would add host latency to every decode step).
+// Raise a kernel's dynamic shared-memory limit (once per device and kernel).
 cudaError_t allow_smem(const void* fn, size_t bytes) {
-    static std::mutex mu;
-    static std::set<const void*> done;
-    std::lock_guard<std::mutex> lock(mu);
-    if (done.count(fn)) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e == cudaSuccess) done.insert(fn);
-    return e;
+    return set_func_attr_once(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
 cudaError_t launch_cluster(const void* fn, dim3 grid, int block, size_t smem, int cl,
@@ -420,11 +411,19 @@ cudaError_t launch_qbar(const Params& p, const void* q_rot, float* qbar, cudaStr
     dim3 grid(p.nQC, p.B);
     if (p.dtype == HGA_BF16) {
         auto fn = qbar_kernel<__nv_bfloat16>;
-        if (smem > 48 * 1024) cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (smem > 48 * 1024) {
+            cudaError_t e = set_func_attr_once((const void*)fn,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
         fn<<<grid, kQbarThreads, smem, st>>>(p, (const __nv_bfloat16*)q_rot, qbar);
     } else {
         auto fn = qbar_kernel<float>;
-        if (smem > 48 * 1024) cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (smem > 48 * 1024) {
+            cudaError_t e = set_func_attr_once((const void*)fn,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
         fn<<<grid, kQbarThreads, smem, st>>>(p, (const float*)q_rot, qbar);
     }
     return cudaGetLastError();

@@ -156,17 +156,14 @@ cudaError_t launch_route_chunks_tiled(const Params& p, const float* qbar, const 
     dim3 grid((p.nQC + kQB - 1) / kQB, p.B * p.Hkv);
     const void* fn = p.d == 128 ? (const void*)route_chunks_tiled_kernel<128>
                                 : (const void*)route_chunks_tiled_kernel<64>;
-    static bool attr = false;
-    if (!attr) {
-        const size_t max_smem = (size_t)(128 * kQB + kKS * kCT + kQB * 2048) * sizeof(float);
-        cudaError_t e = cudaFuncSetAttribute(route_chunks_tiled_kernel<128>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)max_smem);
+    {
+        const int max_smem = (int)((size_t)(128 * kQB + kKS * kCT + kQB * 2048) * sizeof(float));
+        cudaError_t e = set_func_attr_once((const void*)route_chunks_tiled_kernel<128>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(route_chunks_tiled_kernel<64>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_smem);
+            e = set_func_attr_once((const void*)route_chunks_tiled_kernel<64>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
         if (e != cudaSuccess) return e;
-        attr = true;
     }
     Params pp = p;
     void* args[] = {&pp, (void*)&qbar, (void*)&chunk_sum, &sel, &n_sel, &scores};
