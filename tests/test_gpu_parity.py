@@ -197,6 +197,16 @@ def test_prefill_parity_ragged_small(L, F, dtype):
     compare_prefill(w, x)
 
 
+def test_prefill_parity_batch2():
+    """Two sequences in one call (ragged length, reduced heads): the second
+    sequence's units, query rows and key rows in every prefill kernel."""
+    w = synth.WORKLOADS["prefill_4k"].replace(
+        name="batch2", batch=2, seq_len=968, n_q_heads=16, n_kv_heads=2, top_k_chunks=4,
+        top_k_groups=11, n_local=1, n_sink=1)
+    x = synth.draw(w, seed=5)
+    compare_prefill(w, x)
+
+
 def test_prefill_parity_chunked_span():
     """A prefill span that starts and ends inside chunks (a chunked prefill,
     tokens [170, 860) of 1000): the attention kernel skips the 32-token query
