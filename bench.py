@@ -411,12 +411,20 @@ def host_link_peak_gbs(dev) -> float:
     return best
 
 
-def cpu_baseline(args, n_chunks_sample=4):
+def cpu_baseline(args, n_chunks_sample=4, threads=None):
     """The oracle, as it stands, on a bounded sample of the 64K workload:
     whole-sequence work (key rotation, summaries) timed once and charged per
     token; per-query-chunk work (query rotation, q-bar, routing, attention)
-    timed on `n_chunks_sample` query chunks."""
+    timed on `n_chunks_sample` query chunks. `threads`: the oracle's thread
+    count for this measurement (None: all host cores); restored afterwards."""
     from oracle import hga_oracle as O
+    if threads is not None:
+        all_threads = O.num_threads()
+        O.set_threads(threads)
+        try:
+            return cpu_baseline(args, n_chunks_sample)
+        finally:
+            O.set_threads(all_threads)
     w = synth.WORKLOADS[args.workload]
     x = synth.draw(w, seed=args.seed)
     cfg = O.cfg_of(w)
@@ -546,6 +554,8 @@ def main():
         if n == 1 and dist.rank == 0 and not args.no_cpu_baseline:
             cb = cpu_baseline(args)
             cb.pop("seconds")
+            one = cpu_baseline(args, threads=1)
+            cb["value_1_thread"] = one["value"]
             line["cpu_baseline"] = cb
         if dist.rank == 0:
             print(json.dumps(line), flush=True)
