@@ -46,6 +46,12 @@
  *     asked, and computes everything else in double.
  *   - causal rule: a query at position p sees keys at positions <= p.
  *
+ * Parity unpinned: the pairing, the representative position and the routing
+ * query's aggregation are choices the pages cannot decide, so no test pins
+ * them to the pages; they are fixed as above and taken identically on the
+ * GPU side. The rest is pinned by closed forms, invariants and brute force
+ * (tests/test_oracle_pins.py).
+ *
  * Arithmetic is double throughout; loops follow the definitions with no
  * blocking or reordering. Independent units may run in parallel (OpenMP);
  * that changes no arithmetic.

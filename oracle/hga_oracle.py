@@ -9,7 +9,9 @@ workload description it is given by attribute only).
 
 Method source: "Technische Samenvatting: Hierarchical Global Attention (HGA)"
 (gist.science), section "Kernmechanisme" items 1-4; see hga_oracle.c for the
-readings taken where the page is silent.
+readings taken where the page is silent. Parity unpinned (the pages cannot
+decide them): the RoPE pairing, the representative position and the routing
+query's aggregation; everything else is pinned in tests/test_oracle_pins.py.
 """
 from __future__ import annotations
 
