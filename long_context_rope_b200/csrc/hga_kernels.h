@@ -41,7 +41,7 @@ cudaError_t launch_route_chunks(const Params& p, const void* q_rot, float* qbar,
                                 const float* chunk_sum, int32_t* sel, int32_t* n_sel,
                                 float* scores, cudaStream_t st);
 
-// Prefill form of level-1 routing: 16 query chunks per CTA share one pass
+// Prefill form of level-1 routing: 8 query chunks per CTA share one pass
 // over the chunk-summary table (needs nQC >= 8 and nC <= 2048).
 bool route_chunks_tiled_supports(const Params& p);
 cudaError_t launch_route_chunks_tiled(const Params& p, const float* qbar, const float* chunk_sum,
