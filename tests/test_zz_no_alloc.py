@@ -42,6 +42,26 @@ def test_noalloc_rejects_more_than_its_scratch_holds(hga):
     assert hga.library().hga_status_string(st).decode().startswith("HGA_ERR_SCRATCH_LIMIT")
 
 
+def test_noalloc_validates_like_the_warm_gather(hga):
+    # decode only, pool at least top_k_groups slots, 16-byte pointers; all
+    # checked on the host before any CUDA call (fake pointers, never read)
+    L = hga.library()
+    P = ctypes.c_void_p(16 * 1024)
+    by = ctypes.byref
+    dec = hga.config_from(synth.WORKLOADS["prefill_4k"], q_begin=4095, q_len=1)
+    pre = hga.config_from(synth.WORKLOADS["prefill_4k"])
+    assert L.hga_gather_kv_warm_noalloc(by(dec), P, P, P, P, P, P, P, None, 128, 0, None, P, P,
+                                        None) == -1
+    assert L.hga_gather_kv_warm_noalloc(by(pre), P, P, P, P, P, P, P, P, 128, 0, None, P, P,
+                                        None) == -8
+    assert L.hga_gather_kv_warm_noalloc(by(dec), P, P, P, P, P, P, P, P, 64, 0, None, P, P,
+                                        None) == -2
+    assert L.hga_gather_kv_warm_noalloc(by(dec), P, P, P, P, P, P, P, P, 128, -1, None, P, P,
+                                        None) == -2
+    assert L.hga_gather_kv_warm_noalloc(by(dec), P, P, P, P, P, P, P, P, 128, 0,
+                                        ctypes.c_void_p(16 * 1024 + 4), P, P, None) == -3
+
+
 @pytest.mark.gpu
 def test_noalloc_matches_warm_gather_on_two_calls_in_a_row(hga):
     from long_context_rope_b200 import pipeline
