@@ -2,8 +2,10 @@
 //
 // Every entry point validates its arguments on the host, builds the
 // kernel-side Params, and enqueues kernels on the caller's stream. Nothing
-// is allocated; the only state is one device error word per device (a
-// file-scope __device__ int whose address is looked up once per device).
+// is allocated. State: per device, the error word (a file-scope __device__
+// int) and the fixed scratch array of hga_gather_kv_warm_noalloc, whose
+// addresses are looked up once per device; on the host, which kernel
+// attributes have been set on which device.
 #include <math.h>
 #include <stddef.h>
 #include <map>
