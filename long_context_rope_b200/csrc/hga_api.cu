@@ -167,7 +167,7 @@ static_assert(offsetof(hga_config, rope_theta) == 48, "hga_config layout is part
 
 extern "C" {
 
-int32_t hga_version(void) { return 10200; }
+int32_t hga_version(void) { return 10300; }
 
 const char* hga_status_string(hga_status s) {
     switch (s) {
