@@ -26,7 +26,9 @@
  *     Inputs are never modified. The library allocates no memory.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream). Work is only enqueued; nothing blocks the host except
- *     hga_get_device_error.
+ *     hga_get_device_error. The stream must belong to the current device
+ *     (the library's per-device state is looked up for the current device);
+ *     a stream of another device gives HGA_ERR_CUDA and launches nothing.
  *   - Arguments are validated on the host before anything is launched; a call
  *     that returns an error has launched nothing. Every data pointer must be
  *     16-byte aligned.
@@ -34,7 +36,18 @@
  *     the host. Kernels that read a caller-supplied list check every entry;
  *     an entry out of range, an entry naming a forced chunk, or a list that is
  *     not strictly ascending sets the device error word (read it with
- *     hga_get_device_error) and the entry is skipped. No kernel traps.
+ *     hga_get_device_error) and the entry is skipped: the unit computes over
+ *     its remaining keys, and every other unit of the launch, and every later
+ *     launch, computes exactly as if the word were clear (the word is only
+ *     written by kernels, never read by them). No kernel traps.
+ *   - Every device-side wait (a pipeline stage of the attention and gather
+ *     kernels) is bounded, by default by 1 s (hga_set_wait_limit_ns). A wait
+ *     that runs out records HGA_ERR_TIMEOUT in the device error word (it
+ *     overrides an invalid-entry code there), the CTA stops its work, waits
+ *     (again bounded) for the copies and tensor-core operations it has
+ *     already issued, frees its tensor memory and exits; the output rows of
+ *     the units it did not finish are undefined (not written, or computed
+ *     from part of the key set).
  *   - Layouts (row-major, innermost last):
  *       queries / outputs   [B, q_len, Hq, d]       (token q_begin + t at row t)
  *       keys / values       [B, Hkv, L, d]          (full store, HGA_KV_FULL)
@@ -261,9 +274,18 @@ hga_status hga_attend(const hga_config* cfg, const void* q_rot, const void* k_re
 const char* hga_status_string(hga_status status);
 
 /* Synchronise `stream`, then read and clear the device error word of the
- * current device. Returns HGA_OK, HGA_ERR_DEVICE_INDEX (detail_out, if not
- * NULL, receives the first offending kernel's code) or HGA_ERR_CUDA. */
+ * current device. Returns HGA_OK, HGA_ERR_TIMEOUT (a wait gave up),
+ * HGA_ERR_DEVICE_INDEX (an invalid entry; detail_out, if not NULL, receives
+ * the code of the first one recorded: 1 chunk entry, 2 group entry, 3 count;
+ * 4 = timeout) or HGA_ERR_CUDA. */
 hga_status hga_get_device_error(void* stream, int32_t* detail_out);
+
+/* Limit, in nanoseconds, of every bounded device-side wait in the launches
+ * enqueued after this call, process-wide (0 restores the default, 1 s). A
+ * healthy wait lasts microseconds; a watchdog that must report a stalled
+ * launch sooner sets a shorter limit. The drain after a give-up always uses
+ * the default limit. */
+void hga_set_wait_limit_ns(uint64_t limit_ns);
 
 /* Library version as major * 10000 + minor * 100 + patch. */
 int32_t hga_version(void);

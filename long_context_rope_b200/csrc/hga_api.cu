@@ -8,6 +8,7 @@
 // attributes have been set on which device.
 #include <math.h>
 #include <stddef.h>
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -67,6 +68,19 @@ hga_status warm_scratch(int32_t** out) {
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
+// Limit of every bounded device wait of later launches (hga_set_wait_limit_ns).
+std::atomic<unsigned long long> g_wait_ns{1000000000ull};
+
+// The per-device state (error word, scratch array) is looked up for the
+// current device, so a call's stream must belong to it.
+hga_status check_stream_device(cudaStream_t st) {
+    if (st == nullptr) return HGA_OK;  // the legacy default stream of the current device
+    int cur = 0, sdev = 0;
+    if (cudaGetDevice(&cur) != cudaSuccess || cudaStreamGetDevice(st, &sdev) != cudaSuccess)
+        return HGA_ERR_CUDA;
+    return cur == sdev ? HGA_OK : HGA_ERR_CUDA;
+}
+
 // Checks shared by every call; fills p.
 hga_status make_params(const hga_config* c, Params* p) {
     if (c == nullptr) return HGA_ERR_NULL;
@@ -121,16 +135,19 @@ hga_status make_params(const hga_config* c, Params* p) {
                              ? pow(c->rope_theta, -2.0 * (double)i / (double)c->head_dim)
                              : 0.0;
     p->err = nullptr;
+    p->wait_ns = g_wait_ns.load(std::memory_order_relaxed);
     return HGA_OK;
 }
 
 hga_status launched(cudaError_t e) { return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA; }
 
-// Last step before any launch: attach this device's error word.
-#define HGA_ATTACH_ERR(p)                                  \
-    do {                                                   \
-        hga_status es_ = error_word(&(p).err);             \
-        if (es_ != HGA_OK) return es_;                     \
+// Last step before any launch: check that the stream belongs to the current
+// device, then attach that device's error word.
+#define HGA_ATTACH_ERR(p, stream)                                              \
+    do {                                                                       \
+        hga_status es_ = check_stream_device((cudaStream_t)(stream));          \
+        if (es_ == HGA_OK) es_ = error_word(&(p).err);                         \
+        if (es_ != HGA_OK) return es_;                                         \
     } while (0)
 
 }  // namespace
@@ -167,7 +184,12 @@ static_assert(offsetof(hga_config, rope_theta) == 48, "hga_config layout is part
 
 extern "C" {
 
-int32_t hga_version(void) { return 10300; }
+int32_t hga_version(void) { return 10400; }
+
+void hga_set_wait_limit_ns(uint64_t limit_ns) {
+    g_wait_ns.store(limit_ns == 0 ? 1000000000ull : (unsigned long long)limit_ns,
+                    std::memory_order_relaxed);
+}
 
 const char* hga_status_string(hga_status s) {
     switch (s) {
@@ -198,7 +220,7 @@ hga_status hga_apply_rope(const hga_config* cfg, const void* x, void* x_rot, int
     if (n_outer * n_tokens * n_heads == 0) return HGA_OK;
     if (x == nullptr || x_rot == nullptr) return HGA_ERR_NULL;
     if (!aligned16(x) || !aligned16(x_rot)) return HGA_ERR_ALIGN;
-    HGA_ATTACH_ERR(p);
+    HGA_ATTACH_ERR(p, stream);
     return launched(launch_rope(p, x, x_rot, n_outer, n_tokens, n_heads, pos0,
                                 (cudaStream_t)stream));
 }
@@ -215,7 +237,7 @@ hga_status hga_build_summaries(const hga_config* cfg, const void* k_raw, float* 
     if (!aligned16(k_raw) || !aligned16(chunk_sum) || !aligned16(group_sum) ||
         (k_rot_out && !aligned16(k_rot_out)))
         return HGA_ERR_ALIGN;
-    HGA_ATTACH_ERR(p);
+    HGA_ATTACH_ERR(p, stream);
     return launched(launch_summaries(p, k_raw, chunk_sum, group_sum, k_rot_out, chunk_begin,
                                      chunk_end, (cudaStream_t)stream));
 }
@@ -231,7 +253,7 @@ hga_status hga_route_chunks(const hga_config* cfg, const void* q_rot, const floa
     if (!aligned16(q_rot) || !aligned16(chunk_sum) || !aligned16(qbar_out) ||
         !aligned16(sel_chunks) || !aligned16(n_sel_chunks) || (scores_out && !aligned16(scores_out)))
         return HGA_ERR_ALIGN;
-    HGA_ATTACH_ERR(p);
+    HGA_ATTACH_ERR(p, stream);
     cudaStream_t st = (cudaStream_t)stream;
     if (!route_chunks_fuses_qbar(p)) {
         cudaError_t e = launch_qbar(p, q_rot, qbar_out, st);
@@ -255,7 +277,7 @@ hga_status hga_route_groups(const hga_config* cfg, const float* qbar, const floa
         !aligned16(n_sel_chunks) || !aligned16(sel_groups) || !aligned16(n_sel_groups) ||
         (scores_out && !aligned16(scores_out)))
         return HGA_ERR_ALIGN;
-    HGA_ATTACH_ERR(p);
+    HGA_ATTACH_ERR(p, stream);
     return launched(launch_route_groups(p, qbar, group_sum, sel_chunks, n_sel_chunks, sel_groups,
                                         n_sel_groups, scores_out, (cudaStream_t)stream));
 }
@@ -301,7 +323,7 @@ hga_status hga_route(const hga_config* cfg, const void* q_rot, const float* chun
     s = check_route_args(p, q_rot, chunk_sum, group_sum, qbar_out, sel_chunks, n_sel_chunks,
                          sel_groups, n_sel_groups);
     if (s != HGA_OK) return s;
-    HGA_ATTACH_ERR(p);
+    HGA_ATTACH_ERR(p, stream);
     cudaStream_t st = (cudaStream_t)stream;
     if (decode_step_supports(p))
         return launched(launch_decode_step(p, q_rot, chunk_sum, group_sum, nullptr, nullptr,
@@ -325,7 +347,7 @@ hga_status hga_decode_step(const hga_config* cfg, const void* q_rot, const float
     if (!k_cache || !v_cache || !out) return HGA_ERR_NULL;
     if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return HGA_ERR_ALIGN;
     if (p.kv_layout != HGA_KV_FULL) return HGA_ERR_UNSUPPORTED;
-    HGA_ATTACH_ERR(p);
+    HGA_ATTACH_ERR(p, stream);
     cudaStream_t st = (cudaStream_t)stream;
     if (decode_step_supports(p))
         return launched(launch_decode_step(p, q_rot, chunk_sum, group_sum, k_cache, v_cache,
@@ -369,7 +391,7 @@ hga_status hga_gather_kv(const hga_config* cfg, const void* k_src, const void* v
     if (!aligned16(k_src) || !aligned16(v_src) || !aligned16(sel_groups) ||
         !aligned16(n_sel_groups) || !aligned16(k_dst) || !aligned16(v_dst))
         return HGA_ERR_ALIGN;
-    HGA_ATTACH_ERR(p);
+    HGA_ATTACH_ERR(p, stream);
     const void* kd = nullptr;
     const void* vd = nullptr;
     if ((s = device_view(k_src, src_is_host != 0, &kd)) != HGA_OK) return s;
@@ -398,7 +420,7 @@ hga_status hga_gather_kv_warm(const hga_config* cfg, const void* k_host, const v
     if (p.q_len != 1) return HGA_ERR_UNSUPPORTED;
     if (n_slots < p.kg || step < 0) return HGA_ERR_SHAPE;
     if (!gather_warm_supports(p, n_slots)) return HGA_ERR_UNSUPPORTED;
-    HGA_ATTACH_ERR(p);
+    HGA_ATTACH_ERR(p, stream);
     const void* kd = nullptr;
     const void* vd = nullptr;
     if ((s = device_view(k_host, true, &kd)) != HGA_OK) return s;
@@ -430,9 +452,9 @@ hga_status hga_gather_kv_warm_noalloc(const hga_config* cfg, const void* k_host,
     if (n_slots < p.kg || step < 0) return HGA_ERR_SHAPE;
     if (!gather_warm_supports(p, n_slots)) return HGA_ERR_UNSUPPORTED;
     if ((int64_t)p.B * p.Hkv * p.kg > kWarmScratchEntries) return HGA_ERR_SCRATCH_LIMIT;
+    HGA_ATTACH_ERR(p, stream);
     int32_t* src = nullptr;
     if ((s = warm_scratch(&src)) != HGA_OK) return s;
-    HGA_ATTACH_ERR(p);
     const void* kd = nullptr;
     const void* vd = nullptr;
     if ((s = device_view(k_host, true, &kd)) != HGA_OK) return s;
@@ -459,7 +481,7 @@ hga_status hga_attend(const hga_config* cfg, const void* q_rot, const void* k_re
     if (p.kv_layout == HGA_KV_WINDOWS &&
         (p.q_len != 1 || p.q_begin != p.L - 1 || k_gat == nullptr))
         return HGA_ERR_UNSUPPORTED;
-    HGA_ATTACH_ERR(p);
+    HGA_ATTACH_ERR(p, stream);
     KvSources kv{k_res, v_res, k_gat, v_gat};
     cudaStream_t st = (cudaStream_t)stream;
     if (tc_kernel_supports(p, k_gat != nullptr))
@@ -471,6 +493,7 @@ hga_status hga_attend(const hga_config* cfg, const void* q_rot, const void* k_re
 
 hga_status hga_get_device_error(void* stream, int32_t* detail_out) {
     if (detail_out) *detail_out = 0;
+    if (check_stream_device((cudaStream_t)stream) != HGA_OK) return HGA_ERR_CUDA;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return HGA_ERR_CUDA;
     int* addr = nullptr;
     hga_status s = error_word(&addr);

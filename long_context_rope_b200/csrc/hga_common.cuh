@@ -23,11 +23,14 @@ struct Params {
     int n_sink, n_local, kc, kg, F;
     int nC, q_begin, q_len, j0, nQC;
     int dtype, kv_layout;
-    int* err;                      // device error word (first error wins), never NULL
+    int* err;                      // device error word, never NULL
+    unsigned long long wait_ns;    // limit of each bounded device wait
     double inv_freq[kMaxHalfDim];  // rope_theta^(-2i/d), computed on the host in double
 };
 
-// Error codes written to the device error word (first error wins).
+// Codes written to the device error word. An invalid-entry code (1..3) is
+// recorded only while the word is 0 (the first one wins); a timeout (4)
+// always overwrites it, so a launch that gave up reports that.
 enum DevError : int {
     kDevErrNone = 0,
     kDevErrChunkIndex = 1,   // a chunk selection entry out of range / forced / not ascending
@@ -38,6 +41,10 @@ enum DevError : int {
 
 __device__ __forceinline__ void raise_dev_error(const Params& p, int code) {
     atomicCAS(p.err, 0, code);
+}
+
+__device__ __forceinline__ void raise_timeout(const Params& p) {
+    atomicExch(p.err, (int)kDevErrTimeout);
 }
 
 // Forced chunks of query chunk j in ascending order without duplicates:

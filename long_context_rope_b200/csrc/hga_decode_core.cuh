@@ -93,10 +93,10 @@ __device__ __forceinline__ bool consume_blocks(const Params& p, const uint32_t (
     for (int i = warp; i < nloc; i += kConsumers) {
         const int s = i % kStages;
         const bool got = __all_sync(
-            0xffffffffu, ptx::mbar_wait_bounded(&full[s], (i / kStages) & 1, p.err));
+            0xffffffffu, ptx::mbar_wait_bounded(&full[s], (i / kStages) & 1, p.wait_ns));
         if (!got) {
             if (lane == 0) {
-                raise_dev_error(p, kDevErrTimeout);
+                raise_timeout(p);
                 *bad = 1;
             }
             return false;
@@ -271,6 +271,21 @@ __device__ __forceinline__ void issue_block(Ring& ring, uint64_t* full, int s,
         ptx::tma_load_3d(ring.k[s] + hf * 2048, mk, hf * 64, row, outer, &full[s]);
         ptx::tma_load_3d(ring.v[s] + hf * 2048, mv, hf * 64, row, outer, &full[s]);
     }
+}
+
+// Producer thread, before the ring's memory is reused or the CTA exits:
+// waits (bounded) until every block load of the first n_issued ring slots
+// has landed. Slot i used stage i % kStages in phase i / kStages, and a stage
+// is armed again only after its previous phase completed, so the last armed
+// phase of each stage covers all of that stage's copies. False if a copy did
+// not land within the drain limit.
+__device__ __forceinline__ bool drain_ring(uint64_t* full, int n_issued) {
+    bool ok = true;
+    for (int s = 0; s < kStages && s < n_issued; ++s) {
+        const int last = s + ((n_issued - 1 - s) / kStages) * kStages;
+        ok &= ptx::mbar_drain(&full[s], last / kStages);
+    }
+    return ok;
 }
 
 }  // namespace dec

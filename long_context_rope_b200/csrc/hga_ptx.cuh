@@ -51,22 +51,35 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
-// Longest a single wait may take before the kernel gives up (1 s; a healthy
-// wait here lasts microseconds).
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
+// The limit of an ordinary wait is Params::wait_ns, set by the host
+// (hga_set_wait_limit_ns; default 1 s, where a healthy wait lasts
+// microseconds). kDrainLimitNs limits a drain: the wait, after a launch gave
+// up, for the copies and tensor-core operations it had already issued. It is
+// always the full 1 s, so a short wait limit never lets a CTA exit with a
+// copy in flight.
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
-// Wait for phase `parity` of `bar` to complete. Gives up (returns false) when
-// the wait exceeds kWaitLimitNs or when *err (the device error word, checked
-// every 256 polls) becomes non-zero because another CTA gave up.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, const int* err) {
+// Wait for phase `parity` of `bar` to complete. Gives up (returns false) only
+// when the wait exceeds limit_ns (the timer is read after every failed poll).
+// It does not look at the device error word: an invalid selection entry
+// recorded by any CTA, in this launch or an earlier one, never cuts another
+// wait short.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint64_t limit_ns) {
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 0;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 255u) {
-            if (*reinterpret_cast<const volatile int*>(err) != 0) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-        }
-    }
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    return true;
+}
+
+// Drain of one barrier that a single thread arms with arrive.expect_tx before
+// each batch of copies, and arms again only after the previous batch's phase
+// has completed: waits (kDrainLimitNs) until the last armed phase,
+// `last_phase` (0-based; < 0 = never armed), has completed, i.e. until every
+// copy counted on it has landed. False if they did not land in time.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, int last_phase) {
+    if (last_phase < 0) return true;
+    return mbar_wait_bounded(bar, (uint32_t)last_phase & 1u, kDrainLimitNs);
 }
 
 // ------------------------------------------------------ bulk (TMA) copies

@@ -94,11 +94,12 @@ __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
     if (warp == kConsumers) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
-            for (int i = 0; i < nloc; ++i) {
+            int i = 0;
+            for (; i < nloc; ++i) {
                 const int s = i % kStages;
                 if (i >= kStages &&
-                    !ptx::mbar_wait_bounded(&sm.empty[s], ((i / kStages) - 1) & 1, p.err)) {
-                    raise_dev_error(p, kDevErrTimeout);
+                    !ptx::mbar_wait_bounded(&sm.empty[s], ((i / kStages) - 1) & 1, p.wait_ns)) {
+                    raise_timeout(p);
                     sm.bad = 1;
                     break;
                 }
@@ -107,6 +108,11 @@ __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
                 const int row = rw & ~kSrcGathered;
                 dec::issue_block(sm.u.ring, sm.full, s, gat ? &maps.k_gat : &maps.k_res,
                                  gat ? &maps.v_gat : &maps.v_res, row, (int)(gat ? prob : bh));
+            }
+            // every issued load lands before the ring's memory is reused
+            if (!dec::drain_ring(sm.full, i)) {
+                raise_timeout(p);
+                sm.bad = 1;
             }
         }
     }

@@ -33,7 +33,9 @@
 // in arbitrary group order (forced chunks, then routed groups), so each
 // 128-key tile is 8 independent TMA boxes of 16 rows x 64 columns (x2).
 // Every wait is bounded; on a timeout the CTA records a device error, stops
-// its roles, drains its MMAs, frees TMEM and exits.
+// its roles, waits for the TMA loads and MMAs it has issued, frees TMEM and
+// exits. The device error word is never read here, so an invalid selection
+// entry only removes that entry's keys from its own unit.
 #include "hga_blocks.cuh"
 #include "hga_kernels.h"
 #include "hga_ptx.cuh"
@@ -97,22 +99,21 @@ __device__ __forceinline__ bool unit_at(const Params& p, int u, Unit& un) {
     return un.tok0 < p.q_begin + p.q_len && un.tok0 + 32 > p.q_begin;
 }
 
-// Bounded wait shared by the roles of one CTA: gives up after the time limit,
-// when another role of this CTA gave up (*abort), or when any CTA of the grid
-// recorded an error (*err); a give-up sets *abort so the other roles stop.
+// Bounded wait shared by the roles of one CTA: gives up after the launch's
+// wait limit or when another role of this CTA gave up (*abort); a give-up
+// sets *abort so the other roles stop. The device error word is not
+// consulted: an invalid selection entry (of this unit or any other, in this
+// launch or an earlier one) never stops a wait.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                         const int* err) {
+                                         uint64_t limit_ns) {
     const uint64_t t0 = ptx::globaltimer_ns();
-    for (uint32_t i = 0;; ++i) {
-        if (ptx::mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 255u) {
-            if (*abort || *reinterpret_cast<const volatile int*>(err) != 0 ||
-                ptx::globaltimer_ns() - t0 > ptx::kWaitLimitNs)
-                break;
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (*abort || ptx::globaltimer_ns() - t0 > limit_ns) {
+            *abort = 1;
+            return false;
         }
     }
-    *abort = 1;
-    return false;
+    return true;
 }
 
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_s, uint32_t k_s) {
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             if (!unit_at(p, u, un)) continue;
             const int bf = k & 1;
             if (k >= 2 &&
-                !__all_sync(0xffffffffu, wait_bar(&sm.list_empty[bf], ((k >> 1) - 1) & 1, abort, p.err)))
+                !__all_sync(0xffffffffu, wait_bar(&sm.list_empty[bf], ((k >> 1) - 1) & 1, abort, p.wait_ns)))
                 break;
             const int64_t prob = un.bh * p.nQC + un.jj;
             const int nb = build_key_blocks_warp(p, un.j, sel + prob * p.kg, nsel + prob, false,
@@ -212,18 +213,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     } else if (warp == 0) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
-            int k = 0, g0 = 0;
+            int k = 0, g0 = 0, nq_armed = 0;
+            int last_gk = -1, last_gv = -1;  // last tile whose K / V loads were issued
             Unit un;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
                 if (!unit_at(p, u, un)) continue;
                 const int bf = k & 1;
-                if (!wait_bar(&sm.list_full[bf], (k >> 1) & 1, abort, p.err)) break;
+                if (!wait_bar(&sm.list_full[bf], (k >> 1) & 1, abort, p.wait_ns)) break;
                 const int nb = sm.nb[bf];
                 const int n = n_tiles_of(nb);
-                if (k >= 1 && !wait_bar(&sm.q_empty, (k - 1) & 1, abort, p.err)) break;
+                if (k >= 1 && !wait_bar(&sm.q_empty, (k - 1) & 1, abort, p.wait_ns)) break;
                 const int tq = un.tok0 - p.q_begin;
                 ptx::mbar_arrive_expect_tx(&sm.bar_q, 2 * kTile);
+                ++nq_armed;
                 for (int x = 0; x < 2; ++x) {
                     ptx::tma_load_4d(sm.q[x], &maps.q, 0, un.h * 8, tq + 16 * x, un.b, &sm.bar_q);
                     ptx::tma_load_4d(sm.q[x] + kPanel, &maps.q, 64, un.h * 8, tq + 16 * x, un.b,
@@ -231,11 +234,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                 }
                 for (int t = 0; t < n; ++t) {
                     const int g = g0 + t, s = g & 1;
-                    if (g >= 2 && !wait_bar(&sm.k_empty[s], ((g >> 1) - 1) & 1, abort, p.err)) {
+                    if (g >= 2 && !wait_bar(&sm.k_empty[s], ((g >> 1) - 1) & 1, abort, p.wait_ns)) {
                         ok = false;
                         break;
                     }
                     ptx::mbar_arrive_expect_tx(&sm.k_full[s], kTile);
+                    last_gk = g;
                     for (int i = 0; i < kBlocksPerTile; ++i) {
                         const int blk = t * kBlocksPerTile + i;
                         const int row = blk < nb ? sm.blk_row[bf][blk] : p.L;  // past the end: zero fill
@@ -243,11 +247,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                         ptx::tma_load_3d(sm.k[s] + kPanel + i * 2048, &maps.k, 64, row, (int)un.bh,
                                          &sm.k_full[s]);
                     }
-                    if (g >= 2 && !wait_bar(&sm.v_empty[s], ((g >> 1) - 1) & 1, abort, p.err)) {
+                    if (g >= 2 && !wait_bar(&sm.v_empty[s], ((g >> 1) - 1) & 1, abort, p.wait_ns)) {
                         ok = false;
                         break;
                     }
                     ptx::mbar_arrive_expect_tx(&sm.v_full[s], kTile);
+                    last_gv = g;
                     for (int i = 0; i < kBlocksPerTile; ++i) {
                         const int blk = t * kBlocksPerTile + i;
                         const int row = blk < nb ? sm.blk_row[bf][blk] : p.L;
@@ -261,6 +266,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                 g0 += n;
                 ++k;
             }
+            // Drain: every tile load issued above has landed before the CTA
+            // can exit. Each barrier is armed again only after its previous
+            // phase completed, so waiting for its last armed phase covers
+            // all of its copies. (A no-op wait in a launch that did not abort.)
+            bool drained = ptx::mbar_drain(&sm.bar_q, nq_armed - 1);
+            for (int s = 0; s < 2; ++s) {
+                const int gk = last_gk - ((last_gk - s) & 1);  // last tile of stage s
+                const int gv = last_gv - ((last_gv - s) & 1);
+                drained &= ptx::mbar_drain(&sm.k_full[s], gk >= 0 ? gk >> 1 : -1);
+                drained &= ptx::mbar_drain(&sm.v_full[s], gv >= 0 ? gv >> 1 : -1);
+            }
+            if (!drained) *abort = 1;
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
@@ -272,12 +289,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
                 if (!unit_at(p, u, un)) continue;
                 const int bf = k & 1;
-                ok = wait_bar(&sm.list_full[bf], (k >> 1) & 1, abort, p.err);
+                ok = wait_bar(&sm.list_full[bf], (k >> 1) & 1, abort, p.wait_ns);
                 if (!ok) break;
                 const int n = n_tiles_of(sm.nb[bf]);
                 const int s0 = g0 & 1;
-                ok = wait_bar(&sm.bar_q, k & 1, abort, p.err) &&
-                     wait_bar(&sm.k_full[s0], (g0 >> 1) & 1, abort, p.err);
+                ok = wait_bar(&sm.bar_q, k & 1, abort, p.wait_ns) &&
+                     wait_bar(&sm.k_full[s0], (g0 >> 1) & 1, abort, p.wait_ns);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 // S_x of the previous unit was read and its P consumed by the PV
@@ -292,8 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                 for (int t = 0; ok && t < n; ++t) {
                     const int g = g0 + t, s = g & 1, s1 = (g + 1) & 1;
                     const bool more = t + 1 < n;
-                    if (!wait_bar(&sm.v_full[s], (g >> 1) & 1, abort, p.err)) { ok = false; break; }
-                    if (more && !wait_bar(&sm.k_full[s1], ((g + 1) >> 1) & 1, abort, p.err)) {
+                    if (!wait_bar(&sm.v_full[s], (g >> 1) & 1, abort, p.wait_ns)) { ok = false; break; }
+                    if (more && !wait_bar(&sm.k_full[s1], ((g + 1) >> 1) & 1, abort, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -303,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                         // P_x of this tile; for t == 0 this also orders the
                         // PV that overwrites O_x after the same warps' epilogue
                         // of the previous unit read it
-                        if (!wait_bar(&sm.p_full[x], g & 1, abort, p.err)) {
+                        if (!wait_bar(&sm.p_full[x], g & 1, abort, p.wait_ns)) {
                             ok = false;
                             break;
                         }
@@ -328,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             ptx::umma_commit(&sm.drain);
             const uint64_t t0 = ptx::globaltimer_ns();
             while (!ptx::mbar_try_wait(&sm.drain, 0) &&
-                   ptx::globaltimer_ns() - t0 < ptx::kWaitLimitNs) {
+                   ptx::globaltimer_ns() - t0 < ptx::kDrainLimitNs) {
             }
         }
     } else {
@@ -347,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
             if (!unit_at(p, u, un)) continue;
             const int bf = k & 1;
-            if (!__all_sync(0xffffffffu, wait_bar(&sm.list_full[bf], (k >> 1) & 1, abort, p.err))) {
+            if (!__all_sync(0xffffffffu, wait_bar(&sm.list_full[bf], (k >> 1) & 1, abort, p.wait_ns))) {
                 ok = false;
                 break;
             }
@@ -359,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             float m_used = -INFINITY, l = 0.f;
             for (int t = 0; t < n; ++t) {
                 const int g = g0 + t;
-                if (!__all_sync(0xffffffffu, wait_bar(&sm.s_full[x], g & 1, abort, p.err))) {
+                if (!__all_sync(0xffffffffu, wait_bar(&sm.s_full[x], g & 1, abort, p.wait_ns))) {
                     ok = false;
                     break;
                 }
@@ -451,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             }
             if (!ok) break;
             if (lane == 0) ptx::mbar_arrive(&sm.list_empty[bf]);
-            if (!__all_sync(0xffffffffu, wait_bar(&sm.o_done[x], k & 1, abort, p.err))) {
+            if (!__all_sync(0xffffffffu, wait_bar(&sm.o_done[x], k & 1, abort, p.wait_ns))) {
                 ok = false;
                 break;
             }
@@ -500,8 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         ptx::tc_fence_before();
     }
     __syncthreads();
-    if (*abort && tid == 0 && *reinterpret_cast<volatile int*>(p.err) == 0)
-        raise_dev_error(p, kDevErrTimeout);
+    if (*abort && tid == 0) raise_timeout(p);
     if (warp == 1) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, kTmemCols);

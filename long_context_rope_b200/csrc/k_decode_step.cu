@@ -382,15 +382,22 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     __syncthreads();
     if (warp == kConsumers) {
         if (lane == 0) {
-            for (int i = n_pre; i < nloc; ++i) {
+            int i = n_pre;
+            for (; i < nloc; ++i) {
                 const int s = i % kStages;
                 if (i >= kStages &&
-                    !ptx::mbar_wait_bounded(&sm.empty[s], ((i / kStages) - 1) & 1, p.err)) {
-                    raise_dev_error(p, kDevErrTimeout);
+                    !ptx::mbar_wait_bounded(&sm.empty[s], ((i / kStages) - 1) & 1, p.wait_ns)) {
+                    raise_timeout(p);
                     sm.bad = 1;
                     break;
                 }
                 dec::issue_block(sm.u.ring, sm.full, s, &maps.k, &maps.v, sm.blk_pos[i], (int)bh);
+            }
+            // every issued load (the early forced blocks included) lands
+            // before the ring's memory is reused
+            if (!dec::drain_ring(sm.full, i)) {
+                raise_timeout(p);
+                sm.bad = 1;
             }
         }
     }

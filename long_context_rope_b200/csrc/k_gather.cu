@@ -71,8 +71,11 @@ __global__ void __launch_bounds__(32) gather_hbm_kernel(Params p, const char* __
         ptx::bulk_g2s(sk, k_src + off, blk, &bar);
         ptx::bulk_g2s(sk + blk, v_src + off, blk, &bar);
     }
-    if (!ptx::mbar_wait_bounded(&bar, 0, p.err)) {
-        raise_dev_error(p, kDevErrTimeout);
+    if (!ptx::mbar_wait_bounded(&bar, 0, p.wait_ns)) {
+        // gave up: wait once more (drain limit) for the copies already issued
+        // into this CTA's shared memory, then exit without storing
+        raise_timeout(p);
+        ptx::mbar_drain(&bar, 0);
         return;
     }
     const int64_t dst_base = prob * (int64_t)p.kg * blk;

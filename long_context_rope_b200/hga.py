@@ -95,6 +95,8 @@ def _load():
     lib.hga_status_string.argtypes = [ctypes.c_int]
     lib.hga_status_string.restype = ctypes.c_char_p
     lib.hga_version.restype = ctypes.c_int32
+    lib.hga_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.hga_set_wait_limit_ns.restype = None
     return lib
 
 
@@ -335,6 +337,11 @@ def get_device_error(stream=None) -> int:
     if st == -5:
         raise HgaError(st, "hga_get_device_error")
     return int(detail.value) if st != HGA_OK else 0
+
+
+def set_wait_limit_ns(limit_ns: int) -> None:
+    """Limit of every bounded device wait of later launches (0 = default 1 s)."""
+    _lib.hga_set_wait_limit_ns(int(limit_ns))
 
 
 def version() -> int:

@@ -11,7 +11,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def _declared():
     text = open(os.path.join(ROOT, "include", "hga.h")).read()
-    return sorted(set(re.findall(r"^\s*(?:hga_status|const char\*|int32_t)\s+(hga_\w+)\s*\(",
+    return sorted(set(re.findall(r"^\s*(?:hga_status|const char\*|int32_t|void)\s+(hga_\w+)\s*\(",
                                  text, flags=re.M)))
 
 

@@ -7,8 +7,9 @@ device-wide synchronisation of cudaFree). Its plan-to-copy scratch is a fixed
 The GPU test runs two calls in a row on one pool through the new entry point
 and on a second, identical pool through hga_gather_kv_warm, and requires the
 same gathered K/V (bitwise, as for every gather test: the call copies), pool
-contents, tags, last-use steps and hit / miss counts after each call. The
-second call finds the first call's contents in the scratch array.
+contents, tags, last-use steps and hit / miss counts after each call. All
+calls go on one explicit stream, so the second call is ordered after the
+first and finds the first call's contents in the scratch array.
 
 This file is named so that pytest collects it last."""
 import ctypes
@@ -83,6 +84,13 @@ def test_noalloc_matches_warm_gather_on_two_calls_in_a_row(hga):
     v_host = x["v"].pin_memory()
     S = 128
     ref, new = pipeline.alloc_warm_pool(cfg, S), pipeline.alloc_warm_pool(cfg, S)
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):  # every call below: this one stream
+        _two_calls(hga, pipeline, w, cfg, x, q_second, cs, gs, k_host, v_host, ref, new)
+
+
+def _two_calls(hga, pipeline, w, cfg, x, q_second, cs, gs, k_host, v_host, ref, new):
     for step, q_raw in enumerate((x["q_raw"], q_second)):
         q_rot = pipeline.rotate_queries(cfg, q_raw.cuda())
         rb = pipeline.alloc_route(cfg)
@@ -94,8 +102,7 @@ def test_noalloc_matches_warm_gather_on_two_calls_in_a_row(hga):
         hga.gather_kv_warm_noalloc(cfg, k_host, v_host, rb.sel_groups, rb.n_sel_groups, new.k,
                                    new.v, new.tag, new.last, step, g_new[0], g_new[1],
                                    stats=new.stats)
-        torch.cuda.synchronize()
-        assert hga.get_device_error() == 0
+        assert hga.get_device_error() == 0  # synchronises the current (explicit) stream
         n = rb.n_sel_groups.cpu().reshape(-1)
         assert int(n.min()) > 0
         for u in range(w.batch * w.n_kv_heads):
