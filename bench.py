@@ -24,7 +24,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from long_context_rope_b200 import synth  # noqa: E402
+from long_context_rope_b200 import dist_util, synth  # noqa: E402
 
 METRIC = "routed attn prefill tok/s & decode µs/step at 64K; % of HBM/TC roofline"
 
@@ -48,39 +48,6 @@ def load_peaks():
                     tc_sustained=float(pk["bf16_tflops_sustained"]), src="measured")
     except Exception:
         return dict(hbm=6650.0, tc=1590.0, tc_sustained=1400.0, src="fallback")
-
-
-# ------------------------------------------------------------ distributed
-class Dist:
-    def __init__(self, n_gpus: int):
-        self.world = int(os.environ.get("WORLD_SIZE", "1"))
-        self.rank = int(os.environ.get("RANK", "0"))
-        self.local = int(os.environ.get("LOCAL_RANK", "0"))
-        self.pg = None
-        if self.world > 1:
-            import datetime
-            import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
-            self.pg = dist
-        else:
-            torch.cuda.set_device(0)
-
-    def barrier(self):
-        if self.pg:
-            self.pg.barrier()
-
-    def max(self, x: float) -> float:
-        if not self.pg:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
-        return float(t.item())
-
-    def close(self):
-        if self.pg:
-            self.pg.destroy_process_group()
 
 
 # ------------------------------------------------------------------ clocks
@@ -188,7 +155,7 @@ def run_prefill(args, dist, peaks):
     from long_context_rope_b200 import hga, pipeline
     w = synth.WORKLOADS[args.workload]
     cfg = hga.config_from(w)
-    seed = synth.seed_for_rank(args.seed, dist.rank)
+    seed = dist.seed(args.seed)
     x = synth.draw(w, seed=seed)
     dev = torch.device("cuda", torch.cuda.current_device())
     st = torch.cuda.current_stream()
@@ -284,7 +251,7 @@ def run_decode(name, args, dist):
     from long_context_rope_b200 import hga, pipeline
     w = synth.WORKLOADS[name]
     cfg = hga.config_from(w)
-    x = synth.draw(w, seed=synth.seed_for_rank(args.seed, dist.rank))
+    x = synth.draw(w, seed=dist.seed(args.seed))
     dev = torch.device("cuda", torch.cuda.current_device())
     st = torch.cuda.current_stream()
     k_raw = x["k_raw"].to(dev)
@@ -498,7 +465,7 @@ def main():
         print(json.dumps(line), flush=True)
         return
 
-    dist = Dist(args.gpus)
+    dist = dist_util.Dist("nccl")
     try:
         pre = run_prefill(args, dist, peaks)
         decodes = []

@@ -1,12 +1,12 @@
-"""World-size-2 gloo test of the weak-scaling host logic: each rank draws its
-own sequence (different seeds), times are reduced with a max over ranks, and
-the whole-job rate counts every rank's tokens."""
+"""World-size-2 gloo test of the weak-scaling host logic that bench.py runs
+(long_context_rope_b200.dist_util.Dist, with gloo instead of NCCL): the
+process group comes up from the torchrun environment variables, each rank
+draws its own sequence (different seeds), the barrier passes, times are
+reduced with a max over ranks, and the whole-job rate counts every rank's
+tokens."""
 import os
 import socket
 
-import pytest
-import torch
-import torch.distributed as dist
 import torch.multiprocessing as mp
 
 
@@ -19,20 +19,21 @@ def _free_port():
 
 
 def _worker(rank, world, port, q):
-    os.environ["MASTER_ADDR"] = "127.0.0.1"
-    os.environ["MASTER_PORT"] = str(port)
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      LOCAL_RANK=str(rank), WORLD_SIZE=str(world))
+    from long_context_rope_b200 import dist_util, synth
+    d = dist_util.Dist("gloo", timeout_s=60)
     try:
-        from long_context_rope_b200 import dist_util, synth
-        seed = dist_util.rank_seed(0)
+        seed = d.seed(0)
         w = synth.WORKLOADS["tiny_f32"]
         x = synth.draw(w, seed=seed)
         first = float(x["k_raw"][0, 0, 0, 0])
-        t = dist_util.max_over_ranks(1.0 + rank)
-        rate = dist_util.whole_job_rate(w.seq_len, t, world)
-        q.put((rank, seed, first, t, rate))
+        d.barrier()
+        t = d.max(1.0 + rank)
+        rate = dist_util.whole_job_rate(w.seq_len, t, d.world)
+        q.put((d.rank, seed, first, t, rate))
     finally:
-        dist.destroy_process_group()
+        d.close()
 
 
 def test_weak_scaling_host_logic_gloo():
@@ -47,6 +48,18 @@ def test_weak_scaling_host_logic_gloo():
         p.join(timeout=60)
         assert p.exitcode == 0
     (r0, s0, f0, t0, rate0), (r1, s1, f1, t1, rate1) = res
+    assert (r0, r1) == (0, 1)
     assert s0 != s1 and f0 != f1          # independent sequences
     assert t0 == t1 == 2.0                # max over ranks
     assert rate0 == rate1 == 2 * 1024 / 2.0
+
+
+def test_single_process_is_identity(monkeypatch):
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    from long_context_rope_b200 import dist_util
+    d = dist_util.Dist("gloo")
+    assert (d.world, d.rank, d.active) == (1, 0, False)
+    assert d.max(3.5) == 3.5
+    d.barrier()
+    d.close()

@@ -3,8 +3,9 @@
 Every input comes from the seeded generator; each side computes every
 intermediate itself (the oracle never receives a value the GPU produced).
 Stages compared: rotated queries and keys, chunk and group summaries, q-bar,
-routing scores, selections (with the near-tie exemption), and outputs on
-the units whose routing agrees. Tolerances: tests/parity_util.py.
+routing scores, selections (with the near-tie exemption; groups on the GPU's
+own chunk selection), and the outputs of every unit (on the GPU's own
+selection where routing differs). Tolerances: tests/parity_util.py.
 """
 import numpy as np
 import pytest
@@ -12,8 +13,7 @@ import torch
 
 from long_context_rope_b200 import synth
 from oracle import hga_oracle as O
-from parity_util import (OUT_TOL, assert_close, check_chunk_selection_matches_own_scores,
-                         check_group_selection_matches_own_scores, compare_selections)
+from parity_util import assert_close, compare_outputs, compare_routing
 
 pytestmark = pytest.mark.gpu
 
@@ -74,74 +74,13 @@ def run_gpu_prefill(w, x, r=None):
                 out=_np(out))
 
 
-def compare_routing(w, g, r):
-    """Stage-by-stage routing parity. Returns the boolean mask (per problem)
-    of identical group selections."""
-    kc, kg, G = w.top_k_chunks, w.top_k_groups, w.groups_per_chunk
-    # scores of every candidate; NaN marks non-candidates identically
-    assert np.array_equal(np.isnan(g["chunk_scores"]), np.isnan(r["chunk_scores"]))
-    rs = np.nan_to_num(r["chunk_scores"])
-    scale = np.abs(rs).max(axis=-1, keepdims=True) + 1e-6
-    assert_close("chunk scores / scale", np.nan_to_num(g["chunk_scores"]) / scale, rs / scale,
-                 atol=2e-5)
-    rsc = r["chunk_scores"].reshape(-1, r["chunk_scores"].shape[-1])
-    same_c = compare_selections("chunks", g["sel_chunks"], g["n_sel_chunks"], r["sel_chunks"],
-                                r["n_sel_chunks"], lambda p, x: rsc[p, x])
-    check_chunk_selection_matches_own_scores(g["sel_chunks"], g["n_sel_chunks"],
-                                             g["chunk_scores"], kc)
-    check_group_selection_matches_own_scores(g["sel_groups"], g["n_sel_groups"],
-                                             g["group_scores"], g["sel_chunks"],
-                                             g["n_sel_chunks"], G, kg)
-    # groups: where the chunk selections agree, the candidate lists agree
-    rgs = r["group_scores"].reshape(-1, r["group_scores"].shape[-1])
-    ggs = g["group_scores"].reshape(-1, g["group_scores"].shape[-1])
-    rsel_c = r["sel_chunks"].reshape(-1, kc)
-    idx = np.flatnonzero(same_c)
-    assert np.array_equal(np.isnan(ggs[idx]), np.isnan(rgs[idx]))
-    gscale = np.abs(np.nan_to_num(rgs[idx])).max(axis=-1, keepdims=True) + 1e-6
-    assert_close("group scores / scale", np.nan_to_num(ggs[idx]) / gscale,
-                 np.nan_to_num(rgs[idx]) / gscale, atol=2e-5)
-
-    def ref_group_score(p, gi):
-        pos = list(rsel_c[p]).index(gi // G) * G + gi % G
-        return rgs[p, pos]
-
-    gsg = g["sel_groups"].reshape(-1, kg)[idx]
-    gng = g["n_sel_groups"].reshape(-1)[idx]
-    rsg = r["sel_groups"].reshape(-1, kg)[idx]
-    rng_ = r["n_sel_groups"].reshape(-1)[idx]
-    same_g_sub = compare_selections("groups", gsg, gng, rsg, rng_,
-                                    lambda p, x: ref_group_score(idx[p], x))
-    same = np.zeros_like(same_c)
-    same[idx[same_g_sub]] = True
-    assert same.mean() >= 0.99, f"only {same.mean():.3f} of problems route identically"
-    return same
-
-
-def compare_outputs(w, g_out, r_out, same, units=None):
-    """Max-abs parity of the outputs of the units whose routing agrees."""
-    B, H, C, gq = w.batch, w.n_kv_heads, w.chunk_size, w.n_q_heads // w.n_kv_heads
-    j0 = w.q_begin // C
-    nQC = (w.q_begin + w.q_len - 1) // C - j0 + 1
-    if units is None:
-        units = [(b, h, jj) for b in range(B) for h in range(H) for jj in range(nQC)]
-    tol = OUT_TOL[w.dtype]
-    worst = 0.0
-    n_cmp = 0
-    for (b, h, jj) in units:
-        if not same[(b * H + h) * nQC + jj]:
-            continue
-        j = j0 + jj
-        t0 = max(j * C, w.q_begin) - w.q_begin
-        t1 = min((j + 1) * C, w.q_begin + w.q_len) - w.q_begin
-        gg = g_out[b, t0:t1, h * gq:(h + 1) * gq]
-        rr = r_out[b, t0:t1, h * gq:(h + 1) * gq]
-        assert np.isfinite(gg).all()
-        worst = max(worst, float(np.abs(gg - rr).max()))
-        n_cmp += 1
-    assert n_cmp > 0
-    assert worst <= tol, f"max abs error {worst} > {tol}"
-    return worst
+def _oracle_on_gpu_selection(w, r, v, g):
+    """The oracle's attention (its own bf16 rotations) over the GPU's own
+    group selection, for the given units."""
+    def run(units):
+        return O.attend(O.cfg_of(w), r["q_rot"], r["k_rot"], v, g["sel_groups"],
+                        g["n_sel_groups"], units=np.array(units, dtype=np.int32))
+    return run
 
 
 def compare_prefill(w, x, units=None):
@@ -154,10 +93,15 @@ def compare_prefill(w, x, units=None):
     assert_close("chunk_sum", g["chunk_sum"], r["chunk_sum"], atol=2e-5, rtol=2e-5)
     assert_close("group_sum", g["group_sum"], r["group_sum"], atol=2e-5, rtol=2e-5)
     assert_close("qbar", g["qbar"], r["qbar"], atol=2e-5, rtol=2e-5)
-    same = compare_routing(w, g, r)
-    if units is not None:
-        units = [tuple(u) for u in units]
-    return compare_outputs(w, g["out"], r["out"], same, units)
+    same = compare_routing(w, g, r, O)
+    assert same.mean() >= 0.99, f"only {same.mean():.3f} of problems route identically"
+    worst, n_alt = compare_outputs(w, g["out"], r["out"], same,
+                                   _oracle_on_gpu_selection(w, r, _np_v(x), g), units)
+    return worst
+
+
+def _np_v(x):
+    return x["v"].float().numpy()
 
 
 @pytest.mark.parametrize("name", ["tiny_f32", "prefill_4k"])
@@ -169,19 +113,34 @@ def test_prefill_parity_full(name):
 
 
 def test_prefill_end_to_end_from_raw_inputs():
-    """Everything from the raw drawn inputs on both sides (each rotates its own
-    queries and keys). bf16 rounding-boundary flips between the fp32 and the
-    double rotation may move a near-tied routing decision, so this test asks
-    for >= 98% identical routing and checks outputs where routing agrees."""
+    """Everything from the raw drawn inputs on both sides: each side rotates
+    its own queries and keys, so the GPU's q-bar differs from the oracle's by
+    the bf16 rounding flips of its fp32 rotation (each at most one bf16 ulp,
+    checked here). Every routing decision that differs from the oracle's must
+    be explained by that input difference: the two oracle scores of each
+    swapped pair lie within the near-tie band plus the score perturbation the
+    measured q-bar and summary differences can cause (score_slack, which
+    also bounds the GPU's score of every candidate). Groups are compared on
+    the GPU's chunk selection (the oracle re-run on it); every unit's output
+    is compared, on the GPU's selection where it differs."""
     w = synth.WORKLOADS["prefill_4k"]
     x = synth.draw(w, seed=2)
     r = O.pipeline(w, x)
     g = run_gpu_prefill(w, x)
-    same = (g["sel_groups"] == r["sel_groups"]).all(-1) & (g["n_sel_groups"] == r["n_sel_groups"])
-    same &= (g["sel_chunks"] == r["sel_chunks"]).all(-1)
-    assert same.mean() >= 0.98, same.mean()
-    worst = compare_outputs(w, g["out"], r["out"], same.reshape(-1))
-    print(f"end-to-end: {same.mean():.4f} identical routing, max abs error {worst:.3e}")
+    bf16_ulp_check("q_rot", g["q_rot"], r["q_rot"])
+    bf16_ulp_check("k_rot", g["k_rot"], r["k_rot"])
+    assert_close("chunk_sum", g["chunk_sum"], r["chunk_sum"], atol=2e-5, rtol=2e-5)
+    assert_close("group_sum", g["group_sum"], r["group_sum"], atol=2e-5, rtol=2e-5)
+    same = compare_routing(w, g, r, O, slack=True)
+    assert same.mean() >= 0.95, same.mean()
+
+    def oracle_alt(units):  # the oracle's rotations, the GPU's selection
+        return O.attend(O.cfg_of(w), r["q_rot"], r["k_rot"], _np_v(x), g["sel_groups"],
+                        g["n_sel_groups"], units=np.array(units, dtype=np.int32))
+
+    worst, n_alt = compare_outputs(w, g["out"], r["out"], same, oracle_alt)
+    print(f"end-to-end: {same.mean():.4f} identical routing ({n_alt} units on the GPU's "
+          f"selection), max abs error {worst:.3e}")
 
 
 @pytest.mark.parametrize("L,F,dtype", [(1000, 32, "bf16"), (16 * 64 + 16 * 5 + 3, 7, "bf16"),
@@ -253,13 +212,17 @@ def _decode_setup(w, x, r):
     return cfg, cs, gs, k_rot, q_rot
 
 
-def _decode_compare(w, r, g_out, rb):
-    g = dict(sel_chunks=_np(rb.sel_chunks), n_sel_chunks=_np(rb.n_sel_chunks),
+def _decode_compare(w, x, r, g_out, rb, cs, gs):
+    g = dict(qbar=_np(rb.qbar), chunk_sum=_np(cs), group_sum=_np(gs),
+             sel_chunks=_np(rb.sel_chunks), n_sel_chunks=_np(rb.n_sel_chunks),
              chunk_scores=_np(rb.chunk_scores), sel_groups=_np(rb.sel_groups),
              n_sel_groups=_np(rb.n_sel_groups), group_scores=_np(rb.group_scores))
-    assert_close("qbar", _np(rb.qbar), r["qbar"], atol=2e-5, rtol=2e-5)
-    same = compare_routing(w, g, r)
-    return compare_outputs(w, _np(g_out), r["out"], same)
+    assert_close("qbar", g["qbar"], r["qbar"], atol=2e-5, rtol=2e-5)
+    same = compare_routing(w, g, r, O)
+    assert same.mean() >= 0.99, same.mean()
+    worst, _ = compare_outputs(w, _np(g_out), r["out"], same,
+                               _oracle_on_gpu_selection(w, r, _np_v(x), g))
+    return worst
 
 
 @pytest.mark.parametrize("mode", ["index", "gathered"])
@@ -279,7 +242,7 @@ def test_decode_16x32k(mode):
         pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out, gathered=gat, k_src=k_rot,
                         v_src=v)
     assert hga.get_device_error() == 0
-    worst = _decode_compare(w, r, out, rb)
+    worst = _decode_compare(w, x, r, out, rb, cs, gs)
     print(f"decode {mode}: max abs error {worst:.3e}")
 
 
@@ -307,7 +270,7 @@ def test_tiered_decode_4x64k():
     pipeline.decode(cfg_w, q_rot, cs, gs, k_win, v_win, rb, out, gathered=gat, k_src=k_host,
                     v_src=v_host, src_is_host=True)
     assert hga.get_device_error() == 0
-    worst = _decode_compare(w, r, out, rb)
+    worst = _decode_compare(w, x, r, out, rb, cs, gs)
     print(f"tiered decode: max abs error {worst:.3e}")
 
 

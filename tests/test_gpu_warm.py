@@ -3,7 +3,9 @@ routed groups between the host store and attention.
 
 Over a sequence of decode queries (repeats, new routes, evictions from a
 pool smaller than two routes) every call must give bitwise the same gathered
-K/V as the cold gather from host memory, the same attention output, and pool
+K/V as the cold gather from host memory, the same attention output (and that
+output within the bf16 tolerance of the CPU oracle's attention over the same
+selection, from the oracle's own rotations), and pool
 tags, last-use steps and hit / miss counts equal to a plain-Python model of
 the rule: hits keep their slots; the i-th miss in list order takes the i-th
 victim, victims being the slots not hit this call with the oldest last use
@@ -13,6 +15,8 @@ import pytest
 import torch
 
 from long_context_rope_b200 import synth
+from oracle import hga_oracle as O
+from parity_util import OUT_TOL
 
 pytestmark = pytest.mark.gpu
 
@@ -59,6 +63,13 @@ def test_warm_tier_matches_cold_gather_and_lru_model():
     S = 128  # smaller than two routes of 96 groups: evictions happen
     pool = pipeline.alloc_warm_pool(cfg, S)
     sels = {}
+    # the oracle's own bf16 rotations of the keys and of each query
+    ocfg = O.cfg_of(w)
+    ref = O.pipeline(w, x, want_scores=False, attend_out=False)
+    q_ref = [np.stack([O.rope_f32(ocfg, q[b].float().numpy(), ocfg.q_begin, True)
+                       for b in range(w.batch)]) for q in queries]
+    v_np = x["v"].float().numpy()
+    worst = 0.0
     for step, qi in enumerate(order):
         q_rot = pipeline.rotate_queries(cfg, queries[qi].cuda())
         rb = pipeline.alloc_route(cfg)
@@ -81,6 +92,12 @@ def test_warm_tier_matches_cold_gather_and_lru_model():
             sel = rb.sel_groups[b, h, 0, :n[u]].tolist()
             sels.setdefault(u, []).append(sel)
         assert torch.equal(out_w, out_c), step
+        # the oracle's attention over the GPU's own selection of this step
+        r_out = O.attend(ocfg, q_ref[qi], ref["k_rot"], v_np, rb.sel_groups.cpu().numpy(),
+                         rb.n_sel_groups.cpu().numpy())
+        err = float(np.abs(out_w.float().cpu().numpy() - r_out).max())
+        assert err <= OUT_TOL["bf16"], (step, err)
+        worst = max(worst, err)
         model_stats = pool.stats.cpu().numpy().reshape(-1, 2)
         tags, last = pool.tag.cpu().numpy(), pool.last.cpu().numpy()
         for u in range(w.batch * w.n_kv_heads):
@@ -93,3 +110,4 @@ def test_warm_tier_matches_cold_gather_and_lru_model():
               f"{model_stats[:, 1].sum()}")
     st = _lru_model(S, sels[0])
     assert st[1][1] == 0, "a repeated query must hit every group"
+    print(f"warm tier vs oracle on the GPU's selections: max abs error {worst:.3e}")
