@@ -60,16 +60,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
 // Wait for phase `parity` of `bar` to complete. Gives up (returns false) only
-// when the wait exceeds limit_ns (the timer is read after every failed poll).
-// It does not look at the device error word: an invalid selection entry
-// recorded by any CTA, in this launch or an earlier one, never cuts another
-// wait short.
+// when the wait exceeds limit_ns (the timer is read every 8 polls). It does
+// not look at the device error word: an invalid selection entry recorded by
+// any CTA, in this launch or an earlier one, never cuts another wait short.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint64_t limit_ns) {
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (globaltimer_ns() - t0 > limit_ns) return false;
-    return true;
+    for (uint32_t i = 0;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 7u) == 7u && globaltimer_ns() - t0 > limit_ns) return false;
+    }
 }
 
 // Drain of one barrier that a single thread arms with arrive.expect_tx before
@@ -107,6 +107,13 @@ __device__ __forceinline__ void bulk_commit() {
 
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Wait until at most N of this thread's committed bulk groups are still
+// reading their shared-memory source (their global writes may be pending).
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 
 // ------------------------------------------------ tensor-map (TMA) tiles

@@ -101,19 +101,18 @@ __device__ __forceinline__ bool unit_at(const Params& p, int u, Unit& un) {
 
 // Bounded wait shared by the roles of one CTA: gives up after the launch's
 // wait limit or when another role of this CTA gave up (*abort); a give-up
-// sets *abort so the other roles stop. The device error word is not
-// consulted: an invalid selection entry (of this unit or any other, in this
-// launch or an earlier one) never stops a wait.
+// sets *abort so the other roles stop. Both are checked every 8 polls. The
+// device error word is not consulted: an invalid selection entry (of this
+// unit or any other, in this launch or an earlier one) never stops a wait.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort,
                                          uint64_t limit_ns) {
     const uint64_t t0 = ptx::globaltimer_ns();
-    while (!ptx::mbar_try_wait(bar, parity)) {
-        if (*abort || ptx::globaltimer_ns() - t0 > limit_ns) {
-            *abort = 1;
-            return false;
-        }
+    for (uint32_t i = 0;; ++i) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((i & 7u) == 7u && (*abort || ptx::globaltimer_ns() - t0 > limit_ns)) break;
     }
-    return true;
+    *abort = 1;
+    return false;
 }
 
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_s, uint32_t k_s) {

@@ -6,8 +6,8 @@
 // (cold tier: the full K/V history in host RAM).
 //
 // HBM source: each 16-row group of K and of V is one contiguous block
-// (16 * d elements); one thread issues bulk (TMA) copies global -> shared for
-// SLOTS groups, waits on one mbarrier, then bulk-stores shared -> global.
+// (16 * d elements); per CTA one thread streams its groups through a ring of
+// shared-memory stages with bulk (TMA) loads and bulk stores.
 // Host source: the pinned host store is read with 16-byte loads through its
 // device mapping (zero-copy over the host link); every thread keeps several
 // loads in flight.
@@ -20,8 +20,6 @@ namespace hga {
 
 namespace {
 
-constexpr int kSlotsPerCta = 8;
-
 __device__ __forceinline__ int checked_count(const Params& p, const int32_t* n_sel, int64_t prob) {
     int n = n_sel[prob];
     if (n < 0 || n > p.kg) {
@@ -31,61 +29,111 @@ __device__ __forceinline__ int checked_count(const Params& p, const int32_t* n_s
     return n;
 }
 
-// Grid (ceil(kg / SLOTS), nQC, B*Hkv); one warp; lane 0 drives the copies.
+// HBM source. The copy units are the selection slots of all problems,
+// flattened (unit = problem * kg + slot); CTA c takes the contiguous range
+// [c * per, (c + 1) * per). Lanes first validate their units' selection
+// entries in parallel; then lane 0 runs a ring of kGatherStages shared-memory
+// stages: bulk (TMA) loads of a group's K and V block into a stage, counted
+// on the stage's mbarrier, and bulk stores from the stage to the compact
+// buffers, one bulk group per unit. kGatherStages - 1 loads are in flight
+// while the oldest landed stage is stored; a stage is loaded again only
+// after the store that last read it has finished reading.
+constexpr int kGatherStages = 6;
+constexpr int kGatherUnitsMax = 64;   // units of one CTA (per <= this)
+
 __global__ void __launch_bounds__(32) gather_hbm_kernel(Params p, const char* __restrict__ k_src,
                                                         const char* __restrict__ v_src,
                                                         const int32_t* __restrict__ sel,
                                                         const int32_t* __restrict__ nsel,
                                                         char* __restrict__ k_dst,
-                                                        char* __restrict__ v_dst) {
+                                                        char* __restrict__ v_dst, int per) {
     extern __shared__ __align__(128) char buf[];
-    __shared__ __align__(8) uint64_t bar;
-    if (threadIdx.x != 0) return;
-    const int jj = blockIdx.y;
-    const int64_t bh = blockIdx.z;
-    const int j = p.j0 + jj;
-    const int64_t prob = bh * p.nQC + jj;
+    __shared__ __align__(8) uint64_t full[kGatherStages];
+    __shared__ int64_t src_off[kGatherUnitsMax], dst_off[kGatherUnitsMax];
+    const int lane = threadIdx.x;
     const int es = p.dtype == HGA_BF16 ? 2 : 4;
     const uint32_t blk = (uint32_t)(kGroupRows * p.d * es);
-    const int n = checked_count(p, nsel, prob);
-    const int s_lo = blockIdx.x * kSlotsPerCta;
-    const int s_hi = s_lo + kSlotsPerCta < n ? s_lo + kSlotsPerCta : n;
-    if (s_lo >= s_hi) return;
-    const int32_t* list = sel + prob * p.kg;
-    int gi[kSlotsPerCta];
-    uint32_t bytes = 0;
-    for (int s = s_lo; s < s_hi; ++s) {
-        gi[s - s_lo] = checked_group_entry(p, j, list, s);
-        if (gi[s - s_lo] >= 0) bytes += 2 * blk;
+    const int64_t total = (int64_t)p.B * p.Hkv * p.nQC * p.kg;
+    const int64_t u0 = (int64_t)blockIdx.x * per;
+    // validate this CTA's units; compact the valid ones, in unit order
+    int n = 0;
+    for (int i0 = 0; i0 < per; i0 += 32) {
+        const int64_t u = u0 + i0 + lane;
+        bool ok = false;
+        int64_t so = 0, dof = 0;
+        if (i0 + lane < per && u < total) {
+            const int64_t prob = u / p.kg;
+            const int s = (int)(u % p.kg);
+            const int64_t bh = prob / p.nQC;
+            const int j = p.j0 + (int)(prob % p.nQC);
+            // the count and the two list entries are independent loads (one
+            // round trip); a bad count is recorded once, by the slot-0 unit
+            const int32_t* list = sel + prob * p.kg;
+            const int n_raw = nsel[prob];
+            const int gi = list[s];
+            const int prev = s > 0 ? list[s - 1] : -1;
+            if (s == 0 && (n_raw < 0 || n_raw > p.kg)) raise_dev_error(p, kDevErrCount);
+            const int cnt = min(max(n_raw, 0), p.kg);
+            if (s < cnt) {
+                const int c = gi >= 0 ? gi / p.G : -1;
+                if (gi >= 0 && c < j && !is_forced(p, j, c) && (s == 0 || gi > prev)) {
+                    ok = true;
+                    so = bh * (int64_t)p.L * p.d * es + (int64_t)gi * blk;
+                    dof = u * (int64_t)blk;
+                } else {
+                    raise_dev_error(p, kDevErrGroupIndex);
+                }
+            }
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, ok);
+        if (ok) {
+            const int at = n + __popc(m & ((1u << lane) - 1u));
+            src_off[at] = so;
+            dst_off[at] = dof;
+        }
+        n += __popc(m);
     }
-    if (bytes == 0) return;
-    ptx::mbar_init(&bar, 1);
+    __syncwarp();
+    if (lane != 0 || n == 0) return;
+    for (int s = 0; s < kGatherStages; ++s) ptx::mbar_init(&full[s], 1);
     ptx::fence_mbar_init();
-    ptx::mbar_arrive_expect_tx(&bar, bytes);
-    const int64_t src_base = bh * (int64_t)p.L * p.d * es;
-    for (int s = s_lo; s < s_hi; ++s) {
-        const int g = gi[s - s_lo];
-        if (g < 0) continue;
-        const int64_t off = src_base + (int64_t)g * blk;
-        char* sk = buf + (size_t)(s - s_lo) * 2 * blk;
-        ptx::bulk_g2s(sk, k_src + off, blk, &bar);
-        ptx::bulk_g2s(sk + blk, v_src + off, blk, &bar);
+    auto load = [&](int i) {
+        char* st = buf + (size_t)(i % kGatherStages) * 2 * blk;
+        uint64_t* bar = &full[i % kGatherStages];
+        ptx::mbar_arrive_expect_tx(bar, 2 * blk);
+        ptx::bulk_g2s(st, k_src + src_off[i], blk, bar);
+        ptx::bulk_g2s(st + blk, v_src + src_off[i], blk, bar);
+    };
+    int loaded = 0;
+    for (; loaded < kGatherStages - 1 && loaded < n; ++loaded) load(loaded);
+    bool ok = true;
+    for (int i = 0; i < n; ++i) {
+        const int s = i % kGatherStages;
+        if (!ptx::mbar_wait_bounded(&full[s], (uint32_t)(i / kGatherStages) & 1u, p.wait_ns)) {
+            ok = false;
+            break;
+        }
+        char* st = buf + (size_t)s * 2 * blk;
+        ptx::bulk_s2g(k_dst + dst_off[i], st, blk);
+        ptx::bulk_s2g(v_dst + dst_off[i], st + blk, blk);
+        ptx::bulk_commit();
+        if (loaded < n) {
+            // the stage of unit `loaded` last held unit loaded - kGatherStages
+            // = i - 1, whose store is the second newest bulk group
+            if (loaded >= kGatherStages) ptx::bulk_wait_read<1>();
+            load(loaded);
+            ++loaded;
+        }
     }
-    if (!ptx::mbar_wait_bounded(&bar, 0, p.wait_ns)) {
-        // gave up: wait once more (drain limit) for the copies already issued
-        // into this CTA's shared memory, then exit without storing
+    if (!ok) {
+        // gave up: every issued load lands before the CTA exits (the last
+        // armed phase of each stage); stores were issued only from landed stages
         raise_timeout(p);
-        ptx::mbar_drain(&bar, 0);
-        return;
+        for (int s = 0; s < kGatherStages && s < loaded; ++s) {
+            const int last = s + ((loaded - 1 - s) / kGatherStages) * kGatherStages;
+            ptx::mbar_drain(&full[s], last / kGatherStages);
+        }
     }
-    const int64_t dst_base = prob * (int64_t)p.kg * blk;
-    for (int s = s_lo; s < s_hi; ++s) {
-        if (gi[s - s_lo] < 0) continue;
-        char* sk = buf + (size_t)(s - s_lo) * 2 * blk;
-        ptx::bulk_s2g(k_dst + dst_base + (int64_t)s * blk, sk, blk);
-        ptx::bulk_s2g(v_dst + dst_base + (int64_t)s * blk, sk + blk, blk);
-    }
-    ptx::bulk_commit();
     ptx::bulk_wait_all();
 }
 
@@ -337,14 +385,26 @@ cudaError_t launch_gather(const Params& p, const void* k_src, const void* v_src,
                                                  sel_groups, n_sel_groups, (uint4*)k_dst,
                                                  (uint4*)v_dst);
     } else {
-        const size_t smem = (size_t)kSlotsPerCta * 2 * kGroupRows * p.d * es;
+        const size_t smem = (size_t)kGatherStages * 2 * kGroupRows * p.d * es;
         cudaError_t e = set_func_attr_once((const void*)gather_hbm_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kGatherStages * 2 * kGroupRows * 128 * 4);
         if (e != cudaSuccess) return e;
-        dim3 grid((p.kg + kSlotsPerCta - 1) / kSlotsPerCta, p.nQC, p.B * p.Hkv);
-        gather_hbm_kernel<<<grid, 32, smem, st>>>(p, (const char*)k_src, (const char*)v_src,
-                                                  sel_groups, n_sel_groups, (char*)k_dst,
-                                                  (char*)v_dst);
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return cudaErrorInvalidValue;
+        // one wave: four CTAs per SM fit (48 KB of stages each), each with
+        // 4 .. kGatherUnitsMax units
+        const int64_t total = (int64_t)p.B * p.Hkv * p.nQC * p.kg;
+        int64_t per = (total + 4 * sms - 1) / (4 * sms);
+        per = per < 4 ? 4 : (per > kGatherUnitsMax ? kGatherUnitsMax : per);
+        const int64_t grid = (total + per - 1) / per;
+        if (grid > INT32_MAX) return cudaErrorInvalidValue;
+        gather_hbm_kernel<<<(unsigned)grid, 32, smem, st>>>(p, (const char*)k_src,
+                                                           (const char*)v_src, sel_groups,
+                                                           n_sel_groups, (char*)k_dst,
+                                                           (char*)v_dst, (int)per);
     }
     return cudaGetLastError();
 }
