@@ -26,9 +26,10 @@
  *     Inputs are never modified. The library allocates no memory.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream). Work is only enqueued; nothing blocks the host except
- *     hga_get_device_error. The stream must belong to the current device
- *     (the library's per-device state is looked up for the current device);
- *     a stream of another device gives HGA_ERR_CUDA and launches nothing.
+ *     hga_get_device_error. The stream must belong to the current device:
+ *     the library's per-device state (error word, scratch array) is looked
+ *     up for the current device, and the stream is not queried (a query is
+ *     not allowed while the stream is being captured into a CUDA graph).
  *   - Arguments are validated on the host before anything is launched; a call
  *     that returns an error has launched nothing. Every data pointer must be
  *     16-byte aligned.
@@ -51,8 +52,8 @@
  *   - Layouts (row-major, innermost last):
  *       queries / outputs   [B, q_len, Hq, d]       (token q_begin + t at row t)
  *       keys / values       [B, Hkv, L, d]          (full store, HGA_KV_FULL)
- *       chunk summaries     [B, Hkv, nC, d] fp32    nC = ceil(L / C)
- *       group summaries     [B, Hkv, nC * G, d] fp32
+ *       chunk summaries     [B, Hkv, nC, d]         nC = ceil(L / C)
+ *       group summaries     [B, Hkv, nC * G, d]     (fp32 or bf16: summary_type)
  *       q-bar               [B, Hkv, nQC, d] fp32   query chunks of the span
  *       chunk selections    [B, Hkv, nQC, top_k_chunks] int32
  *       group selections    [B, Hkv, nQC, top_k_groups] int32 (global group
@@ -95,6 +96,18 @@ typedef enum { HGA_BF16 = 0, HGA_F32 = 1 } hga_dtype;
  *                 (the hot tier of "Geheugenarchitectuur"). Decode only. */
 typedef enum { HGA_KV_FULL = 0, HGA_KV_WINDOWS = 1 } hga_kv_layout;
 
+/* Storage type of the chunk and group summary tables (chunk_sum, group_sum).
+ * HGA_SUMMARY_F32:  fp32.
+ * HGA_SUMMARY_BF16: the fp32 summaries rounded to bf16 (nearest even); half
+ *                   the bytes the decode step reads for routing. Routing
+ *                   scores are still fp32 dot products (of the rounded
+ *                   values). Written by hga_build_summaries; read by
+ *                   hga_route and hga_decode_step on their one-launch decode
+ *                   path (one query token, bf16, d = 128, gq <= 8, L % 16 ==
+ *                   0, top_k_chunks <= 64); every other routing call returns
+ *                   HGA_ERR_UNSUPPORTED for it. */
+typedef enum { HGA_SUMMARY_F32 = 0, HGA_SUMMARY_BF16 = 1 } hga_summary_type;
+
 typedef struct {
     int32_t batch;             /* B */
     int32_t seq_len;           /* L: tokens in the K/V history (context length) */
@@ -113,6 +126,7 @@ typedef struct {
     int32_t q_begin;           /* first query position */
     int32_t q_len;             /* number of query tokens (1 = decode) */
     int32_t kv_layout;         /* hga_kv_layout, read by hga_attend only */
+    int32_t summary_type;      /* hga_summary_type of the summary tables (0 = fp32) */
 } hga_config;
 
 /* Rotate x by RoPE (standard rotary position embedding; the summaries of
@@ -133,9 +147,11 @@ hga_status hga_apply_rope(const hga_config* cfg, const void* x, void* x_rot, int
  * [B,Hkv,nC*G,d] (fp32) rows of those chunks and, if k_rot_out is not NULL,
  * the rotated keys R(p_t) k_t [B,Hkv,L,d] of their tokens in cfg->dtype (the
  * attention cache). Building chunk by chunk gives bitwise the same result as
- * building all chunks at once. */
-hga_status hga_build_summaries(const hga_config* cfg, const void* k_raw, float* chunk_sum,
-                               float* group_sum, void* k_rot_out, int32_t chunk_begin,
+ * building all chunks at once. The tables are fp32, or bf16 (each value the
+ * fp32 summary rounded to nearest even) when cfg->summary_type is
+ * HGA_SUMMARY_BF16. */
+hga_status hga_build_summaries(const hga_config* cfg, const void* k_raw, void* chunk_sum,
+                               void* group_sum, void* k_rot_out, int32_t chunk_begin,
                                int32_t chunk_end, void* stream);
 
 /* Level-1 routing ("Kernmechanisme" item 2, Niveau 1, and Deterministische
@@ -146,7 +162,7 @@ hga_status hga_build_summaries(const hga_config* cfg, const void* k_raw, float* 
  * and the top-min(top_k_chunks, #candidates) of them. Writes sel_chunks and
  * n_sel_chunks. scores_out (NULL or [B,Hkv,nQC,nC] fp32) receives every
  * candidate's score and NaN elsewhere. */
-hga_status hga_route_chunks(const hga_config* cfg, const void* q_rot, const float* chunk_sum,
+hga_status hga_route_chunks(const hga_config* cfg, const void* q_rot, const void* chunk_sum,
                             float* qbar_out, int32_t* sel_chunks, int32_t* n_sel_chunks,
                             float* scores_out, void* stream);
 
@@ -157,7 +173,7 @@ hga_status hga_route_chunks(const hga_config* cfg, const void* q_rot, const floa
  * n_sel_groups. scores_out (NULL or [B,Hkv,nQC,top_k_chunks*G] fp32) holds the
  * score of group gamma of the s-th chosen chunk at s*G + gamma, NaN where
  * unused. */
-hga_status hga_route_groups(const hga_config* cfg, const float* qbar, const float* group_sum,
+hga_status hga_route_groups(const hga_config* cfg, const float* qbar, const void* group_sum,
                             const int32_t* sel_chunks, const int32_t* n_sel_chunks,
                             int32_t* sel_groups, int32_t* n_sel_groups, float* scores_out,
                             void* stream);
@@ -170,8 +186,8 @@ hga_status hga_route_groups(const hga_config* cfg, const float* qbar, const floa
  * thread-block cluster); otherwise the two calls' kernels run in sequence.
  * qbar_out [B,Hkv,nQC,d] fp32, sel_chunks / n_sel_chunks, sel_groups /
  * n_sel_groups as for the two calls; all required. */
-hga_status hga_route(const hga_config* cfg, const void* q_rot, const float* chunk_sum,
-                     const float* group_sum, float* qbar_out, int32_t* sel_chunks,
+hga_status hga_route(const hga_config* cfg, const void* q_rot, const void* chunk_sum,
+                     const void* group_sum, float* qbar_out, int32_t* sel_chunks,
                      int32_t* n_sel_chunks, int32_t* sel_groups, int32_t* n_sel_groups,
                      void* stream);
 
@@ -184,8 +200,8 @@ hga_status hga_route(const hga_config* cfg, const void* q_rot, const float* chun
  * this is a single launch: the always-visible blocks are fetched while the
  * routing runs; the attention result equals hga_attend's within fp32
  * summation order. Other configurations run the separate kernels. */
-hga_status hga_decode_step(const hga_config* cfg, const void* q_rot, const float* chunk_sum,
-                           const float* group_sum, const void* k_cache, const void* v_cache,
+hga_status hga_decode_step(const hga_config* cfg, const void* q_rot, const void* chunk_sum,
+                           const void* group_sum, const void* k_cache, const void* v_cache,
                            float* qbar_out, int32_t* sel_chunks, int32_t* n_sel_chunks,
                            int32_t* sel_groups, int32_t* n_sel_groups, void* out, void* stream);
 

@@ -71,15 +71,6 @@ bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u
 // Limit of every bounded device wait of later launches (hga_set_wait_limit_ns).
 std::atomic<unsigned long long> g_wait_ns{1000000000ull};
 
-// The per-device state (error word, scratch array) is looked up for the
-// current device, so a call's stream must belong to it.
-hga_status check_stream_device(cudaStream_t st) {
-    if (st == nullptr) return HGA_OK;  // the legacy default stream of the current device
-    int cur = 0, sdev = 0;
-    if (cudaGetDevice(&cur) != cudaSuccess || cudaStreamGetDevice(st, &sdev) != cudaSuccess)
-        return HGA_ERR_CUDA;
-    return cur == sdev ? HGA_OK : HGA_ERR_CUDA;
-}
 
 // Checks shared by every call; fills p.
 hga_status make_params(const hga_config* c, Params* p) {
@@ -104,6 +95,8 @@ hga_status make_params(const hga_config* c, Params* p) {
     if (c->n_high_freq_pairs < 0 || c->n_high_freq_pairs > c->head_dim / 2) return HGA_ERR_CONFIG;
     if (!(c->rope_theta > 1.0) || !isfinite(c->rope_theta)) return HGA_ERR_CONFIG;
     if (c->kv_layout != HGA_KV_FULL && c->kv_layout != HGA_KV_WINDOWS) return HGA_ERR_CONFIG;
+    if (c->summary_type != HGA_SUMMARY_F32 && c->summary_type != HGA_SUMMARY_BF16)
+        return HGA_ERR_CONFIG;
     if (c->q_begin < 0 || c->q_len < 0 || (int64_t)c->q_begin + c->q_len > c->seq_len)
         return HGA_ERR_SHAPE;
     const int64_t nC = ((int64_t)c->seq_len + c->chunk_size - 1) / c->chunk_size;
@@ -130,6 +123,7 @@ hga_status make_params(const hga_config* c, Params* p) {
     p->nQC = c->q_len > 0 ? (c->q_begin + c->q_len - 1) / c->chunk_size - p->j0 + 1 : 0;
     p->dtype = c->dtype;
     p->kv_layout = c->kv_layout;
+    p->sum_bf16 = c->summary_type == HGA_SUMMARY_BF16 ? 1 : 0;
     for (int i = 0; i < kMaxHalfDim; ++i)
         p->inv_freq[i] = i < c->head_dim / 2
                              ? pow(c->rope_theta, -2.0 * (double)i / (double)c->head_dim)
@@ -141,13 +135,14 @@ hga_status make_params(const hga_config* c, Params* p) {
 
 hga_status launched(cudaError_t e) { return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA; }
 
-// Last step before any launch: check that the stream belongs to the current
-// device, then attach that device's error word.
-#define HGA_ATTACH_ERR(p, stream)                                              \
-    do {                                                                       \
-        hga_status es_ = check_stream_device((cudaStream_t)(stream));          \
-        if (es_ == HGA_OK) es_ = error_word(&(p).err);                         \
-        if (es_ != HGA_OK) return es_;                                         \
+// Last step before any launch: attach the current device's error word. (A
+// call's stream must belong to the current device; that is the caller's
+// rule, not checked here: a stream query is not allowed while the stream is
+// being captured into a CUDA graph.)
+#define HGA_ATTACH_ERR(p)                                  \
+    do {                                                   \
+        hga_status es_ = error_word(&(p).err);             \
+        if (es_ != HGA_OK) return es_;                     \
     } while (0)
 
 }  // namespace
@@ -179,12 +174,13 @@ cudaError_t set_func_attr_once(const void* fn, cudaFuncAttribute attr, int value
 
 using namespace hga;
 
-static_assert(sizeof(hga_config) == 72, "hga_config layout is part of the ABI");
+static_assert(sizeof(hga_config) == 80, "hga_config layout is part of the ABI");
+static_assert(offsetof(hga_config, summary_type) == 72, "hga_config layout is part of the ABI");
 static_assert(offsetof(hga_config, rope_theta) == 48, "hga_config layout is part of the ABI");
 
 extern "C" {
 
-int32_t hga_version(void) { return 10400; }
+int32_t hga_version(void) { return 10500; }
 
 void hga_set_wait_limit_ns(uint64_t limit_ns) {
     g_wait_ns.store(limit_ns == 0 ? 1000000000ull : (unsigned long long)limit_ns,
@@ -220,13 +216,13 @@ hga_status hga_apply_rope(const hga_config* cfg, const void* x, void* x_rot, int
     if (n_outer * n_tokens * n_heads == 0) return HGA_OK;
     if (x == nullptr || x_rot == nullptr) return HGA_ERR_NULL;
     if (!aligned16(x) || !aligned16(x_rot)) return HGA_ERR_ALIGN;
-    HGA_ATTACH_ERR(p, stream);
+    HGA_ATTACH_ERR(p);
     return launched(launch_rope(p, x, x_rot, n_outer, n_tokens, n_heads, pos0,
                                 (cudaStream_t)stream));
 }
 
-hga_status hga_build_summaries(const hga_config* cfg, const void* k_raw, float* chunk_sum,
-                               float* group_sum, void* k_rot_out, int32_t chunk_begin,
+hga_status hga_build_summaries(const hga_config* cfg, const void* k_raw, void* chunk_sum,
+                               void* group_sum, void* k_rot_out, int32_t chunk_begin,
                                int32_t chunk_end, void* stream) {
     Params p;
     hga_status s = make_params(cfg, &p);
@@ -237,12 +233,12 @@ hga_status hga_build_summaries(const hga_config* cfg, const void* k_raw, float* 
     if (!aligned16(k_raw) || !aligned16(chunk_sum) || !aligned16(group_sum) ||
         (k_rot_out && !aligned16(k_rot_out)))
         return HGA_ERR_ALIGN;
-    HGA_ATTACH_ERR(p, stream);
+    HGA_ATTACH_ERR(p);
     return launched(launch_summaries(p, k_raw, chunk_sum, group_sum, k_rot_out, chunk_begin,
                                      chunk_end, (cudaStream_t)stream));
 }
 
-hga_status hga_route_chunks(const hga_config* cfg, const void* q_rot, const float* chunk_sum,
+hga_status hga_route_chunks(const hga_config* cfg, const void* q_rot, const void* chunk_sum,
                             float* qbar_out, int32_t* sel_chunks, int32_t* n_sel_chunks,
                             float* scores_out, void* stream) {
     Params p;
@@ -253,17 +249,18 @@ hga_status hga_route_chunks(const hga_config* cfg, const void* q_rot, const floa
     if (!aligned16(q_rot) || !aligned16(chunk_sum) || !aligned16(qbar_out) ||
         !aligned16(sel_chunks) || !aligned16(n_sel_chunks) || (scores_out && !aligned16(scores_out)))
         return HGA_ERR_ALIGN;
-    HGA_ATTACH_ERR(p, stream);
+    if (p.sum_bf16) return HGA_ERR_UNSUPPORTED;  // bf16 tables: the one-launch decode path only
+    HGA_ATTACH_ERR(p);
     cudaStream_t st = (cudaStream_t)stream;
     if (!route_chunks_fuses_qbar(p)) {
         cudaError_t e = launch_qbar(p, q_rot, qbar_out, st);
         if (e != cudaSuccess) return HGA_ERR_CUDA;
     }
-    return launched(launch_route_chunks(p, q_rot, qbar_out, chunk_sum, sel_chunks, n_sel_chunks,
-                                        scores_out, st));
+    return launched(launch_route_chunks(p, q_rot, qbar_out, (const float*)chunk_sum, sel_chunks,
+                                        n_sel_chunks, scores_out, st));
 }
 
-hga_status hga_route_groups(const hga_config* cfg, const float* qbar, const float* group_sum,
+hga_status hga_route_groups(const hga_config* cfg, const float* qbar, const void* group_sum,
                             const int32_t* sel_chunks, const int32_t* n_sel_chunks,
                             int32_t* sel_groups, int32_t* n_sel_groups, float* scores_out,
                             void* stream) {
@@ -277,14 +274,16 @@ hga_status hga_route_groups(const hga_config* cfg, const float* qbar, const floa
         !aligned16(n_sel_chunks) || !aligned16(sel_groups) || !aligned16(n_sel_groups) ||
         (scores_out && !aligned16(scores_out)))
         return HGA_ERR_ALIGN;
-    HGA_ATTACH_ERR(p, stream);
-    return launched(launch_route_groups(p, qbar, group_sum, sel_chunks, n_sel_chunks, sel_groups,
-                                        n_sel_groups, scores_out, (cudaStream_t)stream));
+    if (p.sum_bf16) return HGA_ERR_UNSUPPORTED;  // bf16 tables: the one-launch decode path only
+    HGA_ATTACH_ERR(p);
+    return launched(launch_route_groups(p, qbar, (const float*)group_sum, sel_chunks, n_sel_chunks,
+                                        sel_groups, n_sel_groups, scores_out,
+                                        (cudaStream_t)stream));
 }
 
 // Shared checks of hga_route / hga_decode_step (routing outputs).
-static hga_status check_route_args(const Params& p, const void* q_rot, const float* chunk_sum,
-                                   const float* group_sum, const float* qbar_out,
+static hga_status check_route_args(const Params& p, const void* q_rot, const void* chunk_sum,
+                                   const void* group_sum, const float* qbar_out,
                                    const int32_t* sel_chunks, const int32_t* n_sel_chunks,
                                    const int32_t* sel_groups, const int32_t* n_sel_groups) {
     (void)p;
@@ -299,21 +298,22 @@ static hga_status check_route_args(const Params& p, const void* q_rot, const flo
 }
 
 // The two routing levels as separate kernels.
-static hga_status route_separate(const Params& p, const void* q_rot, const float* chunk_sum,
-                                 const float* group_sum, float* qbar_out, int32_t* sel_chunks,
+static hga_status route_separate(const Params& p, const void* q_rot, const void* chunk_sum,
+                                 const void* group_sum, float* qbar_out, int32_t* sel_chunks,
                                  int32_t* n_sel_chunks, int32_t* sel_groups,
                                  int32_t* n_sel_groups, cudaStream_t st) {
+    if (p.sum_bf16) return HGA_ERR_UNSUPPORTED;  // bf16 tables: the one-launch decode path only
     if (!route_chunks_fuses_qbar(p) && launch_qbar(p, q_rot, qbar_out, st) != cudaSuccess)
         return HGA_ERR_CUDA;
-    if (launch_route_chunks(p, q_rot, qbar_out, chunk_sum, sel_chunks, n_sel_chunks, nullptr,
-                            st) != cudaSuccess)
+    if (launch_route_chunks(p, q_rot, qbar_out, (const float*)chunk_sum, sel_chunks, n_sel_chunks,
+                            nullptr, st) != cudaSuccess)
         return HGA_ERR_CUDA;
-    return launched(launch_route_groups(p, qbar_out, group_sum, sel_chunks, n_sel_chunks,
-                                        sel_groups, n_sel_groups, nullptr, st));
+    return launched(launch_route_groups(p, qbar_out, (const float*)group_sum, sel_chunks,
+                                        n_sel_chunks, sel_groups, n_sel_groups, nullptr, st));
 }
 
-hga_status hga_route(const hga_config* cfg, const void* q_rot, const float* chunk_sum,
-                     const float* group_sum, float* qbar_out, int32_t* sel_chunks,
+hga_status hga_route(const hga_config* cfg, const void* q_rot, const void* chunk_sum,
+                     const void* group_sum, float* qbar_out, int32_t* sel_chunks,
                      int32_t* n_sel_chunks, int32_t* sel_groups, int32_t* n_sel_groups,
                      void* stream) {
     Params p;
@@ -323,7 +323,7 @@ hga_status hga_route(const hga_config* cfg, const void* q_rot, const float* chun
     s = check_route_args(p, q_rot, chunk_sum, group_sum, qbar_out, sel_chunks, n_sel_chunks,
                          sel_groups, n_sel_groups);
     if (s != HGA_OK) return s;
-    HGA_ATTACH_ERR(p, stream);
+    HGA_ATTACH_ERR(p);
     cudaStream_t st = (cudaStream_t)stream;
     if (decode_step_supports(p))
         return launched(launch_decode_step(p, q_rot, chunk_sum, group_sum, nullptr, nullptr,
@@ -333,8 +333,8 @@ hga_status hga_route(const hga_config* cfg, const void* q_rot, const float* chun
                           sel_groups, n_sel_groups, st);
 }
 
-hga_status hga_decode_step(const hga_config* cfg, const void* q_rot, const float* chunk_sum,
-                           const float* group_sum, const void* k_cache, const void* v_cache,
+hga_status hga_decode_step(const hga_config* cfg, const void* q_rot, const void* chunk_sum,
+                           const void* group_sum, const void* k_cache, const void* v_cache,
                            float* qbar_out, int32_t* sel_chunks, int32_t* n_sel_chunks,
                            int32_t* sel_groups, int32_t* n_sel_groups, void* out, void* stream) {
     Params p;
@@ -347,7 +347,7 @@ hga_status hga_decode_step(const hga_config* cfg, const void* q_rot, const float
     if (!k_cache || !v_cache || !out) return HGA_ERR_NULL;
     if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return HGA_ERR_ALIGN;
     if (p.kv_layout != HGA_KV_FULL) return HGA_ERR_UNSUPPORTED;
-    HGA_ATTACH_ERR(p, stream);
+    HGA_ATTACH_ERR(p);
     cudaStream_t st = (cudaStream_t)stream;
     if (decode_step_supports(p))
         return launched(launch_decode_step(p, q_rot, chunk_sum, group_sum, k_cache, v_cache,
@@ -391,7 +391,7 @@ hga_status hga_gather_kv(const hga_config* cfg, const void* k_src, const void* v
     if (!aligned16(k_src) || !aligned16(v_src) || !aligned16(sel_groups) ||
         !aligned16(n_sel_groups) || !aligned16(k_dst) || !aligned16(v_dst))
         return HGA_ERR_ALIGN;
-    HGA_ATTACH_ERR(p, stream);
+    HGA_ATTACH_ERR(p);
     const void* kd = nullptr;
     const void* vd = nullptr;
     if ((s = device_view(k_src, src_is_host != 0, &kd)) != HGA_OK) return s;
@@ -420,7 +420,7 @@ hga_status hga_gather_kv_warm(const hga_config* cfg, const void* k_host, const v
     if (p.q_len != 1) return HGA_ERR_UNSUPPORTED;
     if (n_slots < p.kg || step < 0) return HGA_ERR_SHAPE;
     if (!gather_warm_supports(p, n_slots)) return HGA_ERR_UNSUPPORTED;
-    HGA_ATTACH_ERR(p, stream);
+    HGA_ATTACH_ERR(p);
     const void* kd = nullptr;
     const void* vd = nullptr;
     if ((s = device_view(k_host, true, &kd)) != HGA_OK) return s;
@@ -452,7 +452,7 @@ hga_status hga_gather_kv_warm_noalloc(const hga_config* cfg, const void* k_host,
     if (n_slots < p.kg || step < 0) return HGA_ERR_SHAPE;
     if (!gather_warm_supports(p, n_slots)) return HGA_ERR_UNSUPPORTED;
     if ((int64_t)p.B * p.Hkv * p.kg > kWarmScratchEntries) return HGA_ERR_SCRATCH_LIMIT;
-    HGA_ATTACH_ERR(p, stream);
+    HGA_ATTACH_ERR(p);
     int32_t* src = nullptr;
     if ((s = warm_scratch(&src)) != HGA_OK) return s;
     const void* kd = nullptr;
@@ -481,7 +481,7 @@ hga_status hga_attend(const hga_config* cfg, const void* q_rot, const void* k_re
     if (p.kv_layout == HGA_KV_WINDOWS &&
         (p.q_len != 1 || p.q_begin != p.L - 1 || k_gat == nullptr))
         return HGA_ERR_UNSUPPORTED;
-    HGA_ATTACH_ERR(p, stream);
+    HGA_ATTACH_ERR(p);
     KvSources kv{k_res, v_res, k_gat, v_gat};
     cudaStream_t st = (cudaStream_t)stream;
     if (tc_kernel_supports(p, k_gat != nullptr))
@@ -493,7 +493,6 @@ hga_status hga_attend(const hga_config* cfg, const void* q_rot, const void* k_re
 
 hga_status hga_get_device_error(void* stream, int32_t* detail_out) {
     if (detail_out) *detail_out = 0;
-    if (check_stream_device((cudaStream_t)stream) != HGA_OK) return HGA_ERR_CUDA;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return HGA_ERR_CUDA;
     int* addr = nullptr;
     hga_status s = error_word(&addr);

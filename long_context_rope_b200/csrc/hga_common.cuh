@@ -23,6 +23,7 @@ struct Params {
     int n_sink, n_local, kc, kg, F;
     int nC, q_begin, q_len, j0, nQC;
     int dtype, kv_layout;
+    int sum_bf16;                  // summary tables stored as bf16 (else fp32)
     int* err;                      // device error word, never NULL
     unsigned long long wait_ns;    // limit of each bounded device wait
     double inv_freq[kMaxHalfDim];  // rope_theta^(-2i/d), computed on the host in double

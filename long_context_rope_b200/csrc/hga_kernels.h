@@ -27,8 +27,9 @@ cudaError_t current_device_index(int* dev);
 cudaError_t launch_rope(const Params& p, const void* x, void* y, int64_t n_outer,
                         int64_t n_tokens, int n_heads, int64_t pos0, cudaStream_t st);
 
-cudaError_t launch_summaries(const Params& p, const void* k_raw, float* chunk_sum,
-                             float* group_sum, void* k_rot, int chunk_begin, int chunk_end,
+// chunk_sum / group_sum: fp32, or bf16 when p.sum_bf16.
+cudaError_t launch_summaries(const Params& p, const void* k_raw, void* chunk_sum,
+                             void* group_sum, void* k_rot, int chunk_begin, int chunk_end,
                              cudaStream_t st);
 
 cudaError_t launch_qbar(const Params& p, const void* q_rot, float* qbar, cudaStream_t st);
@@ -101,8 +102,9 @@ cudaError_t launch_attend_decode(const Params& p, const void* q_rot, const KvSou
 // top_k_chunks <= 64, top_k_groups <= 512, and routing tables that fit one
 // cluster's shared memory. With out == nullptr it stops after routing.
 bool decode_step_supports(const Params& p);
-cudaError_t launch_decode_step(const Params& p, const void* q_rot, const float* chunk_sum,
-                               const float* group_sum, const void* k_cache, const void* v_cache,
+// Summary tables fp32, or bf16 when p.sum_bf16.
+cudaError_t launch_decode_step(const Params& p, const void* q_rot, const void* chunk_sum,
+                               const void* group_sum, const void* k_cache, const void* v_cache,
                                float* qbar, int32_t* sel_chunks, int32_t* n_sel_chunks,
                                int32_t* sel_groups, int32_t* n_sel_groups, void* out,
                                cudaStream_t st);

@@ -15,10 +15,12 @@
 // exchange and no serial selection pass:
 //   level 1  CTA r scores a contiguous slice of the candidate chunks and
 //            ranks them locally (count of larger keys); its local top k_c
-//            (the only ones that can be in the global top k_c) go to every
-//            CTA's finalist table through distributed shared memory;
-//            cluster barrier; every CTA ranks the whole table (rank < k_c
-//            wins) and sorts the winners by chunk index.
+//            (the only ones that can be in the global top k_c) go, in
+//            ascending chunk order, to every CTA's finalist table through
+//            distributed shared memory; cluster barrier; every CTA ranks the
+//            whole table (rank < k_c wins). Slices are contiguous, so the
+//            table is in ascending chunk order and compacting the winners in
+//            table order gives the sorted list without a sort.
 //   level 2  every CTA scores all G groups of the selected chunks (at most
 //            G x k_c rows, shared through L2) and ranks them exactly; the
 //            candidates are already in ascending group order, so one warp
@@ -76,7 +78,6 @@ struct StepSmem {
     uint64_t key2[kMaxCand2];     // level-2 candidates (all of them, every CTA)
     int rank[kMaxSlice > kMaxCand2 ? kMaxSlice : kMaxCand2];  // rank scratch
     int win1[kMaxKc];             // selected chunks, ascending
-    int wl[kMaxKc];               // selected chunks, unordered, as -(index + 1)
     int routed[kMaxKg];           // selected groups, ascending
     int blk_pos[kMaxLocal];
     int n_win1, n_wl, bad;
@@ -127,17 +128,16 @@ __device__ __forceinline__ void count_greater(const T* a, int na, const T* b, in
     }
 }
 
-// Number of forced chunks (sinks, locals) below the current chunk j that
-// fall in [lo, hi).
-__device__ __forceinline__ int forced_below_in(const Params& p, int j, int lo, int hi) {
-    const int s_hi = p.n_sink < j ? p.n_sink : j;
-    const int s_end = p.n_sink < j + 1 ? p.n_sink : j + 1;
-    const int l_lo = j - p.n_local > s_end ? j - p.n_local : s_end;
-    auto overlap = [&](int a, int b) {
-        const int x0 = a > lo ? a : lo, x1 = b < hi ? b : hi;
-        return x1 > x0 ? x1 - x0 : 0;
-    };
-    return overlap(0, s_hi) + (l_lo < j ? overlap(l_lo, j) : 0);
+// Elements 4 * lane .. 4 * lane + 3 of a summary row as fp32 (fp32 or bf16
+// tables; a bf16 value converts to fp32 exactly).
+__device__ __forceinline__ float4 load4(const float* row, int lane) {
+    return __ldg(reinterpret_cast<const float4*>(row) + lane);
+}
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* row, int lane) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(row) + lane);
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
 }
 
 // Score rows [0, n) of a summary table for this warp's share and hand each
@@ -150,7 +150,7 @@ __device__ __forceinline__ void score_rows(const float* q, int n, RowOf row_of, 
 #pragma unroll
         for (int u = 0; u < kRowsInFlight; ++u) {
             const int x = x0 + u < n ? x0 + u : n - 1;
-            const float4 t = __ldg(reinterpret_cast<const float4*>(row_of(x)) + lane);
+            const float4 t = load4(row_of(x), lane);
             v[u][0] = t.x; v[u][1] = t.y; v[u][2] = t.z; v[u][3] = t.w;
         }
         float sc[kRowsInFlight];
@@ -171,9 +171,11 @@ __device__ __forceinline__ void score_rows(const float* q, int n, RowOf row_of, 
     }
 }
 
+// S: element type of the summary tables (float, or bf16 for bf16 tables).
+template <typename S>
 __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     const __grid_constant__ StepMaps maps, Params p, const __nv_bfloat16* __restrict__ q,
-    const float* __restrict__ cs, const float* __restrict__ gs, float* __restrict__ qbar_out,
+    const S* __restrict__ cs, const S* __restrict__ gs, float* __restrict__ qbar_out,
     int32_t* __restrict__ sel_c, int32_t* __restrict__ nsel_c, int32_t* __restrict__ sel_g,
     int32_t* __restrict__ nsel_g, __nv_bfloat16* __restrict__ out, int attend) {
     extern __shared__ uint8_t smem_raw[];
@@ -226,13 +228,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     const int c_lo = r * per1;
     const int c_hi = c_lo + per1 < j ? c_lo + per1 : j;
     const int ns = c_hi > c_lo ? c_hi - c_lo : 0;
-    const float* ctab = cs + bh * (int64_t)p.nC * kD;
+    const S* ctab = cs + bh * (int64_t)p.nC * kD;
     float4 first[kL1Rows];
     if (consumer) {
 #pragma unroll
         for (int u = 0; u < kL1Rows; ++u) {
             const int x = warp * kL1Rows + u;
-            first[u] = x < ns ? __ldg(reinterpret_cast<const float4*>(ctab + (int64_t)(c_lo + x) * kD) + lane)
+            first[u] = x < ns ? load4(ctab + (int64_t)(c_lo + x) * kD, lane)
                               : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
@@ -301,36 +303,46 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     __syncthreads();
     if (consumer) count_greater(sm.key1, ns, sm.key1, ns, sm.rank);
     __syncthreads();
-    {
-        const int present = ns - forced_below_in(p, j, c_lo, c_hi);
-        const int filled = present < cap1 ? present : cap1;
-        for (int x = tid; x < ns; x += blockDim.x) {
-            const uint64_t k = sm.key1[x];
-            if (k != 0ull && sm.rank[x] < cap1)
-                for (int t = 0; t < CL; ++t)
-                    cluster.map_shared_rank(sm.f1, t)[r * cap1 + sm.rank[x]] = k;
+    // this CTA's winners go to slots [r * cap1, (r + 1) * cap1) of every
+    // CTA's finalist table in candidate (= ascending chunk) order, so the
+    // table is ascending: slices are contiguous and ordered by r
+    if (warp == 0) {
+        int base = 0;
+        for (int x0 = 0; x0 < ns; x0 += 32) {
+            const int x = x0 + lane;
+            const uint64_t k = x < ns ? sm.key1[x] : 0ull;
+            const bool win = k != 0ull && sm.rank[x] < cap1;
+            const unsigned m = __ballot_sync(0xffffffffu, win);
+            if (win) {
+                const int at = r * cap1 + base + __popc(m & ((1u << lane) - 1u));
+                for (int t = 0; t < CL; ++t) cluster.map_shared_rank(sm.f1, t)[at] = k;
+            }
+            base += __popc(m);
         }
-        for (int x = filled + tid; x < cap1; x += blockDim.x)
+        for (int x = base + lane; x < cap1; x += 32)
             for (int t = 0; t < CL; ++t) cluster.map_shared_rank(sm.f1, t)[r * cap1 + x] = 0ull;
     }
     cluster.sync();
 
-    // ---- every CTA ranks the whole finalist table: the global top k_c
+    // ---- every CTA ranks the whole finalist table: the global top k_c,
+    // compacted in table order, which is ascending chunk order
     const int nF1 = CL * cap1;
     if (consumer) count_greater(sm.f1, nF1, sm.f1, nF1, sm.rank);
     __syncthreads();
-    for (int x = tid; x < nF1; x += blockDim.x) {
-        const uint64_t k = sm.f1[x];
-        if (k != 0ull && sm.rank[x] < p.kc) sm.wl[atomicAdd(&sm.n_win1, 1)] = -index_of(k) - 1;
+    if (warp == 0) {
+        int base = 0;
+        for (int x0 = 0; x0 < nF1; x0 += 32) {
+            const int x = x0 + lane;
+            const uint64_t k = x < nF1 ? sm.f1[x] : 0ull;
+            const bool win = k != 0ull && sm.rank[x] < p.kc;
+            const unsigned m = __ballot_sync(0xffffffffu, win);
+            if (win) sm.win1[base + __popc(m & ((1u << lane) - 1u))] = index_of(k);
+            base += __popc(m);
+        }
+        if (lane == 0) sm.n_win1 = base;
     }
     __syncthreads();
-    // chunk winners in ascending order: wl holds -(index + 1), so the count of
-    // larger entries is the count of smaller indices
     const int nsel1 = sm.n_win1;  // min(k_c, number of candidates)
-    if (consumer) count_greater(sm.wl, nsel1, sm.wl, nsel1, sm.rank);
-    __syncthreads();
-    for (int i = tid; i < nsel1; i += blockDim.x) sm.win1[sm.rank[i]] = -sm.wl[i] - 1;
-    __syncthreads();
     if (r == 0) {
         for (int i = tid; i < p.kc; i += blockDim.x) sel_c[prob * p.kc + i] = i < nsel1 ? sm.win1[i] : -1;
         if (tid == 0) nsel_c[prob] = nsel1;
@@ -340,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     // (candidate x = group x % G of the (x / G)-th chunk: ascending group
     // index) and ranks them exactly; no second cluster exchange is needed
     const int n2 = nsel1 * p.G;
-    const float* gtab = gs + bh * (int64_t)p.nC * p.G * kD;
+    const S* gtab = gs + bh * (int64_t)p.nC * p.G * kD;
     if (consumer)
         score_rows<16>(qv, n2,
                        [&](int x) { return gtab + ((int64_t)sm.win1[x / p.G] * p.G + x % p.G) * kD; },
@@ -430,24 +442,27 @@ bool step_fits(const Params& p, int cl) {
 }
 
 std::mutex g_step_mu;
-int g_max_active[kMaxDevicesPerProcess][kMaxCluster + 1] = {};  // per device, 0 = not queried
+// per device and summary type, 0 = not queried
+int g_max_active[kMaxDevicesPerProcess][2][kMaxCluster + 1] = {};
 
+template <typename S>
 cudaError_t step_prepare(size_t smem) {
-    cudaError_t e = set_func_attr_once((const void*)decode_step_kernel,
+    cudaError_t e = set_func_attr_once((const void*)decode_step_kernel<S>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = set_func_attr_once((const void*)decode_step_kernel,
+        e = set_func_attr_once((const void*)decode_step_kernel<S>,
                                cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return e;
 }
 
 // Clusters of `cl` CTAs that can be resident at once on the current device
 // (-1 if the query fails).
+template <typename S>
 int active_clusters(int cl, size_t smem) {
     int dev = 0;
     if (current_device_index(&dev) != cudaSuccess) return -1;
     std::lock_guard<std::mutex> lock(g_step_mu);
-    int& slot = g_max_active[dev][cl];
+    int& slot = g_max_active[dev][sizeof(S) == 2 ? 1 : 0][cl];
     if (slot == 0) {
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(cl, 1, 1);
@@ -461,7 +476,7 @@ int active_clusters(int cl, size_t smem) {
         q.attrs = a;
         q.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, decode_step_kernel, &q) != cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&n, decode_step_kernel<S>, &q) != cudaSuccess) {
             cudaGetLastError();
             n = -1;
         }
@@ -472,6 +487,7 @@ int active_clusters(int cl, size_t smem) {
 
 // Cluster size: two CTAs per SM over the whole grid if the tables fit and the
 // clusters can all be resident at once; else the largest size that fits.
+template <typename S>
 int step_cluster(const Params& p, size_t smem) {
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess)
@@ -482,7 +498,7 @@ int step_cluster(const Params& p, size_t smem) {
     for (; cl >= 1; --cl) {
         if (!step_fits(p, cl)) continue;
         if (cl == 1) return 1;
-        const int n = active_clusters(cl, smem);
+        const int n = active_clusters<S>(cl, smem);
         if (n >= units || (n > 0 && cl <= 2)) return cl;
     }
     return 0;
@@ -499,11 +515,13 @@ bool decode_step_supports(const Params& p) {
     return false;
 }
 
-cudaError_t launch_decode_step(const Params& p, const void* q_rot, const float* chunk_sum,
-                               const float* group_sum, const void* k_cache, const void* v_cache,
-                               float* qbar, int32_t* sel_chunks, int32_t* n_sel_chunks,
-                               int32_t* sel_groups, int32_t* n_sel_groups, void* out,
-                               cudaStream_t st) {
+namespace {
+
+template <typename S>
+cudaError_t launch_step(const Params& p, const void* q_rot, const S* chunk_sum,
+                        const S* group_sum, const void* k_cache, const void* v_cache, float* qbar,
+                        int32_t* sel_chunks, int32_t* n_sel_chunks, int32_t* sel_groups,
+                        int32_t* n_sel_groups, void* out, cudaStream_t st) {
     const bool attend = out != nullptr;
     StepMaps maps;
     if (attend) {
@@ -515,9 +533,9 @@ cudaError_t launch_decode_step(const Params& p, const void* q_rot, const float* 
         memset(&maps, 0, sizeof(maps));
     }
     const size_t smem = sizeof(StepSmem) + 1024;
-    cudaError_t e = step_prepare(smem);
+    cudaError_t e = step_prepare<S>(smem);
     if (e != cudaSuccess) return e;
-    const int cl = step_cluster(p, smem);
+    const int cl = step_cluster<S>(p, smem);
     if (cl < 1) return cudaErrorInvalidConfiguration;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cl, (unsigned)(p.B * p.Hkv), 1);
@@ -531,9 +549,24 @@ cudaError_t launch_decode_step(const Params& p, const void* q_rot, const float* 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_step_kernel, maps, p, (const __nv_bfloat16*)q_rot,
+    return cudaLaunchKernelEx(&cfg, decode_step_kernel<S>, maps, p, (const __nv_bfloat16*)q_rot,
                               chunk_sum, group_sum, qbar, sel_chunks, n_sel_chunks, sel_groups,
                               n_sel_groups, (__nv_bfloat16*)out, attend ? 1 : 0);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_step(const Params& p, const void* q_rot, const void* chunk_sum,
+                               const void* group_sum, const void* k_cache, const void* v_cache,
+                               float* qbar, int32_t* sel_chunks, int32_t* n_sel_chunks,
+                               int32_t* sel_groups, int32_t* n_sel_groups, void* out,
+                               cudaStream_t st) {
+    if (p.sum_bf16)
+        return launch_step(p, q_rot, (const __nv_bfloat16*)chunk_sum,
+                           (const __nv_bfloat16*)group_sum, k_cache, v_cache, qbar, sel_chunks,
+                           n_sel_chunks, sel_groups, n_sel_groups, out, st);
+    return launch_step(p, q_rot, (const float*)chunk_sum, (const float*)group_sum, k_cache,
+                       v_cache, qbar, sel_chunks, n_sel_chunks, sel_groups, n_sel_groups, out, st);
 }
 
 }  // namespace hga

@@ -84,9 +84,24 @@ __global__ void __launch_bounds__(256) rope_kernel(Params p, const T* __restrict
 }
 
 // ------------------------------------------------------------- summaries
-template <typename T>
-__global__ void summaries_kernel(Params p, const T* __restrict__ k_raw, float* __restrict__ cs,
-                                 float* __restrict__ gs, T* __restrict__ k_rot, int chunk_begin) {
+// n consecutive summary values (n = 4 or 8) written as fp32, or rounded to
+// bf16 (nearest even) for bf16 summary tables.
+__device__ __forceinline__ void store_sum(float* out, const float* v, int n) {
+    for (int i = 0; i < n; i += 4)
+        *reinterpret_cast<float4*>(out + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+}
+__device__ __forceinline__ void store_sum(__nv_bfloat16* out, const float* v, int n) {
+    if (n == 8) {
+        *reinterpret_cast<uint4*>(out) = f32x8_to_bf16(v);
+    } else {
+        __nv_bfloat162 h[2] = {__floats2bfloat162_rn(v[0], v[1]), __floats2bfloat162_rn(v[2], v[3])};
+        *reinterpret_cast<uint2*>(out) = *reinterpret_cast<const uint2*>(h);
+    }
+}
+
+template <typename T, typename S>
+__global__ void summaries_kernel(Params p, const T* __restrict__ k_raw, S* __restrict__ cs,
+                                 S* __restrict__ gs, T* __restrict__ k_rot, int chunk_begin) {
     constexpr int V = Vec<T>::N;
     const int half = p.d / 2;
     const int G = p.G;
@@ -153,7 +168,7 @@ __global__ void summaries_kernel(Params p, const T* __restrict__ k_raw, float* _
             acc1[e] += __shfl_xor_sync(0xffffffffu, acc1[e], off);
         }
     }
-    auto finish = [&](const float* s0, const float* s1, int64_t first, int n, float* out) {
+    auto finish = [&](const float* s0, const float* s1, int64_t first, int n, S* out) {
         float o0[V], o1[V];
         if (n <= 0) {
 #pragma unroll
@@ -176,18 +191,14 @@ __global__ void summaries_kernel(Params p, const T* __restrict__ k_raw, float* _
                 }
             }
         }
-        Vec<float>::store(out + u * V, o0);
-        Vec<float>::store(out + half + u * V, o1);
-        if (V == 8) {
-            Vec<float>::store(out + u * V + 4, o0 + 4);
-            Vec<float>::store(out + half + u * V + 4, o1 + 4);
-        }
+        store_sum(out + u * V, o0, V);
+        store_sum(out + half + u * V, o1, V);
     };
     if (s == 0) {
         int64_t g0 = c0 + 16 * k;
         int64_t left = (int64_t)p.L - g0;
         int n = left <= 0 ? 0 : (left >= 16 ? 16 : (int)left);
-        float* out = gs + ((bh * p.nC + ch) * G + k) * (int64_t)p.d;
+        S* out = gs + ((bh * p.nC + ch) * G + k) * (int64_t)p.d;
         finish(acc0, acc1, g0, n, out);
     }
     // chunk sums: reduce the group sums over k (lanes 4, 8, ...)
@@ -201,7 +212,7 @@ __global__ void summaries_kernel(Params p, const T* __restrict__ k_raw, float* _
     if (s == 0 && k == 0) {
         int64_t left = (int64_t)p.L - c0;
         int n = left <= 0 ? 0 : (left >= p.C ? p.C : (int)left);
-        float* out = cs + (bh * p.nC + ch) * (int64_t)p.d;
+        S* out = cs + (bh * p.nC + ch) * (int64_t)p.d;
         finish(acc0, acc1, c0, n, out);
     }
 }
@@ -223,21 +234,31 @@ cudaError_t launch_rope(const Params& p, const void* x, void* y, int64_t n_outer
     return cudaGetLastError();
 }
 
-cudaError_t launch_summaries(const Params& p, const void* k_raw, float* chunk_sum,
-                             float* group_sum, void* k_rot, int chunk_begin, int chunk_end,
+cudaError_t launch_summaries(const Params& p, const void* k_raw, void* chunk_sum,
+                             void* group_sum, void* k_rot, int chunk_begin, int chunk_end,
                              cudaStream_t st) {
     int n = chunk_end - chunk_begin;
     if (n <= 0) return cudaSuccess;
     const int V = p.dtype == HGA_BF16 ? 8 : 4;
     int threads = (p.d / 2 / V) * 4 * p.G;
     dim3 grid(n, p.B * p.Hkv);
-    if (p.dtype == HGA_BF16)
-        summaries_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
-            p, (const __nv_bfloat16*)k_raw, chunk_sum, group_sum, (__nv_bfloat16*)k_rot,
-            chunk_begin);
-    else
-        summaries_kernel<float><<<grid, threads, 0, st>>>(p, (const float*)k_raw, chunk_sum,
-                                                          group_sum, (float*)k_rot, chunk_begin);
+    using bf = __nv_bfloat16;
+    if (p.dtype == HGA_BF16) {
+        if (p.sum_bf16)
+            summaries_kernel<bf, bf><<<grid, threads, 0, st>>>(
+                p, (const bf*)k_raw, (bf*)chunk_sum, (bf*)group_sum, (bf*)k_rot, chunk_begin);
+        else
+            summaries_kernel<bf, float><<<grid, threads, 0, st>>>(
+                p, (const bf*)k_raw, (float*)chunk_sum, (float*)group_sum, (bf*)k_rot, chunk_begin);
+    } else {
+        if (p.sum_bf16)
+            summaries_kernel<float, bf><<<grid, threads, 0, st>>>(
+                p, (const float*)k_raw, (bf*)chunk_sum, (bf*)group_sum, (float*)k_rot, chunk_begin);
+        else
+            summaries_kernel<float, float><<<grid, threads, 0, st>>>(
+                p, (const float*)k_raw, (float*)chunk_sum, (float*)group_sum, (float*)k_rot,
+                chunk_begin);
+    }
     return cudaGetLastError();
 }
 

@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_PKG, "libhga.so")
 HGA_OK = 0
 HGA_BF16, HGA_F32 = 0, 1
 HGA_KV_FULL, HGA_KV_WINDOWS = 0, 1
+HGA_SUMMARY_F32, HGA_SUMMARY_BF16 = 0, 1
 STATUS = {0: "HGA_OK", -1: "HGA_ERR_NULL", -2: "HGA_ERR_SHAPE", -3: "HGA_ERR_ALIGN",
           -4: "HGA_ERR_CONFIG", -5: "HGA_ERR_CUDA", -6: "HGA_ERR_DEVICE_INDEX",
           -7: "HGA_ERR_TIMEOUT", -8: "HGA_ERR_UNSUPPORTED", -9: "HGA_ERR_MEMORY",
@@ -40,7 +41,7 @@ class HgaConfig(ctypes.Structure):
         "batch", "seq_len", "n_q_heads", "n_kv_heads", "head_dim", "chunk_size",
         "groups_per_chunk", "n_sink", "n_local", "top_k_chunks", "top_k_groups",
         "n_high_freq_pairs")] + [("rope_theta", ctypes.c_double)] + [
-        (n, ctypes.c_int32) for n in ("dtype", "q_begin", "q_len", "kv_layout")]
+        (n, ctypes.c_int32) for n in ("dtype", "q_begin", "q_len", "kv_layout", "summary_type")]
 
     @property
     def n_chunks(self) -> int:
@@ -58,6 +59,9 @@ class HgaConfig(ctypes.Structure):
 
     def torch_dtype(self) -> torch.dtype:
         return torch.bfloat16 if self.dtype == HGA_BF16 else torch.float32
+
+    def summary_torch_dtype(self) -> torch.dtype:
+        return torch.bfloat16 if self.summary_type == HGA_SUMMARY_BF16 else torch.float32
 
     def copy(self, **kw) -> "HgaConfig":
         c = HgaConfig()
@@ -119,6 +123,7 @@ def config_from(w, **overrides) -> HgaConfig:
     c.q_begin = int(w.q_begin)
     c.q_len = int(w.q_len)
     c.kv_layout = HGA_KV_FULL
+    c.summary_type = HGA_SUMMARY_F32
     for k, v in overrides.items():
         setattr(c, k, v)
     return c
@@ -173,8 +178,8 @@ def build_summaries(cfg: HgaConfig, k_raw, chunk_sum, group_sum, k_rot=None, chu
     dt = cfg.torch_dtype()
     _check(_lib.hga_build_summaries(
         ctypes.byref(cfg), _ptr(k_raw, "k_raw", dt, (B, H, L, d)),
-        _ptr(chunk_sum, "chunk_sum", torch.float32, (B, H, nC, d)),
-        _ptr(group_sum, "group_sum", torch.float32, (B, H, nC * G, d)),
+        _ptr(chunk_sum, "chunk_sum", cfg.summary_torch_dtype(), (B, H, nC, d)),
+        _ptr(group_sum, "group_sum", cfg.summary_torch_dtype(), (B, H, nC * G, d)),
         _ptr(k_rot, "k_rot", dt, (B, H, L, d), nullable=True), int(chunk_begin),
         int(nC if chunk_end is None else chunk_end), _stream(stream)), "hga_build_summaries")
 
@@ -185,7 +190,7 @@ def route_chunks(cfg: HgaConfig, q_rot, chunk_sum, qbar, sel_chunks, n_sel_chunk
     _check(_lib.hga_route_chunks(
         ctypes.byref(cfg), _ptr(q_rot, "q_rot", cfg.torch_dtype(),
                                 (B, cfg.q_len, cfg.n_q_heads, d)),
-        _ptr(chunk_sum, "chunk_sum", torch.float32, (B, H, cfg.n_chunks, d)),
+        _ptr(chunk_sum, "chunk_sum", cfg.summary_torch_dtype(), (B, H, cfg.n_chunks, d)),
         _ptr(qbar, "qbar", torch.float32, (B, H, nQC, d)),
         _ptr(sel_chunks, "sel_chunks", torch.int32, (B, H, nQC, cfg.top_k_chunks)),
         _ptr(n_sel_chunks, "n_sel_chunks", torch.int32, (B, H, nQC)),
@@ -198,7 +203,7 @@ def route_groups(cfg: HgaConfig, qbar, group_sum, sel_chunks, n_sel_chunks, sel_
     B, H, d, nQC, G = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.n_qchunks, cfg.groups_per_chunk
     _check(_lib.hga_route_groups(
         ctypes.byref(cfg), _ptr(qbar, "qbar", torch.float32, (B, H, nQC, d)),
-        _ptr(group_sum, "group_sum", torch.float32, (B, H, cfg.n_chunks * G, d)),
+        _ptr(group_sum, "group_sum", cfg.summary_torch_dtype(), (B, H, cfg.n_chunks * G, d)),
         _ptr(sel_chunks, "sel_chunks", torch.int32, (B, H, nQC, cfg.top_k_chunks)),
         _ptr(n_sel_chunks, "n_sel_chunks", torch.int32, (B, H, nQC)),
         _ptr(sel_groups, "sel_groups", torch.int32, (B, H, nQC, cfg.top_k_groups)),
@@ -212,8 +217,8 @@ def _route_ptrs(cfg: HgaConfig, q_rot, chunk_sum, group_sum, qbar, sel_chunks, n
     B, H, d, nQC, G = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.n_qchunks, cfg.groups_per_chunk
     return [
         _ptr(q_rot, "q_rot", cfg.torch_dtype(), (B, cfg.q_len, cfg.n_q_heads, d)),
-        _ptr(chunk_sum, "chunk_sum", torch.float32, (B, H, cfg.n_chunks, d)),
-        _ptr(group_sum, "group_sum", torch.float32, (B, H, cfg.n_chunks * G, d)),
+        _ptr(chunk_sum, "chunk_sum", cfg.summary_torch_dtype(), (B, H, cfg.n_chunks, d)),
+        _ptr(group_sum, "group_sum", cfg.summary_torch_dtype(), (B, H, cfg.n_chunks * G, d)),
         _ptr(qbar, "qbar", torch.float32, (B, H, nQC, d)),
         _ptr(sel_chunks, "sel_chunks", torch.int32, (B, H, nQC, cfg.top_k_chunks)),
         _ptr(n_sel_chunks, "n_sel_chunks", torch.int32, (B, H, nQC)),

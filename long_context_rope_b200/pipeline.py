@@ -56,8 +56,9 @@ def alloc_warm_pool(cfg: hga.HgaConfig, n_slots: int, device="cuda") -> WarmPool
 
 def alloc_summaries(cfg: hga.HgaConfig, device="cuda"):
     B, H, d, nC, G = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.n_chunks, cfg.groups_per_chunk
-    cs = torch.empty(B, H, nC, d, dtype=torch.float32, device=device)
-    gs = torch.empty(B, H, nC * G, d, dtype=torch.float32, device=device)
+    dt = cfg.summary_torch_dtype()
+    cs = torch.empty(B, H, nC, d, dtype=dt, device=device)
+    gs = torch.empty(B, H, nC * G, d, dtype=dt, device=device)
     return cs, gs
 
 

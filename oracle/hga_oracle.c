@@ -106,6 +106,11 @@ double hgaref_round_bf16(double x) {
     return (double)f;
 }
 
+/* out[i] = hgaref_round_bf16(in[i]) for i < n (bf16 summary tables). */
+void hgaref_round_bf16_n(const double* in, double* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = hgaref_round_bf16(in[i]);
+}
+
 /* Rotate rows x[n_tok][n_heads][d] where token t sits at position pos0 + t.
  * round_bf16 != 0 rounds each result to bf16 (the storage type of the cache). */
 void hgaref_rope(const hgaref_cfg* c, const float* x, int64_t n_tok, int n_heads,

@@ -59,6 +59,7 @@ def lib():
             handle = ctypes.CDLL(build())
             sig = {
                 "hgaref_round_bf16": (ctypes.c_double, [ctypes.c_double]),
+                "hgaref_round_bf16_n": (None, [_P, _P, ctypes.c_int64]),
                 "hgaref_rope": (None, [_P, _P, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
                                        ctypes.c_int, _P]),
                 "hgaref_build_summaries": (None, [_P, _P, _P, _P]),
@@ -121,6 +122,14 @@ def n_qchunks(cfg: OracleCfg) -> int:
 
 def round_bf16(x: float) -> float:
     return lib().hgaref_round_bf16(float(x))
+
+
+def round_bf16_array(a) -> np.ndarray:
+    """Every element rounded to bf16 (as round_bf16), float64 out."""
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    out = np.empty_like(a)
+    lib().hgaref_round_bf16_n(_ptr(a), _ptr(out), a.size)
+    return out
 
 
 def rope(cfg: OracleCfg, x, pos0: int, round_bf16: bool) -> np.ndarray:
@@ -222,13 +231,16 @@ def num_threads() -> int:
     return int(lib().hgaref_num_threads())
 
 
-def pipeline(w, inputs, units=None, want_scores: bool = True, attend_out: bool = True):
+def pipeline(w, inputs, units=None, want_scores: bool = True, attend_out: bool = True,
+             bf16_summaries: bool = False):
     """The whole oracle hot path on drawn inputs (torch CPU tensors or numpy).
 
     Steps, each the oracle's own: rotate queries and keys (rounded to bf16 for
     bf16 workloads: the storage type of the query and of the attention cache),
-    build summaries from the raw keys, q-bar, chunk routing, group routing,
-    and exact attention (on `units` only, if given).
+    build summaries from the raw keys (rounded to bf16 when bf16_summaries:
+    the bf16 summary-table variant routes on the rounded values), q-bar,
+    chunk routing, group routing, and exact attention (on `units` only, if
+    given).
     """
     cfg = cfg_of(w)
     rb = w.dtype == "bf16"
@@ -244,6 +256,8 @@ def pipeline(w, inputs, units=None, want_scores: bool = True, attend_out: bool =
     for b in range(B):
         q_rot[b] = rope_f32(cfg, q_raw[b], cfg.q_begin, rb)
     cs, gs = build_summaries(cfg, k_raw)
+    if bf16_summaries:
+        cs, gs = round_bf16_array(cs), round_bf16_array(gs)
     qb = qbar(cfg, q_rot)
     sel_c, nsel_c, sc_c = route_chunks(cfg, qb, cs, want_scores)
     sel_g, nsel_g, sc_g = route_groups(cfg, qb, gs, sel_c, nsel_c, want_scores)

@@ -31,14 +31,27 @@ def test_exports_every_declared_symbol(hga):
 
 
 def test_struct_layout_matches_header(hga):
-    # 12 int32 (48 bytes), a double at offset 48, 4 int32: 72 bytes, 8-byte aligned
-    assert ctypes.sizeof(hga.HgaConfig) == 72
+    # 12 int32 (48 bytes), a double at offset 48, 5 int32 (76), 8-byte aligned: 80
+    assert ctypes.sizeof(hga.HgaConfig) == 80
     assert hga.HgaConfig.rope_theta.offset == 48
+    assert hga.HgaConfig.summary_type.offset == 72
 
 
 def _cfg(hga, **kw):
     from long_context_rope_b200 import synth
     return hga.config_from(synth.WORKLOADS["prefill_4k"], **kw)
+
+
+def test_summary_type_validation_without_gpu(hga):
+    L = hga.library()
+    P = 16 * 1024  # never dereferenced: refused on the host
+    by = ctypes.byref
+    bad = _cfg(hga, summary_type=7)
+    assert L.hga_route_chunks(by(bad), P, P, P, P, P, None, None) == -4
+    bf = _cfg(hga, summary_type=hga.HGA_SUMMARY_BF16)
+    # the separate routing calls do not read bf16 tables
+    assert L.hga_route_chunks(by(bf), P, P, P, P, P, None, None) == -8
+    assert L.hga_route_groups(by(bf), P, P, P, P, P, P, None, None) == -8
 
 
 def test_status_strings(hga):

@@ -229,3 +229,60 @@ def test_decode_loop_appends_and_finalises_chunks():
             print(f"pos {pos}: chunks {int(rb.n_sel_chunks[0, 0, 0])} groups "
                   f"{int(rb.n_sel_groups[0, 0, 0])} max abs error {worst:.3e}")
     assert n_checked == len(check)
+
+
+def test_decode_step_bf16_summaries_vs_oracle():
+    """bf16 summary tables (the variant that halves the routing bytes of a
+    decode step): hga_build_summaries writes the fp32 summaries rounded to
+    bf16, and the one-launch step routes on them. The oracle's reading is its
+    double summaries rounded to bf16 (nearest even, through fp32); the GPU's
+    tables are equal up to one bf16 ulp where the fp32 and double sums fall on
+    either side of a rounding boundary, so routing is compared with the
+    slack bound of those measured differences (tests/parity_util.py), and
+    every output against the oracle on the GPU's selection where it
+    differs. The separate routing calls refuse bf16 tables."""
+    from long_context_rope_b200 import hga, pipeline
+    w = BASE.replace(name="bf16sum", batch=4, seq_len=16384)
+    x = synth.draw(w, seed=8)
+    r = O.pipeline(w, x, bf16_summaries=True)
+    cfg = hga.config_from(w, summary_type=hga.HGA_SUMMARY_BF16)
+    k_raw = x["k_raw"].cuda()
+    cs, gs = pipeline.alloc_summaries(cfg)
+    assert cs.dtype == torch.bfloat16
+    pipeline.summaries(cfg, k_raw, cs, gs, None)
+    k_rot = torch.from_numpy(np.ascontiguousarray(r["k_rot"])).to(torch.bfloat16).cuda()
+    q_rot = torch.from_numpy(np.ascontiguousarray(r["q_rot"])).to(torch.bfloat16).cuda()
+    v = x["v"].cuda()
+    rb = pipeline.alloc_route(cfg)
+    out = torch.full_like(q_rot, float("nan"))
+    pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out)
+    torch.cuda.synchronize()
+    assert hga.get_device_error() == 0
+    # a GPU table value is the bf16 rounding of an fp32 summary within the
+    # fp32 tolerance (2e-5 abs + rel) of the oracle's double one, so it lies
+    # within that tolerance plus one bf16 ulp of the oracle's rounded value
+    for name, got, want in (("chunk_sum", cs, r["chunk_sum"]), ("group_sum", gs, r["group_sum"])):
+        got = _np(got).astype(np.float64)
+        diff = got != want
+        bound = 2e-5 * (1.0 + np.abs(want)) + np.abs(want) * 2.0 ** -7
+        assert np.all(np.abs(got - want) <= bound), name
+        assert diff.mean() <= 1e-3, (name, diff.mean())
+    g = dict(qbar=_np(rb.qbar), chunk_sum=_np(cs), group_sum=_np(gs),
+             sel_chunks=_np(rb.sel_chunks), n_sel_chunks=_np(rb.n_sel_chunks), chunk_scores=None,
+             sel_groups=_np(rb.sel_groups), n_sel_groups=_np(rb.n_sel_groups), group_scores=None)
+    assert_close("qbar", g["qbar"], r["qbar"], atol=2e-5, rtol=2e-5)
+    same = compare_routing(w, g, r, O, slack=True)
+    assert same.mean() >= 0.9, same.mean()
+    vv = x["v"].float().numpy()
+
+    def oracle_alt(units):
+        return O.attend(O.cfg_of(w), r["q_rot"], r["k_rot"], vv, g["sel_groups"],
+                        g["n_sel_groups"], units=np.array(units, dtype=np.int32))
+
+    worst, n_alt = compare_outputs(w, _np(out), r["out"], same, oracle_alt)
+    rb2 = pipeline.alloc_route(cfg, with_scores=True)
+    with pytest.raises(hga.HgaError) as e:
+        pipeline.route(cfg, q_rot, cs, gs, rb2, separate=True)
+    assert e.value.status == -8
+    print(f"bf16 summaries: {same.mean():.3f} identical routing ({n_alt} units on the GPU's "
+          f"selection), max abs error {worst:.3e}")

@@ -89,6 +89,18 @@ def test_round_bf16_matches_torch_cast():
     np.testing.assert_array_equal(got, want.astype(np.float64))
 
 
+def test_round_bf16_array_matches_scalar_and_torch_cast():
+    """The array form used for bf16 summary tables: element by element the
+    scalar rounding, and torch's bf16 cast for float32-exact inputs."""
+    rng = np.random.default_rng(4)
+    xs = (rng.standard_normal(3000) * 10.0 ** rng.integers(-4, 4, 3000)).reshape(30, 100)
+    got = O.round_bf16_array(xs)
+    np.testing.assert_array_equal(got.ravel(), [O.round_bf16(float(x)) for x in xs.ravel()])
+    x32 = xs.astype(np.float32)
+    want = torch.from_numpy(x32).to(torch.bfloat16).float().numpy().astype(np.float64)
+    np.testing.assert_array_equal(O.round_bf16_array(x32), want)
+
+
 # ----------------------------------------------------------- summaries ---
 
 def _k(cfg, seed=4):
