@@ -37,7 +37,8 @@ TC_TRAFFIC_BYTES = 2 * 574.3e6
 TC_TRAFFIC_NOTE = ("ncu dram__bytes_read+write of attend_tc_kernel at 32K context x2 "
                    "(profiles/attend_tc_prefill_32k_ncu.md)")
 PREFILL = "prefill_64k"
-DECODES = ("decode_16x32k", "tiered_decode_4x64k")
+# ":bf16sum" = the same workload with bf16 summary tables
+DECODES = ("decode_16x32k", "decode_16x32k:bf16sum", "tiered_decode_4x64k")
 
 
 def load_peaks():
@@ -190,6 +191,8 @@ def run_prefill(args, dist, peaks):
     if hga.get_device_error() != 0:
         raise RuntimeError("device error word set during warm-up")
     flops = prefill_flops(cfg, rb.n_sel_groups.cpu().numpy())
+    recall = planted_recall(w, x["planted"], rb.sel_chunks.cpu().numpy(),
+                            rb.n_sel_chunks.cpu().numpy())
 
     K = args.steps
     ev = Events(5 * K)
@@ -211,7 +214,7 @@ def run_prefill(args, dist, peaks):
     attend_ms = float(np.mean(stage["attend"]))
     res = dict(total_ms=dist.max(total_ms), attend_ms=dist.max(attend_ms),
                stage_ms={n: float(np.mean(vs)) for n, vs in stage.items()},
-               flops=flops, tokens=w.batch * w.q_len, clocks=clk.summary(),
+               flops=flops, tokens=w.batch * w.q_len, clocks=clk.summary(), recall=recall,
                launches_per_step=5)
 
     # end to end through the public API with host buffers (pinned), H2D + D2H inside
@@ -249,8 +252,10 @@ def run_prefill(args, dist, peaks):
 
 def run_decode(name, args, dist):
     from long_context_rope_b200 import hga, pipeline
-    w = synth.WORKLOADS[name]
-    cfg = hga.config_from(w)
+    base, _, variant = name.partition(":")
+    w = synth.WORKLOADS[base]
+    bf16_sum = variant == "bf16sum"
+    cfg = hga.config_from(w, summary_type=hga.HGA_SUMMARY_BF16 if bf16_sum else hga.HGA_SUMMARY_F32)
     x = synth.draw(w, seed=dist.seed(args.seed))
     dev = torch.device("cuda", torch.cuda.current_device())
     st = torch.cuda.current_stream()
@@ -278,7 +283,7 @@ def run_decode(name, args, dist):
         # warm tier: a VRAM pool of 4 x top_k_groups groups per (sequence, KV head)
         pool = pipeline.alloc_warm_pool(cfg, 4 * cfg.top_k_groups, dev)
 
-        def step(separate=False, warm=False):
+        def step_fn(separate=False, warm=False):
             pipeline.decode(cfg_w, q_rot, cs, gs, k_win, v_win, rb, out, gathered=gat,
                             k_src=k_host, v_src=v_host, src_is_host=True, separate=separate,
                             warm=pool if warm else None)
@@ -286,15 +291,20 @@ def run_decode(name, args, dist):
     else:
         v = x["v"].to(dev)
 
-        def step(separate=False, warm=False):
+        def step_fn(separate=False, warm=False):
             pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out, separate=separate)
         launches, launches_sep = 1, 3  # one-launch decode step
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     K = max(args.steps, 20)
 
-    def timed(separate, warm=False):
+    def timed(separate, warm=False, fn=None):
         """Median device time of one step replayed from a CUDA graph (L2
-        flushed between steps), plus the eager median for reference."""
+        flushed between steps), plus the eager median for reference. `fn`
+        (no arguments) replaces the step when given."""
+        if fn is not None:
+            step = lambda separate, warm: fn()  # noqa: E731
+        else:
+            step = step_fn
         for _ in range(max(3, args.warmup)):
             step(separate, warm)
         torch.cuda.synchronize()
@@ -327,10 +337,11 @@ def run_decode(name, args, dist):
         del graph
         return times, eager
 
-    times_sep, eager_sep = timed(True)
+    # the separate routing calls read fp32 tables only
+    times_sep, eager_sep = (None, None) if bf16_sum else timed(True)
     times, eager_us = timed(False)
     us = dist.max(float(np.median(times)))
-    us_sep = dist.max(float(np.median(times_sep)))
+    us_sep = dist.max(float(np.median(times_sep))) if times_sep else None
     warm_info = None
     if w.tiered:
         # steady state of the warm tier for this (fixed) query: its routed groups
@@ -342,23 +353,147 @@ def run_decode(name, args, dist):
                          hit_rate=float(hits_misses[0] / max(1, hits_misses.sum())),
                          host_bytes_per_step=int(hits_misses[1]) * 16 * w.head_dim * 2 * 2,
                          note="fixed query: the all-hits steady state of the warm tier")
+        warm_info["drifting"] = run_warm_drift(w, args, dist, cfg, cfg_w, cs, gs, k_win, v_win,
+                                               k_host, v_host, st)
     n_sel = rb.n_sel_groups.cpu().numpy()
     moved = int(n_sel.sum()) * 16 * w.head_dim * 2 * 2  # routed K+V bytes
+    recall = planted_recall(w, x["planted"], rb.sel_chunks.cpu().numpy(),
+                            rb.n_sel_chunks.cpu().numpy())
+    gather_info = None
+    if not w.tiered and not bf16_sum:
+        # the exact-token gather from HBM alone (hga_gather_kv): (1) one launch
+        # replayed from a CUDA graph after an L2 flush (includes the graph's
+        # launch latency); (2) launches back to back, cycling through the
+        # selections of 8 different queries, so each launch reads groups the
+        # previous seven launches' 700 MB of traffic has evicted from L2 and
+        # the launch latency overlaps the previous launch (the kernel's
+        # throughput). Each launch reads and writes every routed group's K
+        # and V once.
+        times_g, _ = timed(False, fn=lambda: hga.gather_kv(
+            cfg, k_rot, v, False, rb.sel_groups, rb.n_sel_groups, gat[0], gat[1]))
+        sels = []
+        for i in range(8):
+            xi = synth.draw(w, seed=dist.seed(args.seed) + 104729 * (i + 1), with_kv=False)
+            rbi = pipeline.alloc_route(cfg, dev)
+            pipeline.route(cfg, pipeline.rotate_queries(cfg, xi["q_raw"].to(dev)), cs, gs, rbi)
+            sels.append(rbi)
+        torch.cuda.synchronize()
+        moved_seq = sum(int(r.n_sel_groups.sum()) for r in sels) * 16 * w.head_dim * 2 * 2 / 8
+        n_seq = 32
+        flush.fill_(1)
+        ev = Events(2)
+        ev.rec(0, st)
+        for i in range(n_seq):
+            r_i = sels[i % 8]
+            hga.gather_kv(cfg, k_rot, v, False, r_i.sel_groups, r_i.n_sel_groups, gat[0], gat[1])
+        ev.rec(1, st)
+        torch.cuda.synchronize()
+        if hga.get_device_error() != 0:
+            raise RuntimeError("device error word set in the gather run")
+        seq_us = dist.max(ev.ms(0, 1) * 1000.0 / n_seq)
+        g_us = dist.max(float(np.median(times_g)))
+        g_bytes = 2 * moved
+        peak = load_peaks()["hbm"]
+        gather_info = dict(kernel="gather_hbm_kernel (hga_gather_kv, HBM source)",
+                           us=seq_us, bytes=2 * moved_seq,
+                           hbm_gbs=2 * moved_seq / (seq_us * 1e-6) / 1e9,
+                           hbm_frac=2 * moved_seq / (seq_us * 1e-6) / 1e9 / peak,
+                           timing=f"{n_seq} launches back to back over 8 queries' selections",
+                           us_single_graph=g_us, bytes_single=g_bytes,
+                           hbm_frac_single_graph=g_bytes / (g_us * 1e-6) / 1e9 / peak,
+                           launches=1)
     # algorithmic HBM bytes of one step (each byte the step must touch, once)
     n_forced_tok = (min(w.n_sink, w.n_chunks) + w.n_local + 1) * w.chunk_size
     forced_kv = w.batch * w.n_kv_heads * n_forced_tok * w.head_dim * 2 * 2
-    chunk_sums = w.batch * w.n_kv_heads * w.n_chunks * w.head_dim * 4
-    group_sums = int(rb.n_sel_chunks.cpu().numpy().sum()) * w.groups_per_chunk * w.head_dim * 4
+    se = 2 if bf16_sum else 4  # summary element bytes
+    chunk_sums = w.batch * w.n_kv_heads * w.n_chunks * w.head_dim * se
+    group_sums = int(rb.n_sel_chunks.cpu().numpy().sum()) * w.groups_per_chunk * w.head_dim * se
     q_o = 2 * w.batch * w.n_q_heads * w.head_dim * 2
     hbm_bytes = forced_kv + chunk_sums + group_sums + q_o + (2 * moved if w.tiered else moved)
-    return dict(workload=name, us_per_step=us, us_min=float(np.min(times)), steps=K,
+    return dict(workload=name, summary_tables="bf16" if bf16_sum else "fp32", us_per_step=us, us_min=float(np.min(times)), steps=K,
                 hbm_bytes_per_step=hbm_bytes, hbm_gbs=hbm_bytes / (us * 1e-6) / 1e9,
                 hbm_frac=hbm_bytes / (us * 1e-6) / 1e9 / load_peaks()["hbm"],
                 us_per_step_eager=eager_us, cuda_graph=True,
                 launches_per_step=launches, routed_kv_bytes=moved,
                 us_per_step_separate_kernels=us_sep, us_per_step_separate_eager=eager_sep,
                 launches_per_step_separate=launches_sep, warm_tier=warm_info,
+                gather=gather_info, planted_recall=recall,
                 host_link_gbs=(moved / (us * 1e-6) / 1e9) if w.tiered else None)
+
+
+def run_warm_drift(w, args, dist, cfg, cfg_w, cs, gs, k_win, v_win, k_host, v_host, st,
+                   n_queries=8, steps_per_query=4, n_steps=48):
+    """The warm tier on a decode sequence whose planted topic drifts: step s
+    uses query q[(s // steps_per_query) % n_queries], each drawn with its own
+    seed (its own planted source chunk and noise), so routed groups enter and
+    age out of the pool. After one pass over the queries (pool warm-up), the
+    timed steps report the hit rate, the host-link bytes per step and the
+    device time per step (route + warm gather + attention, eager launches)."""
+    from long_context_rope_b200 import hga, pipeline
+    dev = torch.device("cuda", torch.cuda.current_device())
+    qs = []
+    for i in range(n_queries):
+        xi = synth.draw(w, seed=dist.seed(args.seed) + 7919 * (i + 1), with_kv=False)
+        qs.append(pipeline.rotate_queries(cfg, xi["q_raw"].to(dev)))
+    pool = pipeline.alloc_warm_pool(cfg, 4 * cfg.top_k_groups, dev)
+    rb = pipeline.alloc_route(cfg, dev)
+    gat = pipeline.alloc_gathered(cfg, dev)
+    out = torch.empty_like(qs[0])
+
+    def step(s):
+        pipeline.decode(cfg_w, qs[(s // steps_per_query) % n_queries], cs, gs, k_win, v_win, rb,
+                        out, gathered=gat, k_src=k_host, v_src=v_host, src_is_host=True,
+                        warm=pool)
+
+    warm_steps = n_queries * steps_per_query
+    for s in range(warm_steps):
+        step(s)
+    torch.cuda.synchronize()
+    ev = Events(2 * n_steps)
+    hits = misses = 0
+    for i in range(n_steps):
+        ev.rec(2 * i, st)
+        step(warm_steps + i)
+        ev.rec(2 * i + 1, st)
+        hm = pool.stats.sum(dim=(0, 1))
+        hits += int(hm[0])
+        misses += int(hm[1])
+    torch.cuda.synchronize()
+    if hga.get_device_error() != 0:
+        raise RuntimeError("device error word set in the drifting warm-tier run")
+    times = [ev.ms(2 * i, 2 * i + 1) * 1000.0 for i in range(n_steps)]
+    group_bytes = 16 * w.head_dim * 2 * 2
+    return dict(us_per_step=dist.max(float(np.median(times))), steps=n_steps,
+                hit_rate=hits / max(1, hits + misses),
+                host_bytes_per_step=misses * group_bytes / n_steps,
+                schedule=f"{n_queries} planted queries, each for {steps_per_query} consecutive "
+                         f"steps, cycled; pool {pool.tag.shape[-1]} groups per (sequence, KV head)")
+
+
+def planted_recall(w, planted, sel_chunks: np.ndarray, n_sel_chunks: np.ndarray) -> dict:
+    """How often the chunk whose topic was planted into a query chunk is in
+    that query chunk's visible set: selected by level-1 routing, or always
+    visible (sinks, locals, current). Reported as a statistic of the
+    synthetic data, not a parity bar."""
+    C = w.chunk_size
+    j0 = w.q_begin // C
+    seen = routed = total = cand = 0
+    for b, per_b in enumerate(planted):
+        for jj, srcs in enumerate(per_b):
+            j = j0 + jj
+            if jj >= sel_chunks.shape[2]:
+                continue
+            for h in range(w.n_kv_heads):
+                sel = set(sel_chunks[b, h, jj, :n_sel_chunks[b, h, jj]].tolist())
+                for c in srcs:
+                    forced = c < w.n_sink or j - w.n_local <= c <= j
+                    total += 1
+                    seen += int(forced or c in sel)
+                    if not forced:
+                        cand += 1
+                        routed += int(c in sel)
+    return dict(visible=seen / max(1, total), routed_among_candidates=routed / max(1, cand),
+                planted=total, planted_candidates=cand)
 
 
 def host_link_peak_gbs(dev) -> float:
@@ -509,6 +644,7 @@ def main():
                          else None,
                          "flops_per_launch": pre["flops"],
                          "peak_note": tc_note},
+            "planted_recall": pre["recall"],
             "gpu_launches": pre["launches_per_step"] * args.steps,
             "clocks": pre["clocks"],
         }
