@@ -284,10 +284,14 @@ def run_decode(name, args, dist):
         pool = pipeline.alloc_warm_pool(cfg, 4 * cfg.top_k_groups, dev)
 
         def step_fn(separate=False, warm=False):
-            pipeline.decode(cfg_w, q_rot, cs, gs, k_win, v_win, rb, out, gathered=gat,
-                            k_src=k_host, v_src=v_host, src_is_host=True, separate=separate,
-                            warm=pool if warm else None)
-        launches, launches_sep = 3, 4  # route (one launch), gather, attend
+            if separate or warm:  # route (one launch), [warm] gather, attend
+                pipeline.decode(cfg_w, q_rot, cs, gs, k_win, v_win, rb, out, gathered=gat,
+                                k_src=k_host, v_src=v_host, src_is_host=True,
+                                warm=pool if warm else None)
+            else:  # one launch: routed groups read from the host inside the kernel
+                pipeline.decode_tiered(cfg_w, q_rot, cs, gs, k_win, v_win, k_host, v_host, rb,
+                                       out)
+        launches, launches_sep = 1, 3
     else:
         v = x["v"].to(dev)
 
@@ -409,7 +413,9 @@ def run_decode(name, args, dist):
     chunk_sums = w.batch * w.n_kv_heads * w.n_chunks * w.head_dim * se
     group_sums = int(rb.n_sel_chunks.cpu().numpy().sum()) * w.groups_per_chunk * w.head_dim * se
     q_o = 2 * w.batch * w.n_q_heads * w.head_dim * 2
-    hbm_bytes = forced_kv + chunk_sums + group_sums + q_o + (2 * moved if w.tiered else moved)
+    # tiered: the one-launch step reads the routed groups from the host, not
+    # from HBM (the three-launch path also writes and reads them in a buffer)
+    hbm_bytes = forced_kv + chunk_sums + group_sums + q_o + (0 if w.tiered else moved)
     return dict(workload=name, summary_tables="bf16" if bf16_sum else "fp32", us_per_step=us, us_min=float(np.min(times)), steps=K,
                 hbm_bytes_per_step=hbm_bytes, hbm_gbs=hbm_bytes / (us * 1e-6) / 1e9,
                 hbm_frac=hbm_bytes / (us * 1e-6) / 1e9 / load_peaks()["hbm"],
@@ -418,7 +424,8 @@ def run_decode(name, args, dist):
                 us_per_step_separate_kernels=us_sep, us_per_step_separate_eager=eager_sep,
                 launches_per_step_separate=launches_sep, warm_tier=warm_info,
                 gather=gather_info, planted_recall=recall,
-                host_link_gbs=(moved / (us * 1e-6) / 1e9) if w.tiered else None)
+                host_link_gbs=(moved / (us * 1e-6) / 1e9) if w.tiered else None,
+                host_link_gbs_separate=(moved / (us_sep * 1e-6) / 1e9) if w.tiered else None)
 
 
 def run_warm_drift(w, args, dist, cfg, cfg_w, cs, gs, k_win, v_win, k_host, v_host, st,

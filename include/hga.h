@@ -205,6 +205,28 @@ hga_status hga_decode_step(const hga_config* cfg, const void* q_rot, const void*
                            float* qbar_out, int32_t* sel_chunks, int32_t* n_sel_chunks,
                            int32_t* sel_groups, int32_t* n_sel_groups, void* out, void* stream);
 
+/* One decode step over the tiered store of "Geheugenarchitectuur" in a
+ * single launch: the hot tier (summary tables and the forced chunks'
+ * windows) in device memory, the cold tier (the full K/V history) in host
+ * memory. Routing as hga_route; then exact attention ("Kernmechanisme" item
+ * 4) over the forced chunks, read from the resident windows k_win / v_win
+ * [B, Hkv, W * C, d] (W = n_sink + n_local + 1 slots in ascending chunk
+ * order, as for HGA_KV_WINDOWS), and over the selected groups, whose rows
+ * are read from k_host / v_host [B, Hkv, L, d] (page-locked host memory
+ * mapped into the device address space) inside the same kernel, so the
+ * host-link reads overlap the attention over the resident windows and
+ * nothing is staged in a gathered buffer. Writes q-bar, both selections (as
+ * hga_route) and out [B, 1, Hq, d]; the result equals hga_route +
+ * hga_gather_kv (host) + hga_attend in HGA_KV_WINDOWS within fp32 summation
+ * order. Needs cfg->kv_layout == HGA_KV_WINDOWS, a one-token query at
+ * q_begin == L - 1, and the one-launch configuration of hga_decode_step;
+ * else HGA_ERR_UNSUPPORTED. HGA_ERR_MEMORY if a host pointer is not mapped. */
+hga_status hga_decode_step_tiered(const hga_config* cfg, const void* q_rot, const void* chunk_sum,
+                                  const void* group_sum, const void* k_win, const void* v_win,
+                                  const void* k_host, const void* v_host, float* qbar_out,
+                                  int32_t* sel_chunks, int32_t* n_sel_chunks, int32_t* sel_groups,
+                                  int32_t* n_sel_groups, void* out, void* stream);
+
 /* Exact-token retrieval ("Kernmechanisme" item 4; "Geheugenarchitectuur"
  * cold tier): copy the K and V rows of every selected group into compact
  * buffers k_dst, v_dst [B, Hkv, nQC, top_k_groups * g, d]; slot s holds the

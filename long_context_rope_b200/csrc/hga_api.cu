@@ -180,7 +180,7 @@ static_assert(offsetof(hga_config, rope_theta) == 48, "hga_config layout is part
 
 extern "C" {
 
-int32_t hga_version(void) { return 10500; }
+int32_t hga_version(void) { return 10600; }
 
 void hga_set_wait_limit_ns(uint64_t limit_ns) {
     g_wait_ns.store(limit_ns == 0 ? 1000000000ull : (unsigned long long)limit_ns,
@@ -362,6 +362,37 @@ hga_status hga_decode_step(const hga_config* cfg, const void* q_rot, const void*
     if (decode_kernel_supports(p))
         return launched(launch_attend_decode(p, q_rot, kv, sel_groups, n_sel_groups, out, st));
     return launched(launch_attend_simt(p, q_rot, kv, sel_groups, n_sel_groups, out, st));
+}
+
+static hga_status device_view(const void* ptr, bool want_host, const void** dev_ptr);
+
+hga_status hga_decode_step_tiered(const hga_config* cfg, const void* q_rot, const void* chunk_sum,
+                                  const void* group_sum, const void* k_win, const void* v_win,
+                                  const void* k_host, const void* v_host, float* qbar_out,
+                                  int32_t* sel_chunks, int32_t* n_sel_chunks, int32_t* sel_groups,
+                                  int32_t* n_sel_groups, void* out, void* stream) {
+    Params p;
+    hga_status s = make_params(cfg, &p);
+    if (s != HGA_OK) return s;
+    if (p.nQC == 0) return HGA_OK;
+    s = check_route_args(p, q_rot, chunk_sum, group_sum, qbar_out, sel_chunks, n_sel_chunks,
+                         sel_groups, n_sel_groups);
+    if (s != HGA_OK) return s;
+    if (!k_win || !v_win || !k_host || !v_host || !out) return HGA_ERR_NULL;
+    if (!aligned16(k_win) || !aligned16(v_win) || !aligned16(k_host) || !aligned16(v_host) ||
+        !aligned16(out))
+        return HGA_ERR_ALIGN;
+    if (p.kv_layout != HGA_KV_WINDOWS || p.q_len != 1 || p.q_begin != p.L - 1 ||
+        !decode_step_supports(p))
+        return HGA_ERR_UNSUPPORTED;
+    HGA_ATTACH_ERR(p);
+    const void* kd = nullptr;
+    const void* vd = nullptr;
+    if ((s = device_view(k_host, true, &kd)) != HGA_OK) return s;
+    if ((s = device_view(v_host, true, &vd)) != HGA_OK) return s;
+    return launched(launch_decode_step(p, q_rot, chunk_sum, group_sum, k_win, v_win, qbar_out,
+                                       sel_chunks, n_sel_chunks, sel_groups, n_sel_groups, out,
+                                       (cudaStream_t)stream, kd, vd));
 }
 
 static hga_status device_view(const void* ptr, bool want_host, const void** dev_ptr) {

@@ -97,16 +97,20 @@ cudaError_t launch_attend_decode(const Params& p, const void* q_rot, const KvSou
                                  const int32_t* sel_groups, const int32_t* n_sel_groups,
                                  void* out, cudaStream_t st);
 
-// One-launch decode step (q-bar, both routing levels, attention over the
-// full resident cache): bf16, d = 128, one query token, gq <= 8, L % 16 == 0,
-// top_k_chunks <= 64, top_k_groups <= 512, and routing tables that fit one
-// cluster's shared memory. With out == nullptr it stops after routing.
+// One-launch decode step (q-bar, both routing levels, attention): bf16,
+// d = 128, one query token, gq <= 8, L % 16 == 0, top_k_chunks <= 64,
+// top_k_groups <= 512, and routing tables that fit one cluster's shared
+// memory. With out == nullptr it stops after routing. The keys come from
+// k_cache / v_cache in p.kv_layout: the full resident store, or (with
+// k_host / v_host, the full store in mapped host memory) the resident
+// windows of the forced chunks, the routed groups then read from the host.
 bool decode_step_supports(const Params& p);
 // Summary tables fp32, or bf16 when p.sum_bf16.
 cudaError_t launch_decode_step(const Params& p, const void* q_rot, const void* chunk_sum,
                                const void* group_sum, const void* k_cache, const void* v_cache,
                                float* qbar, int32_t* sel_chunks, int32_t* n_sel_chunks,
                                int32_t* sel_groups, int32_t* n_sel_groups, void* out,
-                               cudaStream_t st);
+                               cudaStream_t st, const void* k_host = nullptr,
+                               const void* v_host = nullptr);
 
 }  // namespace hga

@@ -79,7 +79,8 @@ struct StepSmem {
     int rank[kMaxSlice > kMaxCand2 ? kMaxSlice : kMaxCand2];  // rank scratch
     int win1[kMaxKc];             // selected chunks, ascending
     int routed[kMaxKg];           // selected groups, ascending
-    int blk_pos[kMaxLocal];
+    int blk_pos[kMaxLocal];       // position of a local block's first key
+    int blk_row[kMaxLocal];       // its first row in the resident store (TMA source)
     int n_win1, n_wl, bad;
 };
 
@@ -171,13 +172,46 @@ __device__ __forceinline__ void score_rows(const float* q, int n, RowOf row_of, 
     }
 }
 
+// Producer warp, host tier: the K and V rows of one routed group (16 rows of
+// d = 128 bf16 each, contiguous in the full store) read over the host link
+// with 16-byte loads (each lane 8 of each tensor, 512 contiguous bytes per
+// warp load) and stored into ring stage s in the layout the TMA tile loads
+// write: two 64-column panels of 16 rows x 128 bytes, 16-byte chunk c of
+// row r at c ^ (r % 8).
+__device__ __forceinline__ void copy_host_block(dec::Ring& ring, int s, const uint4* kh,
+                                                const uint4* vh) {
+    const int lane = threadIdx.x & 31;
+    uint4 kr[8], vr[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        kr[u] = kh[lane + 32 * u];
+        vr[u] = vh[lane + 32 * u];
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int idx = lane + 32 * u;               // 16-byte piece of the 4 KiB block
+        const int row = idx >> 4, c16 = idx & 15;
+        const int off = (c16 >> 3) * 2048 + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(ring.k[s] + off) = kr[u];
+        *reinterpret_cast<uint4*>(ring.v[s] + off) = vr[u];
+    }
+    // a later tile load into this stage (async proxy) is ordered after these
+    // stores
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // S: element type of the summary tables (float, or bf16 for bf16 tables).
+// k_host / v_host: nullptr, or the full store [B, Hkv, L, d] in mapped host
+// memory (the host tier); then the maps cover the resident windows of the
+// forced chunks ([B, Hkv, W * C, d]) and the routed groups are read from the
+// host by the producer warp.
 template <typename S>
 __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     const __grid_constant__ StepMaps maps, Params p, const __nv_bfloat16* __restrict__ q,
     const S* __restrict__ cs, const S* __restrict__ gs, float* __restrict__ qbar_out,
     int32_t* __restrict__ sel_c, int32_t* __restrict__ nsel_c, int32_t* __restrict__ sel_g,
-    int32_t* __restrict__ nsel_g, __nv_bfloat16* __restrict__ out, int attend) {
+    int32_t* __restrict__ nsel_g, __nv_bfloat16* __restrict__ out, int attend,
+    const uint4* __restrict__ k_host, const uint4* __restrict__ v_host) {
     extern __shared__ uint8_t smem_raw[];
     StepSmem& sm = *reinterpret_cast<StepSmem*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -211,16 +245,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
         }
         ptx::fence_mbar_init();
     }
+    const bool host_tier = k_host != nullptr;
     for (int i = tid; i < nf_loc; i += blockDim.x) {
         const int fi = f_lo + i, w = fi / p.G, gm = fi % p.G;
         const int c = w < s_end ? w : l_begin + (w - s_end);
         sm.blk_pos[i] = c * p.C + kGroupRows * gm;
+        // resident windows: forced chunk w of the list sits in slot w
+        sm.blk_row[i] = host_tier ? w * p.C + kGroupRows * gm : sm.blk_pos[i];
     }
     __syncthreads();
     const int n_pre = nf_loc < kStages ? nf_loc : kStages;
     if (attend && warp == kConsumers && lane == 0)
         for (int i = 0; i < n_pre; ++i)
-            dec::issue_block(sm.u.ring, sm.full, i, &maps.k, &maps.v, sm.blk_pos[i], (int)bh);
+            dec::issue_block(sm.u.ring, sm.full, i, &maps.k, &maps.v, sm.blk_row[i], (int)bh);
 
     // ---- level-1 slice: the first batch of this warp's chunk-summary rows is
     // requested before q-bar, so the two memory latencies overlap
@@ -388,22 +425,42 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     const int r_lo = r * pr;
     int nr_loc = nw - r_lo < pr ? nw - r_lo : pr;
     nr_loc = nr_loc < 0 ? 0 : nr_loc;
-    for (int i = tid; i < nr_loc; i += blockDim.x)
+    for (int i = tid; i < nr_loc; i += blockDim.x) {
         sm.blk_pos[nf_loc + i] = sm.routed[r_lo + i] * kGroupRows;
+        sm.blk_row[nf_loc + i] = sm.routed[r_lo + i] * kGroupRows;
+    }
     const int nloc = nf_loc + nr_loc;
     __syncthreads();
     if (warp == kConsumers) {
-        if (lane == 0) {
-            int i = n_pre;
-            for (; i < nloc; ++i) {
-                const int s = i % kStages;
-                if (i >= kStages &&
-                    !ptx::mbar_wait_bounded(&sm.empty[s], ((i / kStages) - 1) & 1, p.wait_ns)) {
-                    raise_timeout(p);
-                    sm.bad = 1;
+        // lane 0 waits for free stages and issues the tile loads of resident
+        // blocks; a routed block of the host tier is copied by the whole warp
+        // (its stage's barrier then completes on lane 0's plain arrival)
+        int i = n_pre;
+        bool ok = true;
+        for (; i < nloc; ++i) {
+            const int s = i % kStages;
+            if (i >= kStages) {
+                bool got = true;
+                if (lane == 0)
+                    got = ptx::mbar_wait_bounded(&sm.empty[s], ((i / kStages) - 1) & 1, p.wait_ns);
+                if (!__shfl_sync(0xffffffffu, got, 0)) {
+                    ok = false;
                     break;
                 }
-                dec::issue_block(sm.u.ring, sm.full, s, &maps.k, &maps.v, sm.blk_pos[i], (int)bh);
+            }
+            if (host_tier && i >= nf_loc) {
+                const int64_t row = bh * (int64_t)p.L + sm.blk_row[i];
+                copy_host_block(sm.u.ring, s, k_host + row * (kD / 8), v_host + row * (kD / 8));
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&sm.full[s]);
+            } else if (lane == 0) {
+                dec::issue_block(sm.u.ring, sm.full, s, &maps.k, &maps.v, sm.blk_row[i], (int)bh);
+            }
+        }
+        if (lane == 0) {
+            if (!ok) {
+                raise_timeout(p);
+                sm.bad = 1;
             }
             // every issued load (the early forced blocks included) lands
             // before the ring's memory is reused
@@ -508,7 +565,7 @@ int step_cluster(const Params& p, size_t smem) {
 
 bool decode_step_supports(const Params& p) {
     if (!(p.dtype == HGA_BF16 && p.d == kD && p.q_len == 1 && p.gq <= 8 && p.L % kGroupRows == 0 &&
-          p.kv_layout == HGA_KV_FULL && p.kc <= kMaxKc && p.kg <= kMaxKg && p.nQC == 1))
+          p.kc <= kMaxKc && p.kg <= kMaxKg && p.nQC == 1))
         return false;
     for (int cl = 1; cl <= kMaxCluster; ++cl)
         if (step_fits(p, cl)) return true;
@@ -521,13 +578,17 @@ template <typename S>
 cudaError_t launch_step(const Params& p, const void* q_rot, const S* chunk_sum,
                         const S* group_sum, const void* k_cache, const void* v_cache, float* qbar,
                         int32_t* sel_chunks, int32_t* n_sel_chunks, int32_t* sel_groups,
-                        int32_t* n_sel_groups, void* out, cudaStream_t st) {
+                        int32_t* n_sel_groups, void* out, const void* k_host, const void* v_host,
+                        cudaStream_t st) {
     const bool attend = out != nullptr;
     StepMaps maps;
     if (attend) {
         const int64_t BH = (int64_t)p.B * p.Hkv;
-        if (!make_rows_map(&maps.k, k_cache, BH, p.L, kD, kGroupRows) ||
-            !make_rows_map(&maps.v, v_cache, BH, p.L, kD, kGroupRows))
+        const int64_t rows = p.kv_layout == HGA_KV_WINDOWS
+                                 ? (int64_t)(p.n_sink + p.n_local + 1) * p.C
+                                 : (int64_t)p.L;
+        if (!make_rows_map(&maps.k, k_cache, BH, rows, kD, kGroupRows) ||
+            !make_rows_map(&maps.v, v_cache, BH, rows, kD, kGroupRows))
             return cudaErrorInvalidValue;
     } else {
         memset(&maps, 0, sizeof(maps));
@@ -551,7 +612,8 @@ cudaError_t launch_step(const Params& p, const void* q_rot, const S* chunk_sum,
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, decode_step_kernel<S>, maps, p, (const __nv_bfloat16*)q_rot,
                               chunk_sum, group_sum, qbar, sel_chunks, n_sel_chunks, sel_groups,
-                              n_sel_groups, (__nv_bfloat16*)out, attend ? 1 : 0);
+                              n_sel_groups, (__nv_bfloat16*)out, attend ? 1 : 0,
+                              (const uint4*)k_host, (const uint4*)v_host);
 }
 
 }  // namespace
@@ -560,13 +622,14 @@ cudaError_t launch_decode_step(const Params& p, const void* q_rot, const void* c
                                const void* group_sum, const void* k_cache, const void* v_cache,
                                float* qbar, int32_t* sel_chunks, int32_t* n_sel_chunks,
                                int32_t* sel_groups, int32_t* n_sel_groups, void* out,
-                               cudaStream_t st) {
+                               cudaStream_t st, const void* k_host, const void* v_host) {
     if (p.sum_bf16)
         return launch_step(p, q_rot, (const __nv_bfloat16*)chunk_sum,
                            (const __nv_bfloat16*)group_sum, k_cache, v_cache, qbar, sel_chunks,
-                           n_sel_chunks, sel_groups, n_sel_groups, out, st);
+                           n_sel_chunks, sel_groups, n_sel_groups, out, k_host, v_host, st);
     return launch_step(p, q_rot, (const float*)chunk_sum, (const float*)group_sum, k_cache,
-                       v_cache, qbar, sel_chunks, n_sel_chunks, sel_groups, n_sel_groups, out, st);
+                       v_cache, qbar, sel_chunks, n_sel_chunks, sel_groups, n_sel_groups, out,
+                       k_host, v_host, st);
 }
 
 }  // namespace hga

@@ -88,6 +88,7 @@ def _load():
         "hga_attend": [C, P, P, P, P, P, P, P, P, P],
         "hga_route": [C, P, P, P, P, P, P, P, P, P],
         "hga_decode_step": [C, P, P, P, P, P, P, P, P, P, P, P, P],
+        "hga_decode_step_tiered": [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P],
         "hga_gather_kv_warm": [C, P, P, P, P, P, P, P, P, I32, I32, P, P, P, P, P],
         "hga_gather_kv_warm_noalloc": [C, P, P, P, P, P, P, P, P, I32, I32, P, P, P, P],
         "hga_get_device_error": [P, ctypes.POINTER(I32)],
@@ -247,6 +248,24 @@ def decode_step(cfg: HgaConfig, q_rot, chunk_sum, group_sum, k_cache, v_cache, q
         _ptr(k_cache, "k_cache", dt, (B, H, L, d)), _ptr(v_cache, "v_cache", dt, (B, H, L, d)),
         *r[3:], _ptr(out, "out", dt, (B, cfg.q_len, cfg.n_q_heads, d)), _stream(stream)),
         "hga_decode_step")
+
+
+def decode_step_tiered(cfg: HgaConfig, q_rot, chunk_sum, group_sum, k_win, v_win, k_host, v_host,
+                       qbar, sel_chunks, n_sel_chunks, sel_groups, n_sel_groups, out,
+                       stream=None) -> None:
+    """One tiered decode step in one launch: routing, attention over the
+    resident forced windows and the routed groups read from host memory."""
+    B, H, L, d = cfg.batch, cfg.n_kv_heads, cfg.seq_len, cfg.head_dim
+    dt = cfg.torch_dtype()
+    win = (B, H, window_slots(cfg) * cfg.chunk_size, d)
+    r = _route_ptrs(cfg, q_rot, chunk_sum, group_sum, qbar, sel_chunks, n_sel_chunks, sel_groups,
+                    n_sel_groups)
+    _check(_lib.hga_decode_step_tiered(
+        ctypes.byref(cfg), r[0], r[1], r[2], _ptr(k_win, "k_win", dt, win),
+        _ptr(v_win, "v_win", dt, win), _ptr(k_host, "k_host", dt, (B, H, L, d), device=False),
+        _ptr(v_host, "v_host", dt, (B, H, L, d), device=False), *r[3:],
+        _ptr(out, "out", dt, (B, cfg.q_len, cfg.n_q_heads, d)), _stream(stream)),
+        "hga_decode_step_tiered")
 
 
 def gather_kv(cfg: HgaConfig, k_src, v_src, src_is_host: bool, sel_groups, n_sel_groups, k_dst,

@@ -147,6 +147,16 @@ def decode(cfg: hga.HgaConfig, q_rot, cs, gs, k_res, v_res, rb: RouteBuffers, ou
         hga.attend(cfg, q_rot, k_res, v_res, rb.sel_groups, rb.n_sel_groups, out, stream=stream)
 
 
+def decode_tiered(cfg_w: hga.HgaConfig, q_rot, cs, gs, k_win, v_win, k_host, v_host,
+                  rb: RouteBuffers, out, stream=None):
+    """One decode step over the tiered store in one launch
+    (hga_decode_step_tiered): the forced chunks from the resident windows,
+    the routed groups read from the host store inside the kernel."""
+    hga.decode_step_tiered(cfg_w, q_rot, cs, gs, k_win, v_win, k_host, v_host, rb.qbar,
+                           rb.sel_chunks, rb.n_sel_chunks, rb.sel_groups, rb.n_sel_groups, out,
+                           stream)
+
+
 def forced_window_chunks(cfg: hga.HgaConfig):
     """Forced chunks of the decode query chunk, ascending (the slot order of
     the HGA_KV_WINDOWS buffer)."""

@@ -54,6 +54,21 @@ def test_summary_type_validation_without_gpu(hga):
     assert L.hga_route_groups(by(bf), P, P, P, P, P, P, None, None) == -8
 
 
+def test_tiered_step_validation_without_gpu(hga):
+    L = hga.library()
+    P = 16 * 1024  # never dereferenced: refused on the host
+    by = ctypes.byref
+    dec = _cfg(hga, q_begin=4095, q_len=1, kv_layout=hga.HGA_KV_WINDOWS)
+    args = [P] * 13 + [None]
+    nul = list(args)
+    nul[5] = None  # k_host
+    assert L.hga_decode_step_tiered(by(dec), *nul) == -1
+    full = _cfg(hga, q_begin=4095, q_len=1)  # resident windows are required
+    assert L.hga_decode_step_tiered(by(full), *args) == -8
+    mid = _cfg(hga, q_begin=2000, q_len=1, kv_layout=hga.HGA_KV_WINDOWS)  # not the last token
+    assert L.hga_decode_step_tiered(by(mid), *args) == -8
+
+
 def test_status_strings(hga):
     for code, name in hga.STATUS.items():
         assert hga.library().hga_status_string(code).decode().startswith(name)

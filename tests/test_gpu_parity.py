@@ -271,7 +271,21 @@ def test_tiered_decode_4x64k():
                     v_src=v_host, src_is_host=True)
     assert hga.get_device_error() == 0
     worst = _decode_compare(w, x, r, out, rb, cs, gs)
-    print(f"tiered decode: max abs error {worst:.3e}")
+    # the same step in one launch (hga_decode_step_tiered): routed groups read
+    # from the host store inside the attention kernel, nothing gathered
+    rb_f = pipeline.alloc_route(cfg)
+    out_f = torch.full_like(q_rot, float("nan"))
+    pipeline.decode_tiered(cfg_w, q_rot, cs, gs, k_win, v_win, k_host, v_host, rb_f, out_f)
+    torch.cuda.synchronize()
+    assert hga.get_device_error() == 0
+    for name in ("qbar", "sel_chunks", "n_sel_chunks", "sel_groups", "n_sel_groups"):
+        assert torch.equal(getattr(rb_f, name), getattr(rb, name)), name
+    rb_f.chunk_scores, rb_f.group_scores = rb.chunk_scores, rb.group_scores
+    worst_f = _decode_compare(w, x, r, out_f, rb_f, cs, gs)
+    diff = (out_f.float() - out.float()).abs().max().item()
+    assert diff <= 1e-2, diff
+    print(f"tiered decode: max abs error {worst:.3e}; one launch {worst_f:.3e} "
+          f"(vs three launches {diff:.3e})")
 
 
 def test_incremental_summaries_bitwise():
