@@ -45,6 +45,9 @@
  *     oracle rounds its own rotated keys/queries to bf16 (nearest-even) when
  *     asked, and computes everything else in double.
  *   - causal rule: a query at position p sees keys at positions <= p.
+ *   - FP8 K/V caches (the FP8 deployment the pages motivate the method with,
+ *     "Probleemstelling"): each cache entry is an E4M3 code times a per-tensor
+ *     scale; attention runs on those decoded values exactly as on any other.
  *
  * Parity unpinned: the pairing, the representative position and the routing
  * query's aggregation are choices the pages cannot decide, so no test pins
@@ -109,6 +112,29 @@ double hgaref_round_bf16(double x) {
 /* out[i] = hgaref_round_bf16(in[i]) for i < n (bf16 summary tables). */
 void hgaref_round_bf16_n(const double* in, double* out, int64_t n) {
     for (int64_t i = 0; i < n; ++i) out[i] = hgaref_round_bf16(in[i]);
+}
+
+/* Value of one 8-bit floating-point code of the E4M3 kind (the FP8 format of
+ * FP8 K/V caches): bit 7 the sign, bits 6..3 the exponent e with bias 7, bits
+ * 2..0 the mantissa m. e = 0 is subnormal, (m / 8) * 2^-6; otherwise
+ * (1 + m / 8) * 2^(e - 7). The one all-ones pattern below the sign (e = 15,
+ * m = 7) is NaN; there are no infinities, so the largest finite value is
+ * 1.75 * 2^8 = 448. */
+double hgaref_e4m3_value(uint8_t code) {
+    int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        mag = ldexp((double)m / 8.0, -6);
+    else
+        mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+/* out[i] = hgaref_e4m3_value(codes[i]) * scale for i < n: an FP8 K or V
+ * cache entry with its per-tensor scale, as the attention reads it. */
+void hgaref_e4m3_decode_n(const uint8_t* codes, int64_t n, double scale, double* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = hgaref_e4m3_value(codes[i]) * scale;
 }
 
 /* Rotate rows x[n_tok][n_heads][d] where token t sits at position pos0 + t.

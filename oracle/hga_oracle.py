@@ -60,6 +60,8 @@ def lib():
             sig = {
                 "hgaref_round_bf16": (ctypes.c_double, [ctypes.c_double]),
                 "hgaref_round_bf16_n": (None, [_P, _P, ctypes.c_int64]),
+                "hgaref_e4m3_value": (ctypes.c_double, [ctypes.c_uint8]),
+                "hgaref_e4m3_decode_n": (None, [_P, ctypes.c_int64, ctypes.c_double, _P]),
                 "hgaref_rope": (None, [_P, _P, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
                                        ctypes.c_int, _P]),
                 "hgaref_build_summaries": (None, [_P, _P, _P, _P]),
@@ -129,6 +131,20 @@ def round_bf16_array(a) -> np.ndarray:
     a = np.ascontiguousarray(a, dtype=np.float64)
     out = np.empty_like(a)
     lib().hgaref_round_bf16_n(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+def e4m3_value(code: int) -> float:
+    """Value of one E4M3 (FP8) code."""
+    return lib().hgaref_e4m3_value(int(code) & 0xFF)
+
+
+def e4m3_decode(codes, scale: float = 1.0) -> np.ndarray:
+    """Every E4M3 code (uint8 array, any shape) decoded and times scale,
+    float64 out: an FP8 K or V cache as the attention reads it."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, dtype=np.float64)
+    lib().hgaref_e4m3_decode_n(_ptr(c), c.size, float(scale), _ptr(out))
     return out
 
 

@@ -101,6 +101,38 @@ def test_round_bf16_array_matches_scalar_and_torch_cast():
     np.testing.assert_array_equal(O.round_bf16_array(x32), want)
 
 
+def test_e4m3_every_code_matches_torch_float8_cast():
+    """All 256 E4M3 codes decode to the values of torch's float8_e4m3fn type
+    (NaN where torch has NaN)."""
+    codes = np.arange(256, dtype=np.uint8)
+    want = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    got = O.e4m3_decode(codes)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    np.testing.assert_array_equal(got[ok], want[ok])
+    np.testing.assert_array_equal(np.signbit(got[ok]), np.signbit(want[ok]))
+
+
+def test_e4m3_closed_forms():
+    """Values fixed by the format's definition: one, the largest finite value,
+    the smallest normal and subnormal, signed zero, NaN; positive codes are
+    strictly increasing; the scale multiplies every value."""
+    assert O.e4m3_value(0x38) == 1.0
+    assert O.e4m3_value(0xB8) == -1.0
+    assert O.e4m3_value(0x7E) == 448.0
+    assert O.e4m3_value(0x08) == 2.0 ** -6
+    assert O.e4m3_value(0x01) == 2.0 ** -9
+    assert O.e4m3_value(0x07) == 7 * 2.0 ** -9
+    assert O.e4m3_value(0x3C) == 1.5
+    z = O.e4m3_value(0x80)
+    assert z == 0.0 and np.signbit(z)
+    assert np.isnan(O.e4m3_value(0x7F)) and np.isnan(O.e4m3_value(0xFF))
+    pos = O.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    assert np.all(np.diff(pos) > 0)
+    np.testing.assert_array_equal(O.e4m3_decode(np.arange(0x7F, dtype=np.uint8), 0.375),
+                                  pos * 0.375)
+
+
 # ----------------------------------------------------------- summaries ---
 
 def _k(cfg, seed=4):
