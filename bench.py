@@ -37,8 +37,10 @@ TC_TRAFFIC_BYTES = 2 * 574.3e6
 TC_TRAFFIC_NOTE = ("ncu dram__bytes_read+write of attend_tc_kernel at 32K context x2 "
                    "(profiles/attend_tc_prefill_32k_ncu.md)")
 PREFILL = "prefill_64k"
-# ":bf16sum" = the same workload with bf16 summary tables
-DECODES = ("decode_16x32k", "decode_16x32k:bf16sum", "tiered_decode_4x64k")
+# ":bf16sum" = the same workload with bf16 summary tables; ":fp8kv" = with an
+# FP8 (E4M3) key/value cache
+DECODES = ("decode_16x32k", "decode_16x32k:bf16sum", "decode_16x32k:fp8kv",
+           "tiered_decode_4x64k")
 
 
 def load_peaks():
@@ -255,6 +257,8 @@ def run_decode(name, args, dist):
     base, _, variant = name.partition(":")
     w = synth.WORKLOADS[base]
     bf16_sum = variant == "bf16sum"
+    fp8_kv = variant == "fp8kv"
+    kv_es = 1 if fp8_kv else 2  # bytes per K/V element
     cfg = hga.config_from(w, summary_type=hga.HGA_SUMMARY_BF16 if bf16_sum else hga.HGA_SUMMARY_F32)
     x = synth.draw(w, seed=dist.seed(args.seed))
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -294,6 +298,11 @@ def run_decode(name, args, dist):
         launches, launches_sep = 1, 3
     else:
         v = x["v"].to(dev)
+        if fp8_kv:  # the cache stored as E4M3 codes with a per-tensor scale each
+            k_rot, ks = synth.to_e4m3(k_rot)
+            v, vs = synth.to_e4m3(v)
+            cfg = cfg.copy(kv_type=hga.HGA_KV_E4M3, k_scale=ks, v_scale=vs)
+            gat = pipeline.alloc_gathered(cfg, dev)
 
         def step_fn(separate=False, warm=False):
             pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out, separate=separate)
@@ -360,11 +369,11 @@ def run_decode(name, args, dist):
         warm_info["drifting"] = run_warm_drift(w, args, dist, cfg, cfg_w, cs, gs, k_win, v_win,
                                                k_host, v_host, st)
     n_sel = rb.n_sel_groups.cpu().numpy()
-    moved = int(n_sel.sum()) * 16 * w.head_dim * 2 * 2  # routed K+V bytes
+    moved = int(n_sel.sum()) * 16 * w.head_dim * kv_es * 2  # routed K+V bytes
     recall = planted_recall(w, x["planted"], rb.sel_chunks.cpu().numpy(),
                             rb.n_sel_chunks.cpu().numpy())
     gather_info = None
-    if not w.tiered and not bf16_sum:
+    if not w.tiered and not variant:
         # the exact-token gather from HBM alone (hga_gather_kv): (1) one launch
         # replayed from a CUDA graph after an L2 flush (includes the graph's
         # launch latency); (2) launches back to back, cycling through the
@@ -408,7 +417,7 @@ def run_decode(name, args, dist):
                            launches=1)
     # algorithmic HBM bytes of one step (each byte the step must touch, once)
     n_forced_tok = (min(w.n_sink, w.n_chunks) + w.n_local + 1) * w.chunk_size
-    forced_kv = w.batch * w.n_kv_heads * n_forced_tok * w.head_dim * 2 * 2
+    forced_kv = w.batch * w.n_kv_heads * n_forced_tok * w.head_dim * kv_es * 2
     se = 2 if bf16_sum else 4  # summary element bytes
     chunk_sums = w.batch * w.n_kv_heads * w.n_chunks * w.head_dim * se
     group_sums = int(rb.n_sel_chunks.cpu().numpy().sum()) * w.groups_per_chunk * w.head_dim * se
@@ -416,7 +425,8 @@ def run_decode(name, args, dist):
     # tiered: the one-launch step reads the routed groups from the host, not
     # from HBM (the three-launch path also writes and reads them in a buffer)
     hbm_bytes = forced_kv + chunk_sums + group_sums + q_o + (0 if w.tiered else moved)
-    return dict(workload=name, summary_tables="bf16" if bf16_sum else "fp32", us_per_step=us, us_min=float(np.min(times)), steps=K,
+    return dict(workload=name, summary_tables="bf16" if bf16_sum else "fp32",
+                kv_cache="e4m3" if fp8_kv else "bf16", us_per_step=us, us_min=float(np.min(times)), steps=K,
                 hbm_bytes_per_step=hbm_bytes, hbm_gbs=hbm_bytes / (us * 1e-6) / 1e9,
                 hbm_frac=hbm_bytes / (us * 1e-6) / 1e9 / load_peaks()["hbm"],
                 us_per_step_eager=eager_us, cuda_graph=True,

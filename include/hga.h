@@ -108,6 +108,27 @@ typedef enum { HGA_KV_FULL = 0, HGA_KV_WINDOWS = 1 } hga_kv_layout;
  *                   HGA_ERR_UNSUPPORTED for it. */
 typedef enum { HGA_SUMMARY_F32 = 0, HGA_SUMMARY_BF16 = 1 } hga_summary_type;
 
+/* Storage type of the attention keys and values: the stores (k_res / v_res,
+ * k_cache / v_cache, k_win / v_win, k_src / v_src, k_host / v_host), the
+ * gathered buffers and the warm-tier pools.
+ * HGA_KV_AS_DTYPE: cfg->dtype, like the queries.
+ * HGA_KV_E4M3:     one byte per element, an 8-bit floating-point code of the
+ *                  E4M3 kind (bit 7 sign, bits 6..3 exponent with bias 7,
+ *                  bits 2..0 mantissa; no infinities; 0x7F / 0xFF are NaN):
+ *                  the FP8 K/V cache of an FP8 deployment (the setting of
+ *                  "Probleemstelling"). An element's value is its code's
+ *                  value times cfg->k_scale (keys) or cfg->v_scale (values);
+ *                  layouts are the same, with 1-byte elements. Needs dtype
+ *                  HGA_BF16 and head_dim 128; queries must lie in the fp16
+ *                  range (|q| < 65504: the products run on fp16 tensor-core
+ *                  inputs, which hold every E4M3 value exactly). Read by the
+ *                  decode calls (hga_attend with q_len == 1, hga_decode_step,
+ *                  hga_decode_step_tiered) and moved by the gathers
+ *                  (hga_gather_kv, hga_gather_kv_warm[_noalloc]). Prefill
+ *                  attention (q_len > 1) and a rotated-key output of
+ *                  hga_build_summaries return HGA_ERR_UNSUPPORTED. */
+typedef enum { HGA_KV_AS_DTYPE = 0, HGA_KV_E4M3 = 1 } hga_kv_type;
+
 typedef struct {
     int32_t batch;             /* B */
     int32_t seq_len;           /* L: tokens in the K/V history (context length) */
@@ -127,6 +148,9 @@ typedef struct {
     int32_t q_len;             /* number of query tokens (1 = decode) */
     int32_t kv_layout;         /* hga_kv_layout, read by hga_attend only */
     int32_t summary_type;      /* hga_summary_type of the summary tables (0 = fp32) */
+    int32_t kv_type;           /* hga_kv_type of keys and values (0 = cfg->dtype) */
+    float k_scale;             /* HGA_KV_E4M3: scale of the key codes (finite, > 0) */
+    float v_scale;             /* HGA_KV_E4M3: scale of the value codes (finite, > 0) */
 } hga_config;
 
 /* Rotate x by RoPE (standard rotary position embedding; the summaries of

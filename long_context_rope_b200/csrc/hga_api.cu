@@ -97,6 +97,13 @@ hga_status make_params(const hga_config* c, Params* p) {
     if (c->kv_layout != HGA_KV_FULL && c->kv_layout != HGA_KV_WINDOWS) return HGA_ERR_CONFIG;
     if (c->summary_type != HGA_SUMMARY_F32 && c->summary_type != HGA_SUMMARY_BF16)
         return HGA_ERR_CONFIG;
+    if (c->kv_type != HGA_KV_AS_DTYPE && c->kv_type != HGA_KV_E4M3) return HGA_ERR_CONFIG;
+    if (c->kv_type == HGA_KV_E4M3) {
+        if (!(c->k_scale > 0.0f) || !isfinite(c->k_scale) || !(c->v_scale > 0.0f) ||
+            !isfinite(c->v_scale))
+            return HGA_ERR_CONFIG;
+        if (c->dtype != HGA_BF16 || c->head_dim != 128) return HGA_ERR_UNSUPPORTED;
+    }
     if (c->q_begin < 0 || c->q_len < 0 || (int64_t)c->q_begin + c->q_len > c->seq_len)
         return HGA_ERR_SHAPE;
     const int64_t nC = ((int64_t)c->seq_len + c->chunk_size - 1) / c->chunk_size;
@@ -124,6 +131,10 @@ hga_status make_params(const hga_config* c, Params* p) {
     p->dtype = c->dtype;
     p->kv_layout = c->kv_layout;
     p->sum_bf16 = c->summary_type == HGA_SUMMARY_BF16 ? 1 : 0;
+    p->kv_f8 = c->kv_type == HGA_KV_E4M3 ? 1 : 0;
+    p->kv_es = p->kv_f8 ? 1 : (c->dtype == HGA_BF16 ? 2 : 4);
+    p->k_scale = p->kv_f8 ? c->k_scale : 1.0f;
+    p->v_scale = p->kv_f8 ? c->v_scale : 1.0f;
     for (int i = 0; i < kMaxHalfDim; ++i)
         p->inv_freq[i] = i < c->head_dim / 2
                              ? pow(c->rope_theta, -2.0 * (double)i / (double)c->head_dim)
@@ -174,13 +185,15 @@ cudaError_t set_func_attr_once(const void* fn, cudaFuncAttribute attr, int value
 
 using namespace hga;
 
-static_assert(sizeof(hga_config) == 80, "hga_config layout is part of the ABI");
+static_assert(sizeof(hga_config) == 88, "hga_config layout is part of the ABI");
 static_assert(offsetof(hga_config, summary_type) == 72, "hga_config layout is part of the ABI");
+static_assert(offsetof(hga_config, kv_type) == 76, "hga_config layout is part of the ABI");
+static_assert(offsetof(hga_config, v_scale) == 84, "hga_config layout is part of the ABI");
 static_assert(offsetof(hga_config, rope_theta) == 48, "hga_config layout is part of the ABI");
 
 extern "C" {
 
-int32_t hga_version(void) { return 10600; }
+int32_t hga_version(void) { return 10700; }
 
 void hga_set_wait_limit_ns(uint64_t limit_ns) {
     g_wait_ns.store(limit_ns == 0 ? 1000000000ull : (unsigned long long)limit_ns,
@@ -233,6 +246,7 @@ hga_status hga_build_summaries(const hga_config* cfg, const void* k_raw, void* c
     if (!aligned16(k_raw) || !aligned16(chunk_sum) || !aligned16(group_sum) ||
         (k_rot_out && !aligned16(k_rot_out)))
         return HGA_ERR_ALIGN;
+    if (k_rot_out && p.kv_f8) return HGA_ERR_UNSUPPORTED;  // rotated keys are written in dtype
     HGA_ATTACH_ERR(p);
     return launched(launch_summaries(p, k_raw, chunk_sum, group_sum, k_rot_out, chunk_begin,
                                      chunk_end, (cudaStream_t)stream));
@@ -353,10 +367,13 @@ hga_status hga_decode_step(const hga_config* cfg, const void* q_rot, const void*
         return launched(launch_decode_step(p, q_rot, chunk_sum, group_sum, k_cache, v_cache,
                                            qbar_out, sel_chunks, n_sel_chunks, sel_groups,
                                            n_sel_groups, out, st));
+    if (p.kv_f8 && !decode_kernel_supports(p)) return HGA_ERR_UNSUPPORTED;
     s = route_separate(p, q_rot, chunk_sum, group_sum, qbar_out, sel_chunks, n_sel_chunks,
                        sel_groups, n_sel_groups, st);
     if (s != HGA_OK) return s;
     KvSources kv{k_cache, v_cache, nullptr, nullptr};
+    if (p.kv_f8)
+        return launched(launch_attend_decode(p, q_rot, kv, sel_groups, n_sel_groups, out, st));
     if (tc_kernel_supports(p, false))
         return launched(launch_attend_tc(p, q_rot, kv, sel_groups, n_sel_groups, out, st));
     if (decode_kernel_supports(p))
@@ -512,9 +529,12 @@ hga_status hga_attend(const hga_config* cfg, const void* q_rot, const void* k_re
     if (p.kv_layout == HGA_KV_WINDOWS &&
         (p.q_len != 1 || p.q_begin != p.L - 1 || k_gat == nullptr))
         return HGA_ERR_UNSUPPORTED;
+    if (p.kv_f8 && !decode_kernel_supports(p)) return HGA_ERR_UNSUPPORTED;  // decode only
     HGA_ATTACH_ERR(p);
     KvSources kv{k_res, v_res, k_gat, v_gat};
     cudaStream_t st = (cudaStream_t)stream;
+    if (p.kv_f8)
+        return launched(launch_attend_decode(p, q_rot, kv, sel_groups, n_sel_groups, out, st));
     if (tc_kernel_supports(p, k_gat != nullptr))
         return launched(launch_attend_tc(p, q_rot, kv, sel_groups, n_sel_groups, out, st));
     if (decode_kernel_supports(p))

@@ -6,6 +6,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -24,6 +25,9 @@ struct Params {
     int nC, q_begin, q_len, j0, nQC;
     int dtype, kv_layout;
     int sum_bf16;                  // summary tables stored as bf16 (else fp32)
+    int kv_f8;                     // K/V stored as E4M3 codes (else dtype)
+    int kv_es;                     // bytes per K/V element
+    float k_scale, v_scale;        // E4M3 code scales (1 otherwise)
     int* err;                      // device error word, never NULL
     unsigned long long wait_ns;    // limit of each bounded device wait
     double inv_freq[kMaxHalfDim];  // rope_theta^(-2i/d), computed on the host in double

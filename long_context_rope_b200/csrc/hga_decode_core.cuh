@@ -13,6 +13,21 @@
 // accumulate) with a per-warp online softmax in fp32. Partials (max, sum, O)
 // merge first across the warps of a CTA, then across the CTAs of the cluster
 // through distributed shared memory.
+//
+// FP8 (E4M3) keys and values: a 16-row block is 2 KiB per tensor (one
+// 128-byte swizzled panel). The products run on fp16 MMA (m16n8k16, fp32
+// accumulate): every E4M3 value converts to fp16 exactly, two codes per
+// convert instruction; the scales multiply the scores (k_scale) and the
+// normalised output (v_scale). Shared-memory reads are 8-byte loads; the
+// MMA's k and m indices are permuted so that each lane's bytes are
+// contiguous:
+//   S = K Q^T   step kk = 2j + e of the head dimension: logical k 2t4 + {0,1}
+//               is dim 32j + 8t4 + 4e + {0,1}, logical 2t4 + 8 + {0,1} is
+//               dim 32j + 8t4 + 4e + {2,3} (queries permuted the same way);
+//   O^T += V^T P^T  tile mt, output row g is dim 8g + mt and row g + 8 is
+//               dim 64 + 8g + mt.
+// Both are bijections of the 128 dims, so the results are the same dot
+// products and output dims, in another summation order.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -27,7 +42,8 @@ namespace cg = cooperative_groups;
 
 constexpr int kD = 128;
 constexpr int kStages = 8;                       // ring of key blocks
-constexpr int kBlkBytes = kGroupRows * kD * 2;   // 4 KiB per block per tensor
+constexpr int kBlkBytes = kGroupRows * kD * 2;   // 4 KiB per block per tensor (bf16)
+constexpr int kBlkBytesF8 = kGroupRows * kD;     // 2 KiB per block per tensor (E4M3)
 constexpr int kConsumers = 8;                    // consumer warps
 constexpr int kThreads = (kConsumers + 1) * 32;  // + one producer warp
 constexpr int kMaxCluster = 16;
@@ -52,19 +68,48 @@ struct WarpAcc {
     float m[2], l[2];
 };
 
-// Q^T as MMA B fragments: lane (g, t4) holds Q[head g][16kk + 2t4 .. +1] and
-// Q[head g][16kk + 2t4 + 8 .. +9]; heads >= gq are zero.
+// Q^T as MMA B fragments; heads >= gq are zero. bf16: lane (g, t4) holds
+// Q[head g][16kk + 2t4 .. +1] and Q[head g][16kk + 2t4 + 8 .. +9]. E4M3 path:
+// fp16 pairs of dims 32j + 8t4 + {0,1}, {2,3} (step 2j) and {4,5}, {6,7}
+// (step 2j + 1), the permutation the key fragments use.
+template <bool kF8>
 __device__ __forceinline__ void load_q_frags(const Params& p, const __nv_bfloat16* q, int b, int h,
                                              uint32_t (&qf)[8][2]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
     const bool okh = g < p.gq;
     const __nv_bfloat16* qr =
         q + ((int64_t)b * p.q_len * p.Hq + (int64_t)h * p.gq + (okh ? g : 0)) * kD;
+    if constexpr (kF8) {
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-        qf[kk][0] = okh ? *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 2 * t4) : 0u;
-        qf[kk][1] = okh ? *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 2 * t4 + 8) : 0u;
+        for (int j = 0; j < 4; ++j) {
+            const uint4 raw = okh ? *reinterpret_cast<const uint4*>(qr + 32 * j + 8 * t4)
+                                  : make_uint4(0u, 0u, 0u, 0u);
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+            uint32_t f[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 v = __bfloat1622float2(h2[e]);
+                const __half2 hv = __floats2half2_rn(v.x, v.y);
+                f[e] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
+            qf[2 * j][0] = f[0];
+            qf[2 * j][1] = f[1];
+            qf[2 * j + 1][0] = f[2];
+            qf[2 * j + 1][1] = f[3];
+        }
+    } else {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            qf[kk][0] = okh ? *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 2 * t4) : 0u;
+            qf[kk][1] = okh ? *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 2 * t4 + 8) : 0u;
+        }
     }
+}
+
+// E4M3 path: the 16-bit word whose low byte is byte m of a and whose high
+// byte is byte m of b (m = 0..3).
+__device__ __forceinline__ uint16_t byte_pair(uint32_t a, uint32_t b, int m) {
+    return (uint16_t)__byte_perm(a, b, (unsigned)(m | ((m + 4) << 4)));
 }
 
 __device__ __forceinline__ void acc_init(WarpAcc& a) {
@@ -77,16 +122,18 @@ __device__ __forceinline__ void acc_init(WarpAcc& a) {
 }
 
 // Consumer warp `warp` processes local blocks warp, warp + 8, ... < nloc of
-// the ring. blk_pos[i] is the position of block i's first token. Returns
-// false (and sets *bad) if a wait gave up.
+// the ring. blk_pos[i] is the position of block i's first token. pt is the
+// warp's 8 x 16 transpose buffer of P (bf16, or fp16 on the E4M3 path, as
+// bits). Returns false (and sets *bad) if a wait gave up.
+template <bool kF8>
 __device__ __forceinline__ bool consume_blocks(const Params& p, const uint32_t (&qf)[8][2],
                                                Ring& ring, uint64_t* full, uint64_t* empty,
                                                const int* blk_pos, int nloc, int qpos,
-                                               __nv_bfloat16 (*pt)[16], WarpAcc& acc,
-                                               int* bad) {
+                                               uint16_t (*pt)[16], WarpAcc& acc, int* bad) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t4 = lane & 3;
-    const float sc = 1.4426950408889634f / sqrtf((float)kD);
+    const float sc0 = 1.4426950408889634f / sqrtf((float)kD);
+    const float sc = kF8 ? sc0 * p.k_scale : sc0;
     const int mq = lane >> 3;
     const int krow = (mq & 1) * 8 + (lane & 7);      // K ldmatrix row
     const int vkey = (mq >> 1) * 8 + (lane & 7);     // V ldmatrix (trans) row
@@ -103,13 +150,35 @@ __device__ __forceinline__ bool consume_blocks(const Params& p, const uint32_t (
         }
         // S^T = K Q^T for 16 keys x 8 heads (two accumulator chains)
         float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sacc2[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint32_t kb = ptx::smem_u32(ring.k[s]);
+        if constexpr (kF8) {
+            // rows g and g + 8, dims 32j + 8t4 .. +7: 16-byte chunk 2j + t4/2
+            // of the row, XOR-swizzled by the row (g and g + 8 alike)
+            const uint8_t* kb = ring.k[s];
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const int chunk = (kk & 3) * 2 + (mq >> 1);
-            uint32_t a[4];
-            ptx::ldsm_x4(kb + (kk >> 2) * 2048 + krow * 128 + ((chunk ^ (krow & 7)) << 4), a);
-            ptx::mma_16816((kk & 1) ? sacc2 : sacc, a, qf[kk][0], qf[kk][1]);
+            for (int j = 0; j < 4; ++j) {
+                const int off = (((2 * j + (t4 >> 1)) ^ g) << 4) + (t4 & 1) * 8;
+                const uint2 w0 = *reinterpret_cast<const uint2*>(kb + g * 128 + off);
+                const uint2 w1 = *reinterpret_cast<const uint2*>(kb + (g + 8) * 128 + off);
+                uint32_t a[4] = {ptx::e4m3x2_to_f16x2((uint16_t)w0.x),
+                                 ptx::e4m3x2_to_f16x2((uint16_t)w1.x),
+                                 ptx::e4m3x2_to_f16x2((uint16_t)(w0.x >> 16)),
+                                 ptx::e4m3x2_to_f16x2((uint16_t)(w1.x >> 16))};
+                ptx::mma_16816_f16(sacc, a, qf[2 * j][0], qf[2 * j][1]);
+                uint32_t a2[4] = {ptx::e4m3x2_to_f16x2((uint16_t)w0.y),
+                                  ptx::e4m3x2_to_f16x2((uint16_t)w1.y),
+                                  ptx::e4m3x2_to_f16x2((uint16_t)(w0.y >> 16)),
+                                  ptx::e4m3x2_to_f16x2((uint16_t)(w1.y >> 16))};
+                ptx::mma_16816_f16(sacc2, a2, qf[2 * j + 1][0], qf[2 * j + 1][1]);
+            }
+        } else {
+            const uint32_t kb = ptx::smem_u32(ring.k[s]);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int chunk = (kk & 3) * 2 + (mq >> 1);
+                uint32_t a[4];
+                ptx::ldsm_x4(kb + (kk >> 2) * 2048 + krow * 128 + ((chunk ^ (krow & 7)) << 4), a);
+                ptx::mma_16816((kk & 1) ? sacc2 : sacc, a, qf[kk][0], qf[kk][1]);
+            }
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) sacc[e] += sacc2[e];
@@ -132,10 +201,24 @@ __device__ __forceinline__ bool consume_blocks(const Params& p, const uint32_t (
                 p1 = ptx::ex2_approx(sv[hh + 2] - mn);
             }
             acc.m[hh] = mn;
-            // bf16 weights; the running sum uses the same rounded values
-            const __nv_bfloat16 b0 = __float2bfloat16_rn(p0);
-            const __nv_bfloat16 b1 = __float2bfloat16_rn(p1);
-            acc.l[hh] = acc.l[hh] * alpha + __bfloat162float(b0) + __bfloat162float(b1);
+            // bf16 weights (fp16 on the E4M3 path); the running sum uses the
+            // same rounded values
+            uint16_t b0, b1;
+            float r0, r1;
+            if constexpr (kF8) {
+                const __half h0 = __float2half_rn(p0), h1 = __float2half_rn(p1);
+                b0 = __half_as_ushort(h0);
+                b1 = __half_as_ushort(h1);
+                r0 = __half2float(h0);
+                r1 = __half2float(h1);
+            } else {
+                const __nv_bfloat16 h0 = __float2bfloat16_rn(p0), h1 = __float2bfloat16_rn(p1);
+                b0 = __bfloat16_as_ushort(h0);
+                b1 = __bfloat16_as_ushort(h1);
+                r0 = __bfloat162float(h0);
+                r1 = __bfloat162float(h1);
+            }
+            acc.l[hh] = acc.l[hh] * alpha + r0 + r1;
             pt[2 * t4 + hh][g] = b0;
             pt[2 * t4 + hh][g + 8] = b1;
 #pragma unroll
@@ -148,14 +231,40 @@ __device__ __forceinline__ bool consume_blocks(const Params& p, const uint32_t (
         const uint32_t pb0 = *reinterpret_cast<const uint32_t*>(&pt[g][2 * t4]);
         const uint32_t pb1 = *reinterpret_cast<const uint32_t*>(&pt[g][2 * t4 + 8]);
         // O^T[16 dims x 8 heads] += V^T P^T, eight 16-dim tiles
-        const uint32_t vb = ptx::smem_u32(ring.v[s]);
+        if constexpr (kF8) {
+            // keys 2t4, 2t4 + 1, 2t4 + 8, 2t4 + 9; dims 8g .. +7 (rows g of
+            // the tiles) and 64 + 8g .. +7 (rows g + 8): 16-byte chunk g/2
+            // (or 4 + g/2) of the key's row, XOR-swizzled by the key
+            const uint8_t* vb = ring.v[s];
+            auto ldv = [&](int key, int hi) {
+                const int off = (((hi * 4 + (g >> 1)) ^ (key & 7)) << 4) + (g & 1) * 8;
+                return *reinterpret_cast<const uint2*>(vb + key * 128 + off);
+            };
+            const uint2 v0l = ldv(2 * t4, 0), v1l = ldv(2 * t4 + 1, 0);
+            const uint2 v0h = ldv(2 * t4, 1), v1h = ldv(2 * t4 + 1, 1);
+            const uint2 v8l = ldv(2 * t4 + 8, 0), v9l = ldv(2 * t4 + 9, 0);
+            const uint2 v8h = ldv(2 * t4 + 8, 1), v9h = ldv(2 * t4 + 9, 1);
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            const int chunk = (mt & 3) * 2 + (mq & 1);
-            uint32_t a[4];
-            ptx::ldsm_x4_trans(vb + (mt >> 2) * 2048 + vkey * 128 + ((chunk ^ (vkey & 7)) << 4),
-                               a);
-            ptx::mma_16816(acc.o[mt], a, pb0, pb1);
+            for (int mt = 0; mt < 8; ++mt) {
+                const int m = mt & 3;
+                const bool y = mt >= 4;
+                uint32_t a[4] = {
+                    ptx::e4m3x2_to_f16x2(byte_pair(y ? v0l.y : v0l.x, y ? v1l.y : v1l.x, m)),
+                    ptx::e4m3x2_to_f16x2(byte_pair(y ? v0h.y : v0h.x, y ? v1h.y : v1h.x, m)),
+                    ptx::e4m3x2_to_f16x2(byte_pair(y ? v8l.y : v8l.x, y ? v9l.y : v9l.x, m)),
+                    ptx::e4m3x2_to_f16x2(byte_pair(y ? v8h.y : v8h.x, y ? v9h.y : v9h.x, m))};
+                ptx::mma_16816_f16(acc.o[mt], a, pb0, pb1);
+            }
+        } else {
+            const uint32_t vb = ptx::smem_u32(ring.v[s]);
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                const int chunk = (mt & 3) * 2 + (mq & 1);
+                uint32_t a[4];
+                ptx::ldsm_x4_trans(vb + (mt >> 2) * 2048 + vkey * 128 + ((chunk ^ (vkey & 7)) << 4),
+                                   a);
+                ptx::mma_16816(acc.o[mt], a, pb0, pb1);
+            }
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&empty[s]);
@@ -163,7 +272,10 @@ __device__ __forceinline__ bool consume_blocks(const Params& p, const uint32_t (
     return true;
 }
 
-// Consumer warp writes its partial (row max, row sum, O) to wp.
+// Consumer warp writes its partial (row max, row sum, O) to wp. Accumulator
+// tile mt holds dims mt * 16 + {g, g + 8} (bf16 path) or 8g + mt and
+// 64 + 8g + mt (E4M3 path).
+template <bool kF8>
 __device__ __forceinline__ void store_warp_partial(const WarpAcc& acc, Partial& wp) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
     float lsum[2];
@@ -183,11 +295,12 @@ __device__ __forceinline__ void store_warp_partial(const WarpAcc& acc, Partial& 
     }
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-        const int d0 = mt * 16 + g;
+        const int d0 = kF8 ? 8 * g + mt : mt * 16 + g;
+        const int d1 = kF8 ? 64 + 8 * g + mt : d0 + 8;
         wp.o[2 * t4][d0] = acc.o[mt][0];
         wp.o[2 * t4 + 1][d0] = acc.o[mt][1];
-        wp.o[2 * t4][d0 + 8] = acc.o[mt][2];
-        wp.o[2 * t4 + 1][d0 + 8] = acc.o[mt][3];
+        wp.o[2 * t4][d1] = acc.o[mt][2];
+        wp.o[2 * t4 + 1][d1] = acc.o[mt][3];
     }
 }
 
@@ -254,22 +367,30 @@ __device__ __forceinline__ void merge_cluster_and_store(const Params& p, cg::clu
                     den = fmaf(wgt, lc[c], den);
                 }
             }
-            const float o = den > 0.f ? num / den : 0.f;
+            float o = den > 0.f ? num / den : 0.f;
+            if (p.kv_f8) o *= p.v_scale;
             out[((int64_t)b * p.q_len * p.Hq + (int64_t)h * p.gq + n) * kD + tid] =
                 __float2bfloat16_rn(o);
         }
     }
 }
 
-// Issue the TMA loads of one 16-row block (K and V, two 64-column halves
-// each) into ring stage s.
+// Issue the TMA loads of one 16-row block into ring stage s: K and V, two
+// 64-column bf16 halves each, or one 128-byte-wide E4M3 panel each.
+template <bool kF8>
 __device__ __forceinline__ void issue_block(Ring& ring, uint64_t* full, int s,
                                             const CUtensorMap* mk, const CUtensorMap* mv, int row,
                                             int outer) {
-    ptx::mbar_arrive_expect_tx(&full[s], 2 * kBlkBytes);
-    for (int hf = 0; hf < 2; ++hf) {
-        ptx::tma_load_3d(ring.k[s] + hf * 2048, mk, hf * 64, row, outer, &full[s]);
-        ptx::tma_load_3d(ring.v[s] + hf * 2048, mv, hf * 64, row, outer, &full[s]);
+    if constexpr (kF8) {
+        ptx::mbar_arrive_expect_tx(&full[s], 2 * kBlkBytesF8);
+        ptx::tma_load_3d(ring.k[s], mk, 0, row, outer, &full[s]);
+        ptx::tma_load_3d(ring.v[s], mv, 0, row, outer, &full[s]);
+    } else {
+        ptx::mbar_arrive_expect_tx(&full[s], 2 * kBlkBytes);
+        for (int hf = 0; hf < 2; ++hf) {
+            ptx::tma_load_3d(ring.k[s] + hf * 2048, mk, hf * 64, row, outer, &full[s]);
+            ptx::tma_load_3d(ring.v[s] + hf * 2048, mv, hf * 64, row, outer, &full[s]);
+        }
     }
 }
 

@@ -15,8 +15,12 @@
 // = K_blk Q^T and O^T[128 dims x 8 heads] += V^T P^T on warp-level bf16 MMA
 // (m16n8k16, fp32 accumulate) with a per-warp online softmax in fp32. The
 // 8 x CL warp partials (max, sum, O) merge through distributed shared memory:
-// CTA r finalises heads r, r + CL, ...
+// CTA r finalises heads r, r + CL, ... With E4M3 keys and values
+// (HGA_KV_E4M3) the blocks are 2 KiB per tensor and the products run on fp16
+// MMA (hga_decode_core.cuh).
 #include <cooperative_groups.h>
+
+#include <mutex>
 
 #include "hga_blocks.cuh"
 #include "hga_decode_core.cuh"
@@ -47,7 +51,7 @@ struct DecodeSmem {
         dec::Partial warp_part[kConsumers];      // reused once the ring is drained
     } u;
     dec::Partial cta_part;
-    __nv_bfloat16 pt[kConsumers][8][16];         // per-warp P transpose buffer
+    uint16_t pt[kConsumers][8][16];              // per-warp P transpose buffer
     uint64_t full[kStages], empty[kStages];
     int blk_row[kMaxBlocks];
     int blk_pos[kMaxBlocks];
@@ -55,6 +59,7 @@ struct DecodeSmem {
     int bad;
 };
 
+template <bool kF8>
 __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
     const __grid_constant__ DecodeMaps maps, Params p, const __nv_bfloat16* __restrict__ q,
     const int32_t* __restrict__ sel, const int32_t* __restrict__ nsel,
@@ -106,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
                 const int rw = sm.blk_row[lo + i];
                 const bool gat = (rw & kSrcGathered) != 0;
                 const int row = rw & ~kSrcGathered;
-                dec::issue_block(sm.u.ring, sm.full, s, gat ? &maps.k_gat : &maps.k_res,
+                dec::issue_block<kF8>(sm.u.ring, sm.full, s, gat ? &maps.k_gat : &maps.k_res,
                                  gat ? &maps.v_gat : &maps.v_res, row, (int)(gat ? prob : bh));
             }
             // every issued load lands before the ring's memory is reused
@@ -122,14 +127,14 @@ __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
     dec::acc_init(acc);
     if (warp < kConsumers) {
         uint32_t qf[8][2];
-        dec::load_q_frags(p, q, b, h, qf);
-        dec::consume_blocks(p, qf, sm.u.ring, sm.full, sm.empty, sm.blk_pos + lo, nloc,
+        dec::load_q_frags<kF8>(p, q, b, h, qf);
+        dec::consume_blocks<kF8>(p, qf, sm.u.ring, sm.full, sm.empty, sm.blk_pos + lo, nloc,
                             p.q_begin, sm.pt[warp], acc, &sm.bad);
     }
     __syncthreads();  // ring drained: every stage a consumer used was waited for
 
     // ---- per-warp partials -> shared memory (the ring's space is reused)
-    if (warp < kConsumers) dec::store_warp_partial(acc, sm.u.warp_part[warp]);
+    if (warp < kConsumers) dec::store_warp_partial<kF8>(acc, sm.u.warp_part[warp]);
     __syncthreads();
     dec::merge_warps(sm.u.warp_part, sm.cta_part);
     cluster.sync();
@@ -137,16 +142,23 @@ __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
     cluster.sync();
 }
 
+std::mutex g_decode_mu;
+// per device and K/V type: clusters of each size resident at once (0 = not
+// queried) and the largest cluster size that co-schedules
+int g_dec_active[kMaxDevicesPerProcess][2][kMaxCluster + 1] = {};
+int g_dec_max_cluster[kMaxDevicesPerProcess][2] = {};
+
 // Cluster size: as many CTAs per (sequence, KV head) as keep every unit's
 // cluster resident at once (one wave), per the occupancy query for clusters.
-int pick_cluster(const Params& p, size_t smem) {
-    static int max_active[kMaxCluster + 1] = {};
-    int sms = 148, dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+template <bool kF8>
+int pick_cluster(const Params& p, size_t smem, int dev) {
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int units = p.B * p.Hkv;
     int cl = 2 * sms / units;  // two CTAs per SM
     cl = cl < 1 ? 1 : (cl > kMaxCluster ? kMaxCluster : cl);
+    std::lock_guard<std::mutex> lock(g_decode_mu);
+    int* max_active = g_dec_active[dev][kF8 ? 1 : 0];
     for (; cl > 1; --cl) {
         if (max_active[cl] == 0) {
             cudaLaunchConfig_t q = {};
@@ -161,7 +173,10 @@ int pick_cluster(const Params& p, size_t smem) {
             q.attrs = a;
             q.numAttrs = 1;
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, attend_decode_kernel, &q) != cudaSuccess) n = -1;
+            if (cudaOccupancyMaxActiveClusters(&n, attend_decode_kernel<kF8>, &q) != cudaSuccess) {
+                cudaGetLastError();
+                n = -1;
+            }
             max_active[cl] = n;
         }
         if (max_active[cl] >= units) break;
@@ -171,51 +186,62 @@ int pick_cluster(const Params& p, size_t smem) {
 
 }  // namespace
 
-cudaError_t launch_attend_decode(const Params& p, const void* q_rot, const KvSources& kv,
-                                 const int32_t* sel_groups, const int32_t* n_sel_groups,
-                                 void* out, cudaStream_t st) {
+namespace {
+
+template <bool kF8>
+cudaError_t launch_decode_t(const Params& p, const void* q_rot, const KvSources& kv,
+                            const int32_t* sel_groups, const int32_t* n_sel_groups, void* out,
+                            cudaStream_t st) {
     DecodeMaps maps;
     const bool gathered = kv.k_gat != nullptr;
     const int64_t res_rows = p.kv_layout == HGA_KV_WINDOWS
                                  ? (int64_t)(p.n_sink + p.n_local + 1) * p.C
                                  : (int64_t)p.L;
     const int64_t BH = (int64_t)p.B * p.Hkv;
-    bool ok = make_rows_map(&maps.k_res, kv.k_res, BH, res_rows, kD, kGroupRows) &&
-              make_rows_map(&maps.v_res, kv.v_res, BH, res_rows, kD, kGroupRows);
+    auto rows_map = [](CUtensorMap* m, const void* base, int64_t outer, int64_t rows) {
+        return kF8 ? make_rows_map_u8(m, base, outer, rows, kD, kGroupRows)
+                   : make_rows_map(m, base, outer, rows, kD, kGroupRows);
+    };
+    bool ok = rows_map(&maps.k_res, kv.k_res, BH, res_rows) &&
+              rows_map(&maps.v_res, kv.v_res, BH, res_rows);
     if (gathered) {
-        ok = ok && make_rows_map(&maps.k_gat, kv.k_gat, BH * p.nQC, (int64_t)p.kg * kGroupRows, kD,
-                                 kGroupRows) &&
-             make_rows_map(&maps.v_gat, kv.v_gat, BH * p.nQC, (int64_t)p.kg * kGroupRows, kD,
-                           kGroupRows);
+        ok = ok && rows_map(&maps.k_gat, kv.k_gat, BH * p.nQC, (int64_t)p.kg * kGroupRows) &&
+             rows_map(&maps.v_gat, kv.v_gat, BH * p.nQC, (int64_t)p.kg * kGroupRows);
     } else {
         maps.k_gat = maps.k_res;
         maps.v_gat = maps.v_res;
     }
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = sizeof(DecodeSmem) + 1024;
-    // largest cluster that co-schedules, per device (queried once)
-    static int max_cluster_of[kMaxDevicesPerProcess];  // 0 = not yet queried
     int dev = 0;
     cudaError_t e = current_device_index(&dev);
     if (e != cudaSuccess) return e;
-    e = set_func_attr_once((const void*)attend_decode_kernel,
+    e = set_func_attr_once((const void*)attend_decode_kernel<kF8>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = set_func_attr_once((const void*)attend_decode_kernel,
+        e = set_func_attr_once((const void*)attend_decode_kernel<kF8>,
                                cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
-    int& max_cluster = max_cluster_of[dev];
-    if (max_cluster <= 0) {
-        cudaLaunchConfig_t q = {};
-        q.gridDim = dim3(kMaxCluster, 1, 1);
-        q.blockDim = dim3(kThreads);
-        q.dynamicSmemBytes = smem;
-        int mc = 0;
-        if (cudaOccupancyMaxPotentialClusterSize(&mc, attend_decode_kernel, &q) != cudaSuccess)
-            return cudaErrorInvalidConfiguration;
-        max_cluster = mc < 1 ? 1 : mc;
+    int max_cluster = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_decode_mu);
+        int& mc_slot = g_dec_max_cluster[dev][kF8 ? 1 : 0];
+        if (mc_slot <= 0) {
+            cudaLaunchConfig_t q = {};
+            q.gridDim = dim3(kMaxCluster, 1, 1);
+            q.blockDim = dim3(kThreads);
+            q.dynamicSmemBytes = smem;
+            int mc = 0;
+            if (cudaOccupancyMaxPotentialClusterSize(&mc, attend_decode_kernel<kF8>, &q) !=
+                cudaSuccess) {
+                cudaGetLastError();
+                return cudaErrorInvalidConfiguration;
+            }
+            mc_slot = mc < 1 ? 1 : mc;
+        }
+        max_cluster = mc_slot;
     }
-    int cl = pick_cluster(p, smem);
+    int cl = pick_cluster<kF8>(p, smem, dev);
     if (cl > max_cluster) cl = max_cluster;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cl, (unsigned)BH, 1);
@@ -230,8 +256,19 @@ cudaError_t launch_attend_decode(const Params& p, const void* q_rot, const KvSou
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const int gflag = gathered ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, attend_decode_kernel, maps, p, (const __nv_bfloat16*)q_rot,
-                              sel_groups, n_sel_groups, (__nv_bfloat16*)out, gflag);
+    return cudaLaunchKernelEx(&cfg, attend_decode_kernel<kF8>, maps, p,
+                              (const __nv_bfloat16*)q_rot, sel_groups, n_sel_groups,
+                              (__nv_bfloat16*)out, gflag);
+}
+
+}  // namespace
+
+cudaError_t launch_attend_decode(const Params& p, const void* q_rot, const KvSources& kv,
+                                 const int32_t* sel_groups, const int32_t* n_sel_groups,
+                                 void* out, cudaStream_t st) {
+    if (p.kv_f8)
+        return launch_decode_t<true>(p, q_rot, kv, sel_groups, n_sel_groups, out, st);
+    return launch_decode_t<false>(p, q_rot, kv, sel_groups, n_sel_groups, out, st);
 }
 
 bool decode_kernel_supports(const Params& p) {

@@ -71,7 +71,7 @@ struct StepSmem {
         dec::Partial warp_part[kConsumers];
     } u;
     dec::Partial cta_part;
-    __nv_bfloat16 pt[kConsumers][8][16];
+    uint16_t pt[kConsumers][8][16];
     uint64_t full[kStages], empty[kStages];
     uint64_t key1[kMaxSlice];     // own level-1 candidates
     uint64_t f1[kMaxF1];          // level-1 finalists of all CTAs
@@ -173,24 +173,27 @@ __device__ __forceinline__ void score_rows(const float* q, int n, RowOf row_of, 
 }
 
 // Producer warp, host tier: the K and V rows of one routed group (16 rows of
-// d = 128 bf16 each, contiguous in the full store) read over the host link
-// with 16-byte loads (each lane 8 of each tensor, 512 contiguous bytes per
-// warp load) and stored into ring stage s in the layout the TMA tile loads
-// write: two 64-column panels of 16 rows x 128 bytes, 16-byte chunk c of
-// row r at c ^ (r % 8).
+// d = 128 elements each, contiguous in the full store) read over the host
+// link with 16-byte loads (each lane 8 (bf16) or 4 (E4M3) of each tensor,
+// 512 contiguous bytes per warp load) and stored into ring stage s in the
+// layout the TMA tile loads write: 128-byte panels of 16 rows (two for bf16,
+// one for E4M3), 16-byte chunk c of row r at c ^ (r % 8).
+template <bool kF8>
 __device__ __forceinline__ void copy_host_block(dec::Ring& ring, int s, const uint4* kh,
                                                 const uint4* vh) {
     const int lane = threadIdx.x & 31;
-    uint4 kr[8], vr[8];
+    constexpr int kPieces = kF8 ? 4 : 8;             // per lane per tensor
+    constexpr int kRowPieces = kF8 ? 8 : 16;         // 16-byte pieces per row
+    uint4 kr[kPieces], vr[kPieces];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < kPieces; ++u) {
         kr[u] = kh[lane + 32 * u];
         vr[u] = vh[lane + 32 * u];
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        const int idx = lane + 32 * u;               // 16-byte piece of the 4 KiB block
-        const int row = idx >> 4, c16 = idx & 15;
+    for (int u = 0; u < kPieces; ++u) {
+        const int idx = lane + 32 * u;               // 16-byte piece of the block
+        const int row = idx / kRowPieces, c16 = idx % kRowPieces;
         const int off = (c16 >> 3) * 2048 + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
         *reinterpret_cast<uint4*>(ring.k[s] + off) = kr[u];
         *reinterpret_cast<uint4*>(ring.v[s] + off) = vr[u];
@@ -201,11 +204,12 @@ __device__ __forceinline__ void copy_host_block(dec::Ring& ring, int s, const ui
 }
 
 // S: element type of the summary tables (float, or bf16 for bf16 tables).
+// kF8: keys and values are E4M3 codes (else bf16).
 // k_host / v_host: nullptr, or the full store [B, Hkv, L, d] in mapped host
 // memory (the host tier); then the maps cover the resident windows of the
 // forced chunks ([B, Hkv, W * C, d]) and the routed groups are read from the
 // host by the producer warp.
-template <typename S>
+template <typename S, bool kF8>
 __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     const __grid_constant__ StepMaps maps, Params p, const __nv_bfloat16* __restrict__ q,
     const S* __restrict__ cs, const S* __restrict__ gs, float* __restrict__ qbar_out,
@@ -257,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     const int n_pre = nf_loc < kStages ? nf_loc : kStages;
     if (attend && warp == kConsumers && lane == 0)
         for (int i = 0; i < n_pre; ++i)
-            dec::issue_block(sm.u.ring, sm.full, i, &maps.k, &maps.v, sm.blk_row[i], (int)bh);
+            dec::issue_block<kF8>(sm.u.ring, sm.full, i, &maps.k, &maps.v, sm.blk_row[i], (int)bh);
 
     // ---- level-1 slice: the first batch of this warp's chunk-summary rows is
     // requested before q-bar, so the two memory latencies overlap
@@ -450,11 +454,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
             }
             if (host_tier && i >= nf_loc) {
                 const int64_t row = bh * (int64_t)p.L + sm.blk_row[i];
-                copy_host_block(sm.u.ring, s, k_host + row * (kD / 8), v_host + row * (kD / 8));
+                constexpr int kRowVecs = kF8 ? kD / 16 : kD / 8;  // 16-byte pieces per row
+                copy_host_block<kF8>(sm.u.ring, s, k_host + row * kRowVecs, v_host + row * kRowVecs);
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&sm.full[s]);
             } else if (lane == 0) {
-                dec::issue_block(sm.u.ring, sm.full, s, &maps.k, &maps.v, sm.blk_row[i], (int)bh);
+                dec::issue_block<kF8>(sm.u.ring, sm.full, s, &maps.k, &maps.v, sm.blk_row[i], (int)bh);
             }
         }
         if (lane == 0) {
@@ -474,12 +479,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     dec::acc_init(acc);
     if (consumer) {
         uint32_t qf[8][2];
-        dec::load_q_frags(p, q, b, h, qf);
-        dec::consume_blocks(p, qf, sm.u.ring, sm.full, sm.empty, sm.blk_pos, nloc, p.q_begin,
+        dec::load_q_frags<kF8>(p, q, b, h, qf);
+        dec::consume_blocks<kF8>(p, qf, sm.u.ring, sm.full, sm.empty, sm.blk_pos, nloc, p.q_begin,
                             sm.pt[warp], acc, &sm.bad);
     }
     __syncthreads();
-    if (consumer) dec::store_warp_partial(acc, sm.u.warp_part[warp]);
+    if (consumer) dec::store_warp_partial<kF8>(acc, sm.u.warp_part[warp]);
     __syncthreads();
     dec::merge_warps(sm.u.warp_part, sm.cta_part);
     cluster.sync();
@@ -499,27 +504,27 @@ bool step_fits(const Params& p, int cl) {
 }
 
 std::mutex g_step_mu;
-// per device and summary type, 0 = not queried
-int g_max_active[kMaxDevicesPerProcess][2][kMaxCluster + 1] = {};
+// per device, summary type and K/V type, 0 = not queried
+int g_max_active[kMaxDevicesPerProcess][2][2][kMaxCluster + 1] = {};
 
-template <typename S>
+template <typename S, bool kF8>
 cudaError_t step_prepare(size_t smem) {
-    cudaError_t e = set_func_attr_once((const void*)decode_step_kernel<S>,
+    cudaError_t e = set_func_attr_once((const void*)decode_step_kernel<S, kF8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = set_func_attr_once((const void*)decode_step_kernel<S>,
+        e = set_func_attr_once((const void*)decode_step_kernel<S, kF8>,
                                cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return e;
 }
 
 // Clusters of `cl` CTAs that can be resident at once on the current device
 // (-1 if the query fails).
-template <typename S>
+template <typename S, bool kF8>
 int active_clusters(int cl, size_t smem) {
     int dev = 0;
     if (current_device_index(&dev) != cudaSuccess) return -1;
     std::lock_guard<std::mutex> lock(g_step_mu);
-    int& slot = g_max_active[dev][sizeof(S) == 2 ? 1 : 0][cl];
+    int& slot = g_max_active[dev][sizeof(S) == 2 ? 1 : 0][kF8 ? 1 : 0][cl];
     if (slot == 0) {
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(cl, 1, 1);
@@ -533,7 +538,7 @@ int active_clusters(int cl, size_t smem) {
         q.attrs = a;
         q.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, decode_step_kernel<S>, &q) != cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&n, decode_step_kernel<S, kF8>, &q) != cudaSuccess) {
             cudaGetLastError();
             n = -1;
         }
@@ -544,7 +549,7 @@ int active_clusters(int cl, size_t smem) {
 
 // Cluster size: two CTAs per SM over the whole grid if the tables fit and the
 // clusters can all be resident at once; else the largest size that fits.
-template <typename S>
+template <typename S, bool kF8>
 int step_cluster(const Params& p, size_t smem) {
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess)
@@ -555,7 +560,7 @@ int step_cluster(const Params& p, size_t smem) {
     for (; cl >= 1; --cl) {
         if (!step_fits(p, cl)) continue;
         if (cl == 1) return 1;
-        const int n = active_clusters<S>(cl, smem);
+        const int n = active_clusters<S, kF8>(cl, smem);
         if (n >= units || (n > 0 && cl <= 2)) return cl;
     }
     return 0;
@@ -574,7 +579,7 @@ bool decode_step_supports(const Params& p) {
 
 namespace {
 
-template <typename S>
+template <typename S, bool kF8>
 cudaError_t launch_step(const Params& p, const void* q_rot, const S* chunk_sum,
                         const S* group_sum, const void* k_cache, const void* v_cache, float* qbar,
                         int32_t* sel_chunks, int32_t* n_sel_chunks, int32_t* sel_groups,
@@ -587,16 +592,18 @@ cudaError_t launch_step(const Params& p, const void* q_rot, const S* chunk_sum,
         const int64_t rows = p.kv_layout == HGA_KV_WINDOWS
                                  ? (int64_t)(p.n_sink + p.n_local + 1) * p.C
                                  : (int64_t)p.L;
-        if (!make_rows_map(&maps.k, k_cache, BH, rows, kD, kGroupRows) ||
-            !make_rows_map(&maps.v, v_cache, BH, rows, kD, kGroupRows))
-            return cudaErrorInvalidValue;
+        const bool ok = kF8 ? make_rows_map_u8(&maps.k, k_cache, BH, rows, kD, kGroupRows) &&
+                                  make_rows_map_u8(&maps.v, v_cache, BH, rows, kD, kGroupRows)
+                            : make_rows_map(&maps.k, k_cache, BH, rows, kD, kGroupRows) &&
+                                  make_rows_map(&maps.v, v_cache, BH, rows, kD, kGroupRows);
+        if (!ok) return cudaErrorInvalidValue;
     } else {
         memset(&maps, 0, sizeof(maps));
     }
     const size_t smem = sizeof(StepSmem) + 1024;
-    cudaError_t e = step_prepare<S>(smem);
+    cudaError_t e = step_prepare<S, kF8>(smem);
     if (e != cudaSuccess) return e;
-    const int cl = step_cluster<S>(p, smem);
+    const int cl = step_cluster<S, kF8>(p, smem);
     if (cl < 1) return cudaErrorInvalidConfiguration;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cl, (unsigned)(p.B * p.Hkv), 1);
@@ -610,7 +617,7 @@ cudaError_t launch_step(const Params& p, const void* q_rot, const S* chunk_sum,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_step_kernel<S>, maps, p, (const __nv_bfloat16*)q_rot,
+    return cudaLaunchKernelEx(&cfg, decode_step_kernel<S, kF8>, maps, p, (const __nv_bfloat16*)q_rot,
                               chunk_sum, group_sum, qbar, sel_chunks, n_sel_chunks, sel_groups,
                               n_sel_groups, (__nv_bfloat16*)out, attend ? 1 : 0,
                               (const uint4*)k_host, (const uint4*)v_host);
@@ -623,13 +630,23 @@ cudaError_t launch_decode_step(const Params& p, const void* q_rot, const void* c
                                float* qbar, int32_t* sel_chunks, int32_t* n_sel_chunks,
                                int32_t* sel_groups, int32_t* n_sel_groups, void* out,
                                cudaStream_t st, const void* k_host, const void* v_host) {
+    using bf = __nv_bfloat16;
+    const bf* cb = (const bf*)chunk_sum;
+    const bf* gb = (const bf*)group_sum;
+    const float* cf = (const float*)chunk_sum;
+    const float* gf = (const float*)group_sum;
+    if (p.sum_bf16 && p.kv_f8)
+        return launch_step<bf, true>(p, q_rot, cb, gb, k_cache, v_cache, qbar, sel_chunks,
+                                     n_sel_chunks, sel_groups, n_sel_groups, out, k_host, v_host, st);
     if (p.sum_bf16)
-        return launch_step(p, q_rot, (const __nv_bfloat16*)chunk_sum,
-                           (const __nv_bfloat16*)group_sum, k_cache, v_cache, qbar, sel_chunks,
-                           n_sel_chunks, sel_groups, n_sel_groups, out, k_host, v_host, st);
-    return launch_step(p, q_rot, (const float*)chunk_sum, (const float*)group_sum, k_cache,
-                       v_cache, qbar, sel_chunks, n_sel_chunks, sel_groups, n_sel_groups, out,
-                       k_host, v_host, st);
+        return launch_step<bf, false>(p, q_rot, cb, gb, k_cache, v_cache, qbar, sel_chunks,
+                                      n_sel_chunks, sel_groups, n_sel_groups, out, k_host, v_host, st);
+    if (p.kv_f8)
+        return launch_step<float, true>(p, q_rot, cf, gf, k_cache, v_cache, qbar, sel_chunks,
+                                        n_sel_chunks, sel_groups, n_sel_groups, out, k_host, v_host,
+                                        st);
+    return launch_step<float, false>(p, q_rot, cf, gf, k_cache, v_cache, qbar, sel_chunks,
+                                     n_sel_chunks, sel_groups, n_sel_groups, out, k_host, v_host, st);
 }
 
 }  // namespace hga

@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(32) gather_hbm_kernel(Params p, const char* __
     __shared__ __align__(8) uint64_t full[kGatherStages];
     __shared__ int64_t src_off[kGatherUnitsMax], dst_off[kGatherUnitsMax];
     const int lane = threadIdx.x;
-    const int es = p.dtype == HGA_BF16 ? 2 : 4;
+    const int es = p.kv_es;
     const uint32_t blk = (uint32_t)(kGroupRows * p.d * es);
     const int64_t total = (int64_t)p.B * p.Hkv * p.nQC * p.kg;
     const int64_t u0 = (int64_t)blockIdx.x * per;
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(256) gather_host_kernel(Params p, const uint4*
     const int64_t bh = blockIdx.z;
     const int j = p.j0 + jj;
     const int64_t prob = bh * p.nQC + jj;
-    const int es = p.dtype == HGA_BF16 ? 2 : 4;
+    const int es = p.kv_es;
     const int vec_per_blk = kGroupRows * p.d * es / 16;
     const int s_lo = blockIdx.x * kHostSlots;
     if (threadIdx.x < kHostSlots) {
@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(256) warm_copy_kernel(Params p, const uint4* _
     __shared__ int s_src[kHostSlots], s_gi[kHostSlots];
     const int64_t bh = blockIdx.z;
     const int64_t prob = bh * p.nQC;
-    const int es = p.dtype == HGA_BF16 ? 2 : 4;
+    const int es = p.kv_es;
     const int vec_per_blk = kGroupRows * p.d * es / 16;
     const int s_lo = blockIdx.x * kHostSlots;
     if (threadIdx.x < kHostSlots) {
@@ -378,7 +378,7 @@ cudaError_t launch_gather(const Params& p, const void* k_src, const void* v_src,
                           const int32_t* sel_groups, const int32_t* n_sel_groups, void* k_dst,
                           void* v_dst, cudaStream_t st) {
     if (p.nQC == 0) return cudaSuccess;
-    const int es = p.dtype == HGA_BF16 ? 2 : 4;
+    const int es = p.kv_es;
     if (from_host) {
         dim3 grid((p.kg + kHostSlots - 1) / kHostSlots, p.nQC, p.B * p.Hkv);
         gather_host_kernel<<<grid, 256, 0, st>>>(p, (const uint4*)k_src, (const uint4*)v_src,

@@ -23,6 +23,7 @@ HGA_OK = 0
 HGA_BF16, HGA_F32 = 0, 1
 HGA_KV_FULL, HGA_KV_WINDOWS = 0, 1
 HGA_SUMMARY_F32, HGA_SUMMARY_BF16 = 0, 1
+HGA_KV_AS_DTYPE, HGA_KV_E4M3 = 0, 1
 STATUS = {0: "HGA_OK", -1: "HGA_ERR_NULL", -2: "HGA_ERR_SHAPE", -3: "HGA_ERR_ALIGN",
           -4: "HGA_ERR_CONFIG", -5: "HGA_ERR_CUDA", -6: "HGA_ERR_DEVICE_INDEX",
           -7: "HGA_ERR_TIMEOUT", -8: "HGA_ERR_UNSUPPORTED", -9: "HGA_ERR_MEMORY",
@@ -41,7 +42,9 @@ class HgaConfig(ctypes.Structure):
         "batch", "seq_len", "n_q_heads", "n_kv_heads", "head_dim", "chunk_size",
         "groups_per_chunk", "n_sink", "n_local", "top_k_chunks", "top_k_groups",
         "n_high_freq_pairs")] + [("rope_theta", ctypes.c_double)] + [
-        (n, ctypes.c_int32) for n in ("dtype", "q_begin", "q_len", "kv_layout", "summary_type")]
+        (n, ctypes.c_int32) for n in ("dtype", "q_begin", "q_len", "kv_layout", "summary_type",
+                                      "kv_type")] + [
+        ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
 
     @property
     def n_chunks(self) -> int:
@@ -62,6 +65,10 @@ class HgaConfig(ctypes.Structure):
 
     def summary_torch_dtype(self) -> torch.dtype:
         return torch.bfloat16 if self.summary_type == HGA_SUMMARY_BF16 else torch.float32
+
+    def kv_torch_dtype(self) -> torch.dtype:
+        """Element type of the key/value stores and buffers."""
+        return torch.float8_e4m3fn if self.kv_type == HGA_KV_E4M3 else self.torch_dtype()
 
     def copy(self, **kw) -> "HgaConfig":
         c = HgaConfig()
@@ -125,6 +132,8 @@ def config_from(w, **overrides) -> HgaConfig:
     c.q_len = int(w.q_len)
     c.kv_layout = HGA_KV_FULL
     c.summary_type = HGA_SUMMARY_F32
+    c.kv_type = HGA_KV_AS_DTYPE
+    c.k_scale = c.v_scale = 1.0
     for k, v in overrides.items():
         setattr(c, k, v)
     return c
@@ -240,12 +249,12 @@ def decode_step(cfg: HgaConfig, q_rot, chunk_sum, group_sum, k_cache, v_cache, q
                 n_sel_chunks, sel_groups, n_sel_groups, out, stream=None) -> None:
     """Routing plus attention over the full resident cache (one launch for decode)."""
     B, H, L, d = cfg.batch, cfg.n_kv_heads, cfg.seq_len, cfg.head_dim
-    dt = cfg.torch_dtype()
+    dt, kvt = cfg.torch_dtype(), cfg.kv_torch_dtype()
     r = _route_ptrs(cfg, q_rot, chunk_sum, group_sum, qbar, sel_chunks, n_sel_chunks, sel_groups,
                     n_sel_groups)
     _check(_lib.hga_decode_step(
         ctypes.byref(cfg), r[0], r[1], r[2],
-        _ptr(k_cache, "k_cache", dt, (B, H, L, d)), _ptr(v_cache, "v_cache", dt, (B, H, L, d)),
+        _ptr(k_cache, "k_cache", kvt, (B, H, L, d)), _ptr(v_cache, "v_cache", kvt, (B, H, L, d)),
         *r[3:], _ptr(out, "out", dt, (B, cfg.q_len, cfg.n_q_heads, d)), _stream(stream)),
         "hga_decode_step")
 
@@ -256,14 +265,14 @@ def decode_step_tiered(cfg: HgaConfig, q_rot, chunk_sum, group_sum, k_win, v_win
     """One tiered decode step in one launch: routing, attention over the
     resident forced windows and the routed groups read from host memory."""
     B, H, L, d = cfg.batch, cfg.n_kv_heads, cfg.seq_len, cfg.head_dim
-    dt = cfg.torch_dtype()
+    dt, kvt = cfg.torch_dtype(), cfg.kv_torch_dtype()
     win = (B, H, window_slots(cfg) * cfg.chunk_size, d)
     r = _route_ptrs(cfg, q_rot, chunk_sum, group_sum, qbar, sel_chunks, n_sel_chunks, sel_groups,
                     n_sel_groups)
     _check(_lib.hga_decode_step_tiered(
-        ctypes.byref(cfg), r[0], r[1], r[2], _ptr(k_win, "k_win", dt, win),
-        _ptr(v_win, "v_win", dt, win), _ptr(k_host, "k_host", dt, (B, H, L, d), device=False),
-        _ptr(v_host, "v_host", dt, (B, H, L, d), device=False), *r[3:],
+        ctypes.byref(cfg), r[0], r[1], r[2], _ptr(k_win, "k_win", kvt, win),
+        _ptr(v_win, "v_win", kvt, win), _ptr(k_host, "k_host", kvt, (B, H, L, d), device=False),
+        _ptr(v_host, "v_host", kvt, (B, H, L, d), device=False), *r[3:],
         _ptr(out, "out", dt, (B, cfg.q_len, cfg.n_q_heads, d)), _stream(stream)),
         "hga_decode_step_tiered")
 
@@ -271,7 +280,7 @@ def decode_step_tiered(cfg: HgaConfig, q_rot, chunk_sum, group_sum, k_win, v_win
 def gather_kv(cfg: HgaConfig, k_src, v_src, src_is_host: bool, sel_groups, n_sel_groups, k_dst,
               v_dst, stream=None) -> None:
     B, H, L, d, nQC = cfg.batch, cfg.n_kv_heads, cfg.seq_len, cfg.head_dim, cfg.n_qchunks
-    dt = cfg.torch_dtype()
+    dt = cfg.kv_torch_dtype()
     dst_shape = (B, H, nQC, cfg.top_k_groups * cfg.group_size, d)
     _check(_lib.hga_gather_kv(
         ctypes.byref(cfg), _ptr(k_src, "k_src", dt, (B, H, L, d), device=not src_is_host),
@@ -287,7 +296,7 @@ def gather_kv_warm(cfg: HgaConfig, k_host, v_host, sel_groups, n_sel_groups, poo
                    stream=None) -> None:
     """Warm-tier gather for a one-token query span (see hga_gather_kv_warm)."""
     B, H, d, kg, g = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.top_k_groups, cfg.group_size
-    dt = cfg.torch_dtype()
+    dt = cfg.kv_torch_dtype()
     n_slots = pool_tag.shape[-1]
     store = (B, H, cfg.seq_len, d)
     gat_shape = (B, H, cfg.n_qchunks, kg * g, d)
@@ -313,7 +322,7 @@ def gather_kv_warm_noalloc(cfg: HgaConfig, k_host, v_host, sel_groups, n_sel_gro
     plan-to-copy source list lives in the library's fixed scratch array
     (see hga_gather_kv_warm_noalloc). Allocates nothing itself either."""
     B, H, d, kg, g = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.top_k_groups, cfg.group_size
-    dt = cfg.torch_dtype()
+    dt = cfg.kv_torch_dtype()
     n_slots = pool_tag.shape[-1]
     store = (B, H, cfg.seq_len, d)
     gat_shape = (B, H, cfg.n_qchunks, kg * g, d)
@@ -339,15 +348,16 @@ def window_slots(cfg: HgaConfig) -> int:
 def attend(cfg: HgaConfig, q_rot, k_res, v_res, sel_groups, n_sel_groups, out, k_gat=None,
            v_gat=None, stream=None) -> None:
     B, H, L, d, nQC = cfg.batch, cfg.n_kv_heads, cfg.seq_len, cfg.head_dim, cfg.n_qchunks
-    dt = cfg.torch_dtype()
+    dt, kvt = cfg.torch_dtype(), cfg.kv_torch_dtype()
     res_len = L if cfg.kv_layout == HGA_KV_FULL else window_slots(cfg) * cfg.chunk_size
     gat_shape = (B, H, nQC, cfg.top_k_groups * cfg.group_size, d)
     q_shape = (B, cfg.q_len, cfg.n_q_heads, d)
     _check(_lib.hga_attend(
         ctypes.byref(cfg), _ptr(q_rot, "q_rot", dt, q_shape),
-        _ptr(k_res, "k_res", dt, (B, H, res_len, d)), _ptr(v_res, "v_res", dt, (B, H, res_len, d)),
-        _ptr(k_gat, "k_gat", dt, gat_shape, nullable=True),
-        _ptr(v_gat, "v_gat", dt, gat_shape, nullable=True),
+        _ptr(k_res, "k_res", kvt, (B, H, res_len, d)),
+        _ptr(v_res, "v_res", kvt, (B, H, res_len, d)),
+        _ptr(k_gat, "k_gat", kvt, gat_shape, nullable=True),
+        _ptr(v_gat, "v_gat", kvt, gat_shape, nullable=True),
         _ptr(sel_groups, "sel_groups", torch.int32, (B, H, nQC, cfg.top_k_groups)),
         _ptr(n_sel_groups, "n_sel_groups", torch.int32, (B, H, nQC)),
         _ptr(out, "out", dt, q_shape), _stream(stream)), "hga_attend")

@@ -48,8 +48,8 @@ def alloc_warm_pool(cfg: hga.HgaConfig, n_slots: int, device="cuda") -> WarmPool
     B, H, d, g = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.group_size
     i32 = dict(dtype=torch.int32, device=device)
     return WarmPool(
-        k=torch.zeros(B, H, n_slots, g, d, dtype=cfg.torch_dtype(), device=device),
-        v=torch.zeros(B, H, n_slots, g, d, dtype=cfg.torch_dtype(), device=device),
+        k=torch.zeros(B, H, n_slots, g, d, dtype=cfg.kv_torch_dtype(), device=device),
+        v=torch.zeros(B, H, n_slots, g, d, dtype=cfg.kv_torch_dtype(), device=device),
         tag=torch.full((B, H, n_slots), -1, **i32), last=torch.full((B, H, n_slots), -1, **i32),
         src=torch.empty(B, H, cfg.top_k_groups, **i32), stats=torch.zeros(B, H, 2, **i32))
 
@@ -81,8 +81,8 @@ def alloc_route(cfg: hga.HgaConfig, device="cuda", with_scores: bool = False) ->
 def alloc_gathered(cfg: hga.HgaConfig, device="cuda"):
     shape = (cfg.batch, cfg.n_kv_heads, cfg.n_qchunks, cfg.top_k_groups * cfg.group_size,
              cfg.head_dim)
-    return (torch.zeros(shape, dtype=cfg.torch_dtype(), device=device),
-            torch.zeros(shape, dtype=cfg.torch_dtype(), device=device))
+    return (torch.zeros(shape, dtype=cfg.kv_torch_dtype(), device=device),
+            torch.zeros(shape, dtype=cfg.kv_torch_dtype(), device=device))
 
 
 def rotate_queries(cfg: hga.HgaConfig, q_raw: torch.Tensor, stream=None) -> torch.Tensor:

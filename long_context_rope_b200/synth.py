@@ -19,6 +19,10 @@ Recipe (one torch CPU generator per call, seeded; draw order fixed):
      `plant_count` distinct chunks drawn uniformly from [0, j), added to every
      query token of chunk j for all query heads of the topic's KV head.
 All values are drawn in float32 and then cast to the workload's dtype.
+
+FP8 K/V caches (the E4M3 storage variant) are made from drawn or rotated
+tensors by `to_e4m3`: a per-tensor scale amax / 448 and torch's
+float8_e4m3fn cast, the same kind of storage conversion as the bf16 cast.
 """
 from __future__ import annotations
 
@@ -189,6 +193,22 @@ def bytes_per_step(w: Workload) -> Dict[str, int]:
     return {"k": n_kv * es, "v": n_kv * es, "q": n_q * es, "o": n_q * es}
 
 
+E4M3_MAX = 448.0
+
+
+def to_e4m3(x: torch.Tensor):
+    """An FP8 cache of x: (codes as torch.float8_e4m3fn, scale), with the
+    per-tensor scale amax(|x|) / 448 so the largest element maps to the
+    format's largest finite value; each code is x / scale cast to E4M3
+    (values clamped to +-448 first, so none overflows to NaN)."""
+    xf = x.float()
+    amax = float(xf.abs().max()) if xf.numel() else 0.0
+    scale = amax / E4M3_MAX if amax > 0 else 1.0
+    scale = float(torch.tensor(scale, dtype=torch.float32))  # an fp32 scale, as the ABI takes
+    codes = (xf / scale).clamp_(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
+    return codes, scale
+
+
 def seed_for_rank(base_seed: int, rank: int) -> int:
     """Each rank of a weak-scaling run draws its own independent sequence."""
     return int(base_seed) + 1000003 * int(rank)
@@ -208,4 +228,4 @@ def describe(w: Workload) -> str:
 
 
 __all__ = ["Workload", "WORKLOADS", "draw", "bytes_per_step", "seed_for_rank",
-           "ceil_div", "describe"]
+           "ceil_div", "describe", "to_e4m3", "E4M3_MAX"]

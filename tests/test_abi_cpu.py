@@ -31,10 +31,13 @@ def test_exports_every_declared_symbol(hga):
 
 
 def test_struct_layout_matches_header(hga):
-    # 12 int32 (48 bytes), a double at offset 48, 5 int32 (76), 8-byte aligned: 80
-    assert ctypes.sizeof(hga.HgaConfig) == 80
+    # 12 int32 (48 bytes), a double at offset 48, 6 int32 (80), two floats: 88
+    assert ctypes.sizeof(hga.HgaConfig) == 88
     assert hga.HgaConfig.rope_theta.offset == 48
     assert hga.HgaConfig.summary_type.offset == 72
+    assert hga.HgaConfig.kv_type.offset == 76
+    assert hga.HgaConfig.k_scale.offset == 80
+    assert hga.HgaConfig.v_scale.offset == 84
 
 
 def _cfg(hga, **kw):
@@ -52,6 +55,26 @@ def test_summary_type_validation_without_gpu(hga):
     # the separate routing calls do not read bf16 tables
     assert L.hga_route_chunks(by(bf), P, P, P, P, P, None, None) == -8
     assert L.hga_route_groups(by(bf), P, P, P, P, P, P, None, None) == -8
+
+
+def test_fp8_kv_validation_without_gpu(hga):
+    """E4M3 K/V: scales must be finite and positive, the queries bf16 and
+    d = 128; prefill attention and a rotated-key output are refused."""
+    L = hga.library()
+    P = 16 * 1024  # never dereferenced: refused on the host
+    by = ctypes.byref
+    attend = [P] * 3 + [None, None] + [P] * 3 + [None]
+    assert L.hga_attend(by(_cfg(hga, kv_type=5)), *attend) == -4
+    for ks, vs in ((0.0, 1.0), (1.0, -1.0), (float("nan"), 1.0), (1.0, float("inf"))):
+        bad = _cfg(hga, kv_type=hga.HGA_KV_E4M3, k_scale=ks, v_scale=vs)
+        assert L.hga_attend(by(bad), *attend) == -4, (ks, vs)
+    ok = dict(kv_type=hga.HGA_KV_E4M3, k_scale=0.01, v_scale=0.02)
+    assert L.hga_attend(by(_cfg(hga, dtype=hga.HGA_F32, **ok)), *attend) == -8
+    assert L.hga_attend(by(_cfg(hga, **ok)), *attend) == -8  # prefill span (q_len > 1)
+    assert L.hga_build_summaries(by(_cfg(hga, **ok)), P, P, P, P, 0, 4, None) == -8
+    # decode span: the host checks pass, so a NULL output is what is reported
+    dec = _cfg(hga, q_begin=4095, q_len=1, **ok)
+    assert L.hga_attend(by(dec), *attend[:-2], None, None) == -1
 
 
 def test_tiered_step_validation_without_gpu(hga):
