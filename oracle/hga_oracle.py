@@ -285,6 +285,23 @@ def pipeline(w, inputs, units=None, want_scores: bool = True, attend_out: bool =
     return res
 
 
+def per_q_head(w, inputs):
+    """Per-query-head routing (the variant in which every query head routes
+    on its own rotated queries instead of the KV head's shared q-bar), stated
+    as the plain routing of an expanded problem: query head h gets its own
+    copy of the raw keys and values of its KV head h // gq, so its routing
+    query is the mean of its own queries over the chunk's tokens, it scores
+    and selects over that KV head's summaries, and it attends over its own
+    selection. Returns (w_h, inputs_h) to give to pipeline(); w_h has as many
+    KV heads as query heads (w.replace is the workload's own copy-with)."""
+    gq = w.n_q_heads // w.n_kv_heads
+    w_h = w.replace(n_kv_heads=w.n_q_heads)
+    inputs_h = dict(inputs)
+    inputs_h["k_raw"] = np.repeat(_as_np(inputs["k_raw"]), gq, axis=1)
+    inputs_h["v"] = np.repeat(_as_np(inputs["v"]), gq, axis=1)
+    return w_h, inputs_h
+
+
 def _as_np(t) -> np.ndarray:
     if isinstance(t, np.ndarray):
         return np.ascontiguousarray(t, dtype=np.float32)

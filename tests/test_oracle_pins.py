@@ -476,3 +476,55 @@ def test_decode_query_at_last_position():
     gsel, gnsel, _ = O.route_groups(cfg_d, qb, gs, sel, nsel)
     out = O.attend(cfg_d, qd, k, v, gsel, gnsel)
     np.testing.assert_allclose(out[0, 0], _dense_sdpa(q, k, v)[0, 127], atol=1e-12)
+
+
+# ------------------------------------------------- per-query-head routing ---
+
+def _per_head_case(equal_heads: bool):
+    from long_context_rope_b200 import synth
+    w = synth.WORKLOADS["prefill_4k"].replace(name="perhead", seq_len=2048, n_q_heads=8,
+                                              n_kv_heads=2, top_k_chunks=2, top_k_groups=5)
+    x = synth.draw(w, seed=21)
+    if equal_heads:  # every query head of a KV head carries the same query
+        q = x["q_raw"].clone()
+        gq = w.n_q_heads // w.n_kv_heads
+        for h in range(w.n_q_heads):
+            q[:, :, h] = x["q_raw"][:, :, (h // gq) * gq]
+        x = dict(x, q_raw=q)
+    return w, x
+
+
+def test_per_q_head_routing_reduces_to_shared_routing():
+    """With the query heads of each KV head all equal, each head's own routing
+    query is the shared q-bar, so per-query-head routing selects exactly the
+    shared selections (per query head) and attends to the same keys."""
+    w, x = _per_head_case(equal_heads=True)
+    gq = w.n_q_heads // w.n_kv_heads
+    r = O.pipeline(w, x)
+    rh = O.pipeline(*O.per_q_head(w, x))
+    for h in range(w.n_q_heads):
+        for key in ("sel_chunks", "n_sel_chunks", "sel_groups", "n_sel_groups"):
+            np.testing.assert_array_equal(rh[key][:, h], r[key][:, h // gq], err_msg=key)
+        np.testing.assert_allclose(rh["qbar"][:, h], r["qbar"][:, h // gq], rtol=1e-12,
+                                   atol=1e-12)
+    np.testing.assert_allclose(rh["out"], r["out"], rtol=0, atol=1e-12)
+
+
+def test_per_q_head_qbar_is_the_heads_own_mean():
+    """Distinct query heads: head h's routing query is the mean of its own
+    rotated queries over the chunk's tokens, and its summaries are its KV
+    head's."""
+    w, x = _per_head_case(equal_heads=False)
+    gq = w.n_q_heads // w.n_kv_heads
+    r = O.pipeline(w, x)
+    rh = O.pipeline(*O.per_q_head(w, x))
+    C = w.chunk_size
+    q_rot = rh["q_rot"].astype(np.float64)
+    for j in range(w.seq_len // C):
+        want = q_rot[:, j * C:(j + 1) * C].mean(axis=1)  # [B, Hq, d]
+        np.testing.assert_allclose(rh["qbar"][:, :, j], want, rtol=1e-12, atol=1e-12)
+    for h in range(w.n_q_heads):
+        np.testing.assert_array_equal(rh["chunk_sum"][:, h], r["chunk_sum"][:, h // gq])
+    # distinct queries do route differently somewhere
+    assert any(not np.array_equal(rh["sel_groups"][:, h], r["sel_groups"][:, h // gq])
+               for h in range(w.n_q_heads))
