@@ -129,6 +129,21 @@ typedef enum { HGA_SUMMARY_F32 = 0, HGA_SUMMARY_BF16 = 1 } hga_summary_type;
  *                  hga_build_summaries return HGA_ERR_UNSUPPORTED. */
 typedef enum { HGA_KV_AS_DTYPE = 0, HGA_KV_E4M3 = 1 } hga_kv_type;
 
+/* Which heads route.
+ * HGA_ROUTE_PER_KV_HEAD: one routing query per (sequence, KV head, query
+ *     chunk), the q-bar of the conventions above; the KV head's query heads
+ *     attend over one shared selection.
+ * HGA_ROUTE_PER_Q_HEAD:  one routing query per (sequence, query head, query
+ *     chunk): the mean of that head's own rotated queries over the chunk's
+ *     query tokens. It scores its KV head's summaries (KV head h / (Hq/Hkv))
+ *     and the head attends over its own selection. q-bar, the selection
+ *     lists and their counts then have Hq rows where the layouts above say
+ *     Hkv ([B, Hq, nQC, ...]). Decode (q_len == 1) only: hga_route,
+ *     hga_decode_step and hga_decode_step_tiered on their one-launch path,
+ *     and hga_attend in index mode; every other call returns
+ *     HGA_ERR_UNSUPPORTED. */
+typedef enum { HGA_ROUTE_PER_KV_HEAD = 0, HGA_ROUTE_PER_Q_HEAD = 1 } hga_routing;
+
 typedef struct {
     int32_t batch;             /* B */
     int32_t seq_len;           /* L: tokens in the K/V history (context length) */
@@ -151,6 +166,7 @@ typedef struct {
     int32_t kv_type;           /* hga_kv_type of keys and values (0 = cfg->dtype) */
     float k_scale;             /* HGA_KV_E4M3: scale of the key codes (finite, > 0) */
     float v_scale;             /* HGA_KV_E4M3: scale of the value codes (finite, > 0) */
+    int32_t routing;           /* hga_routing (0 = per KV head) */
 } hga_config;
 
 /* Rotate x by RoPE (standard rotary position embedding; the summaries of

@@ -98,6 +98,8 @@ hga_status make_params(const hga_config* c, Params* p) {
     if (c->summary_type != HGA_SUMMARY_F32 && c->summary_type != HGA_SUMMARY_BF16)
         return HGA_ERR_CONFIG;
     if (c->kv_type != HGA_KV_AS_DTYPE && c->kv_type != HGA_KV_E4M3) return HGA_ERR_CONFIG;
+    if (c->routing != HGA_ROUTE_PER_KV_HEAD && c->routing != HGA_ROUTE_PER_Q_HEAD)
+        return HGA_ERR_CONFIG;
     if (c->kv_type == HGA_KV_E4M3) {
         if (!(c->k_scale > 0.0f) || !isfinite(c->k_scale) || !(c->v_scale > 0.0f) ||
             !isfinite(c->v_scale))
@@ -117,7 +119,9 @@ hga_status make_params(const hga_config* c, Params* p) {
     p->C = c->chunk_size;
     p->G = c->groups_per_chunk;
     p->g = kGroupRows;
-    p->gq = c->n_q_heads / c->n_kv_heads;
+    const bool per_q = c->routing == HGA_ROUTE_PER_Q_HEAD;
+    p->Hu = per_q ? c->n_q_heads : c->n_kv_heads;
+    p->gq = per_q ? 1 : c->n_q_heads / c->n_kv_heads;
     p->n_sink = c->n_sink;
     p->n_local = c->n_local;
     p->kc = c->top_k_chunks;
@@ -185,7 +189,8 @@ cudaError_t set_func_attr_once(const void* fn, cudaFuncAttribute attr, int value
 
 using namespace hga;
 
-static_assert(sizeof(hga_config) == 88, "hga_config layout is part of the ABI");
+static_assert(sizeof(hga_config) == 96, "hga_config layout is part of the ABI");
+static_assert(offsetof(hga_config, routing) == 88, "hga_config layout is part of the ABI");
 static_assert(offsetof(hga_config, summary_type) == 72, "hga_config layout is part of the ABI");
 static_assert(offsetof(hga_config, kv_type) == 76, "hga_config layout is part of the ABI");
 static_assert(offsetof(hga_config, v_scale) == 84, "hga_config layout is part of the ABI");
@@ -193,7 +198,7 @@ static_assert(offsetof(hga_config, rope_theta) == 48, "hga_config layout is part
 
 extern "C" {
 
-int32_t hga_version(void) { return 10700; }
+int32_t hga_version(void) { return 10800; }
 
 void hga_set_wait_limit_ns(uint64_t limit_ns) {
     g_wait_ns.store(limit_ns == 0 ? 1000000000ull : (unsigned long long)limit_ns,
@@ -264,6 +269,7 @@ hga_status hga_route_chunks(const hga_config* cfg, const void* q_rot, const void
         !aligned16(sel_chunks) || !aligned16(n_sel_chunks) || (scores_out && !aligned16(scores_out)))
         return HGA_ERR_ALIGN;
     if (p.sum_bf16) return HGA_ERR_UNSUPPORTED;  // bf16 tables: the one-launch decode path only
+    if (p.Hu != p.Hkv) return HGA_ERR_UNSUPPORTED;  // per query head: the decode step only
     HGA_ATTACH_ERR(p);
     cudaStream_t st = (cudaStream_t)stream;
     if (!route_chunks_fuses_qbar(p)) {
@@ -289,6 +295,7 @@ hga_status hga_route_groups(const hga_config* cfg, const float* qbar, const void
         (scores_out && !aligned16(scores_out)))
         return HGA_ERR_ALIGN;
     if (p.sum_bf16) return HGA_ERR_UNSUPPORTED;  // bf16 tables: the one-launch decode path only
+    if (p.Hu != p.Hkv) return HGA_ERR_UNSUPPORTED;  // per query head: the decode step only
     HGA_ATTACH_ERR(p);
     return launched(launch_route_groups(p, qbar, (const float*)group_sum, sel_chunks, n_sel_chunks,
                                         sel_groups, n_sel_groups, scores_out,
@@ -316,7 +323,7 @@ static hga_status route_separate(const Params& p, const void* q_rot, const void*
                                  const void* group_sum, float* qbar_out, int32_t* sel_chunks,
                                  int32_t* n_sel_chunks, int32_t* sel_groups,
                                  int32_t* n_sel_groups, cudaStream_t st) {
-    if (p.sum_bf16) return HGA_ERR_UNSUPPORTED;  // bf16 tables: the one-launch decode path only
+    if (p.sum_bf16 || p.Hu != p.Hkv) return HGA_ERR_UNSUPPORTED;  // one-launch path only
     if (!route_chunks_fuses_qbar(p) && launch_qbar(p, q_rot, qbar_out, st) != cudaSuccess)
         return HGA_ERR_CUDA;
     if (launch_route_chunks(p, q_rot, qbar_out, (const float*)chunk_sum, sel_chunks, n_sel_chunks,
@@ -368,6 +375,7 @@ hga_status hga_decode_step(const hga_config* cfg, const void* q_rot, const void*
                                            qbar_out, sel_chunks, n_sel_chunks, sel_groups,
                                            n_sel_groups, out, st));
     if (p.kv_f8 && !decode_kernel_supports(p)) return HGA_ERR_UNSUPPORTED;
+    if (p.Hu != p.Hkv) return HGA_ERR_UNSUPPORTED;  // per query head: one-launch path only
     s = route_separate(p, q_rot, chunk_sum, group_sum, qbar_out, sel_chunks, n_sel_chunks,
                        sel_groups, n_sel_groups, st);
     if (s != HGA_OK) return s;
@@ -439,6 +447,7 @@ hga_status hga_gather_kv(const hga_config* cfg, const void* k_src, const void* v
     if (!aligned16(k_src) || !aligned16(v_src) || !aligned16(sel_groups) ||
         !aligned16(n_sel_groups) || !aligned16(k_dst) || !aligned16(v_dst))
         return HGA_ERR_ALIGN;
+    if (p.Hu != p.Hkv) return HGA_ERR_UNSUPPORTED;  // gathers follow per-KV-head lists
     HGA_ATTACH_ERR(p);
     const void* kd = nullptr;
     const void* vd = nullptr;
@@ -465,7 +474,7 @@ hga_status hga_gather_kv_warm(const hga_config* cfg, const void* k_host, const v
         !aligned16(pool_tag) || !aligned16(pool_last) || !aligned16(src_out) ||
         !aligned16(k_dst) || !aligned16(v_dst) || (stats_out && !aligned16(stats_out)))
         return HGA_ERR_ALIGN;
-    if (p.q_len != 1) return HGA_ERR_UNSUPPORTED;
+    if (p.q_len != 1 || p.Hu != p.Hkv) return HGA_ERR_UNSUPPORTED;
     if (n_slots < p.kg || step < 0) return HGA_ERR_SHAPE;
     if (!gather_warm_supports(p, n_slots)) return HGA_ERR_UNSUPPORTED;
     HGA_ATTACH_ERR(p);
@@ -496,7 +505,7 @@ hga_status hga_gather_kv_warm_noalloc(const hga_config* cfg, const void* k_host,
         !aligned16(pool_tag) || !aligned16(pool_last) || !aligned16(k_dst) ||
         !aligned16(v_dst) || (stats_out && !aligned16(stats_out)))
         return HGA_ERR_ALIGN;
-    if (p.q_len != 1) return HGA_ERR_UNSUPPORTED;
+    if (p.q_len != 1 || p.Hu != p.Hkv) return HGA_ERR_UNSUPPORTED;
     if (n_slots < p.kg || step < 0) return HGA_ERR_SHAPE;
     if (!gather_warm_supports(p, n_slots)) return HGA_ERR_UNSUPPORTED;
     if ((int64_t)p.B * p.Hkv * p.kg > kWarmScratchEntries) return HGA_ERR_SCRATCH_LIMIT;
@@ -530,10 +539,12 @@ hga_status hga_attend(const hga_config* cfg, const void* q_rot, const void* k_re
         (p.q_len != 1 || p.q_begin != p.L - 1 || k_gat == nullptr))
         return HGA_ERR_UNSUPPORTED;
     if (p.kv_f8 && !decode_kernel_supports(p)) return HGA_ERR_UNSUPPORTED;  // decode only
+    if (p.Hu != p.Hkv && (!decode_kernel_supports(p) || k_gat != nullptr))
+        return HGA_ERR_UNSUPPORTED;  // per query head: decode, index mode
     HGA_ATTACH_ERR(p);
     KvSources kv{k_res, v_res, k_gat, v_gat};
     cudaStream_t st = (cudaStream_t)stream;
-    if (p.kv_f8)
+    if (p.kv_f8 || p.Hu != p.Hkv)
         return launched(launch_attend_decode(p, q_rot, kv, sel_groups, n_sel_groups, out, st));
     if (tc_kernel_supports(p, k_gat != nullptr))
         return launched(launch_attend_tc(p, q_rot, kv, sel_groups, n_sel_groups, out, st));

@@ -25,6 +25,9 @@ struct Params {
     int nC, q_begin, q_len, j0, nQC;
     int dtype, kv_layout;
     int sum_bf16;                  // summary tables stored as bf16 (else fp32)
+    int Hu;                        // routing units per sequence: Hkv, or Hq (per query head);
+                                   // gq = query heads per unit; unit h reads KV head
+                                   // h / (Hu / Hkv)
     int kv_f8;                     // K/V stored as E4M3 codes (else dtype)
     int kv_es;                     // bytes per K/V element
     float k_scale, v_scale;        // E4M3 code scales (1 otherwise)

@@ -304,30 +304,37 @@ __device__ __forceinline__ void store_warp_partial(const WarpAcc& acc, Partial& 
     }
 }
 
-// All threads of the CTA: merge the 8 warp partials into cta.
-__device__ __forceinline__ void merge_warps(const Partial* warp_part, Partial& cta) {
-    for (int x = threadIdx.x; x < 8 * kD; x += blockDim.x) {
-        const int n = x / kD, d = x % kD;
+// All threads of the CTA: merge the 8 warp partials into cta. First the
+// per-(warp, head) weights 2^(m_w - M) and the merged max and sum (64 + 8
+// threads), then the weighted sums of O; wgt is an 8 x 8 scratch. Ends with
+// the CTA's barrier.
+__device__ __forceinline__ void merge_warps(const Partial* warp_part, Partial& cta,
+                                            float (*wgt)[8]) {
+    const int t = threadIdx.x;
+    if (t < 8 * kConsumers) {
+        const int w = t >> 3, n = t & 7;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, warp_part[w].m[n]);
-        float num = 0.f, den = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < kConsumers; ++w) {
-                const float mw = warp_part[w].m[n];
-                if (mw == -INFINITY) continue;
-                const float wgt = ptx::ex2_approx(mw - M);
-                num = fmaf(wgt, warp_part[w].o[n][d], num);
-                den = fmaf(wgt, warp_part[w].l[n], den);
-            }
-        }
-        cta.o[n][d] = num;
-        if (d == 0) {
-            cta.m[n] = M;
-            cta.l[n] = den;
-        }
+        for (int v = 0; v < kConsumers; ++v) M = fmaxf(M, warp_part[v].m[n]);
+        const float mw = warp_part[w].m[n];
+        wgt[w][n] = (M == -INFINITY || mw == -INFINITY) ? 0.f : ptx::ex2_approx(mw - M);
+        if (w == 0) cta.m[n] = M;
     }
+    __syncthreads();
+    if (t < 8) {
+        float den = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumers; ++w) den = fmaf(wgt[w][t], warp_part[w].l[t], den);
+        cta.l[t] = den;
+    }
+    for (int x = t; x < 8 * kD; x += blockDim.x) {
+        const int n = x / kD, d = x % kD;
+        float num = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumers; ++w) num = fmaf(wgt[w][n], warp_part[w].o[n][d], num);
+        cta.o[n][d] = num;
+    }
+    __syncthreads();
 }
 
 // After a cluster barrier: CTA r merges the CL CTA partials of heads

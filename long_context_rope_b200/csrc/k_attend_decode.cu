@@ -51,6 +51,7 @@ struct DecodeSmem {
         dec::Partial warp_part[kConsumers];      // reused once the ring is drained
     } u;
     dec::Partial cta_part;
+    float wgt[kConsumers][8];                    // warp-merge weights
     uint16_t pt[kConsumers][8][16];              // per-warp P transpose buffer
     uint64_t full[kStages], empty[kStages];
     int blk_row[kMaxBlocks];
@@ -70,8 +71,9 @@ __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
     cg::cluster_group cluster = cg::this_cluster();
     const int CL = (int)cluster.num_blocks();
     const int r = (int)cluster.block_rank();
-    const int64_t bh = blockIdx.y;
-    const int b = (int)(bh / p.Hkv), h = (int)(bh % p.Hkv);
+    const int64_t bh = blockIdx.y;  // routing unit: (sequence, KV head) or (sequence, query head)
+    const int b = (int)(bh / p.Hu), h = (int)(bh % p.Hu);
+    const int64_t kvh = (int64_t)b * p.Hkv + h / (p.Hu / p.Hkv);  // its K/V row
     const int j = p.j0;
     const int64_t prob = bh * p.nQC;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -112,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
                 const bool gat = (rw & kSrcGathered) != 0;
                 const int row = rw & ~kSrcGathered;
                 dec::issue_block<kF8>(sm.u.ring, sm.full, s, gat ? &maps.k_gat : &maps.k_res,
-                                 gat ? &maps.v_gat : &maps.v_res, row, (int)(gat ? prob : bh));
+                                 gat ? &maps.v_gat : &maps.v_res, row, (int)(gat ? prob : kvh));
             }
             // every issued load lands before the ring's memory is reused
             if (!dec::drain_ring(sm.full, i)) {
@@ -136,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
     // ---- per-warp partials -> shared memory (the ring's space is reused)
     if (warp < kConsumers) dec::store_warp_partial<kF8>(acc, sm.u.warp_part[warp]);
     __syncthreads();
-    dec::merge_warps(sm.u.warp_part, sm.cta_part);
+    dec::merge_warps(sm.u.warp_part, sm.cta_part, sm.wgt);
     cluster.sync();
     dec::merge_cluster_and_store(p, cluster, sm.cta_part, b, h, out);
     cluster.sync();
@@ -154,7 +156,7 @@ template <bool kF8>
 int pick_cluster(const Params& p, size_t smem, int dev) {
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int units = p.B * p.Hkv;
+    const int units = p.B * p.Hu;
     int cl = 2 * sms / units;  // two CTAs per SM
     cl = cl < 1 ? 1 : (cl > kMaxCluster ? kMaxCluster : cl);
     std::lock_guard<std::mutex> lock(g_decode_mu);
@@ -244,7 +246,7 @@ cudaError_t launch_decode_t(const Params& p, const void* q_rot, const KvSources&
     int cl = pick_cluster<kF8>(p, smem, dev);
     if (cl > max_cluster) cl = max_cluster;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cl, (unsigned)BH, 1);
+    cfg.gridDim = dim3(cl, (unsigned)((int64_t)p.B * p.Hu), 1);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;

@@ -71,9 +71,11 @@ struct StepSmem {
         dec::Partial warp_part[kConsumers];
     } u;
     dec::Partial cta_part;
+    float wgt[kConsumers][8];                    // warp-merge weights
     uint16_t pt[kConsumers][8][16];
     uint64_t full[kStages], empty[kStages];
     uint64_t key1[kMaxSlice];     // own level-1 candidates
+    uint64_t own1[kMaxKc];        // this CTA's level-1 finalists, ascending
     uint64_t f1[kMaxF1];          // level-1 finalists of all CTAs
     uint64_t key2[kMaxCand2];     // level-2 candidates (all of them, every CTA)
     int rank[kMaxSlice > kMaxCand2 ? kMaxSlice : kMaxCand2];  // rank scratch
@@ -222,10 +224,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     cg::cluster_group cluster = cg::this_cluster();
     const int CL = (int)cluster.num_blocks();
     const int r = (int)cluster.block_rank();
-    const int64_t bh = blockIdx.y;
-    const int b = (int)(bh / p.Hkv), h = (int)(bh % p.Hkv);
+    const int64_t bh = blockIdx.y;  // routing unit: (sequence, KV head) or (sequence, query head)
+    const int b = (int)(bh / p.Hu), h = (int)(bh % p.Hu);
+    const int64_t kvh = (int64_t)b * p.Hkv + h / (p.Hu / p.Hkv);  // its K/V and summary row
     const int j = p.j0;
-    const int64_t prob = bh;  // one query chunk per (sequence, KV head)
+    const int64_t prob = bh;  // one query chunk per unit
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const bool consumer = warp < kConsumers;
 
@@ -259,9 +262,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     }
     __syncthreads();
     const int n_pre = nf_loc < kStages ? nf_loc : kStages;
-    if (attend && warp == kConsumers && lane == 0)
-        for (int i = 0; i < n_pre; ++i)
-            dec::issue_block<kF8>(sm.u.ring, sm.full, i, &maps.k, &maps.v, sm.blk_row[i], (int)bh);
 
     // ---- level-1 slice: the first batch of this warp's chunk-summary rows is
     // requested before q-bar, so the two memory latencies overlap
@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     const int c_lo = r * per1;
     const int c_hi = c_lo + per1 < j ? c_lo + per1 : j;
     const int ns = c_hi > c_lo ? c_hi - c_lo : 0;
-    const S* ctab = cs + bh * (int64_t)p.nC * kD;
+    const S* ctab = cs + kvh * (int64_t)p.nC * kD;
     float4 first[kL1Rows];
     if (consumer) {
 #pragma unroll
@@ -342,11 +342,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
                                 [&](int x, float s) { emit1(rest0 + x, s); });
     }
     __syncthreads();
+    // the forced blocks' loads are issued once the level-1 rows are in: they
+    // are needed only after routing, and the chunk-summary reads above are
+    // on the critical path
+    if (attend && warp == kConsumers && lane == 0)
+        for (int i = 0; i < n_pre; ++i)
+            dec::issue_block<kF8>(sm.u.ring, sm.full, i, &maps.k, &maps.v, sm.blk_row[i], (int)kvh);
     if (consumer) count_greater(sm.key1, ns, sm.key1, ns, sm.rank);
     __syncthreads();
-    // this CTA's winners go to slots [r * cap1, (r + 1) * cap1) of every
-    // CTA's finalist table in candidate (= ascending chunk) order, so the
-    // table is ascending: slices are contiguous and ordered by r
+    // this CTA's winners, in candidate (= ascending chunk) order, padded
+    // with 0 to cap1 entries
     if (warp == 0) {
         int base = 0;
         for (int x0 = 0; x0 < ns; x0 += 32) {
@@ -354,16 +359,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
             const uint64_t k = x < ns ? sm.key1[x] : 0ull;
             const bool win = k != 0ull && sm.rank[x] < cap1;
             const unsigned m = __ballot_sync(0xffffffffu, win);
-            if (win) {
-                const int at = r * cap1 + base + __popc(m & ((1u << lane) - 1u));
-                for (int t = 0; t < CL; ++t) cluster.map_shared_rank(sm.f1, t)[at] = k;
-            }
+            if (win) sm.own1[base + __popc(m & ((1u << lane) - 1u))] = k;
             base += __popc(m);
         }
-        for (int x = base + lane; x < cap1; x += 32)
-            for (int t = 0; t < CL; ++t) cluster.map_shared_rank(sm.f1, t)[r * cap1 + x] = 0ull;
+        for (int x = base + lane; x < cap1; x += 32) sm.own1[x] = 0ull;
     }
     cluster.sync();
+    // the finalist table: CTA t's winners at slots [t * cap1, (t + 1) * cap1),
+    // read from its shared memory; ascending, as the slices are contiguous
+    // and ordered by t
+    for (int x = tid; x < CL * cap1; x += blockDim.x)
+        sm.f1[x] = cluster.map_shared_rank(sm.own1, x / cap1)[x % cap1];
+    __syncthreads();
 
     // ---- every CTA ranks the whole finalist table: the global top k_c,
     // compacted in table order, which is ascending chunk order
@@ -393,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     // (candidate x = group x % G of the (x / G)-th chunk: ascending group
     // index) and ranks them exactly; no second cluster exchange is needed
     const int n2 = nsel1 * p.G;
-    const S* gtab = gs + bh * (int64_t)p.nC * p.G * kD;
+    const S* gtab = gs + kvh * (int64_t)p.nC * p.G * kD;
     if (consumer)
         score_rows<16>(qv, n2,
                        [&](int x) { return gtab + ((int64_t)sm.win1[x / p.G] * p.G + x % p.G) * kD; },
@@ -453,13 +460,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
                 }
             }
             if (host_tier && i >= nf_loc) {
-                const int64_t row = bh * (int64_t)p.L + sm.blk_row[i];
+                const int64_t row = kvh * (int64_t)p.L + sm.blk_row[i];
                 constexpr int kRowVecs = kF8 ? kD / 16 : kD / 8;  // 16-byte pieces per row
                 copy_host_block<kF8>(sm.u.ring, s, k_host + row * kRowVecs, v_host + row * kRowVecs);
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&sm.full[s]);
             } else if (lane == 0) {
-                dec::issue_block<kF8>(sm.u.ring, sm.full, s, &maps.k, &maps.v, sm.blk_row[i], (int)bh);
+                dec::issue_block<kF8>(sm.u.ring, sm.full, s, &maps.k, &maps.v, sm.blk_row[i], (int)kvh);
             }
         }
         if (lane == 0) {
@@ -486,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     __syncthreads();
     if (consumer) dec::store_warp_partial<kF8>(acc, sm.u.warp_part[warp]);
     __syncthreads();
-    dec::merge_warps(sm.u.warp_part, sm.cta_part);
+    dec::merge_warps(sm.u.warp_part, sm.cta_part, sm.wgt);
     cluster.sync();
     dec::merge_cluster_and_store(p, cluster, sm.cta_part, b, h, out);
     cluster.sync();
@@ -554,7 +561,7 @@ int step_cluster(const Params& p, size_t smem) {
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int units = p.B * p.Hkv;
+    const int units = p.B * p.Hu;
     int cl = 2 * sms / units;
     cl = cl < 1 ? 1 : (cl > kMaxCluster ? kMaxCluster : cl);
     for (; cl >= 1; --cl) {
@@ -606,7 +613,7 @@ cudaError_t launch_step(const Params& p, const void* q_rot, const S* chunk_sum,
     const int cl = step_cluster<S, kF8>(p, smem);
     if (cl < 1) return cudaErrorInvalidConfiguration;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cl, (unsigned)(p.B * p.Hkv), 1);
+    cfg.gridDim = dim3(cl, (unsigned)(p.B * p.Hu), 1);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;

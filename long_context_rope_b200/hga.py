@@ -24,6 +24,7 @@ HGA_BF16, HGA_F32 = 0, 1
 HGA_KV_FULL, HGA_KV_WINDOWS = 0, 1
 HGA_SUMMARY_F32, HGA_SUMMARY_BF16 = 0, 1
 HGA_KV_AS_DTYPE, HGA_KV_E4M3 = 0, 1
+HGA_ROUTE_PER_KV_HEAD, HGA_ROUTE_PER_Q_HEAD = 0, 1
 STATUS = {0: "HGA_OK", -1: "HGA_ERR_NULL", -2: "HGA_ERR_SHAPE", -3: "HGA_ERR_ALIGN",
           -4: "HGA_ERR_CONFIG", -5: "HGA_ERR_CUDA", -6: "HGA_ERR_DEVICE_INDEX",
           -7: "HGA_ERR_TIMEOUT", -8: "HGA_ERR_UNSUPPORTED", -9: "HGA_ERR_MEMORY",
@@ -44,7 +45,7 @@ class HgaConfig(ctypes.Structure):
         "n_high_freq_pairs")] + [("rope_theta", ctypes.c_double)] + [
         (n, ctypes.c_int32) for n in ("dtype", "q_begin", "q_len", "kv_layout", "summary_type",
                                       "kv_type")] + [
-        ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
+        ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float), ("routing", ctypes.c_int32)]
 
     @property
     def n_chunks(self) -> int:
@@ -55,6 +56,11 @@ class HgaConfig(ctypes.Structure):
         if self.q_len <= 0:
             return 0
         return (self.q_begin + self.q_len - 1) // self.chunk_size - self.q_begin // self.chunk_size + 1
+
+    @property
+    def route_heads(self) -> int:
+        """Rows of q-bar and of the selection lists per sequence."""
+        return self.n_q_heads if self.routing == HGA_ROUTE_PER_Q_HEAD else self.n_kv_heads
 
     @property
     def group_size(self) -> int:
@@ -134,6 +140,7 @@ def config_from(w, **overrides) -> HgaConfig:
     c.summary_type = HGA_SUMMARY_F32
     c.kv_type = HGA_KV_AS_DTYPE
     c.k_scale = c.v_scale = 1.0
+    c.routing = HGA_ROUTE_PER_KV_HEAD
     for k, v in overrides.items():
         setattr(c, k, v)
     return c
@@ -197,43 +204,46 @@ def build_summaries(cfg: HgaConfig, k_raw, chunk_sum, group_sum, k_rot=None, chu
 def route_chunks(cfg: HgaConfig, q_rot, chunk_sum, qbar, sel_chunks, n_sel_chunks, scores=None,
                  stream=None) -> None:
     B, H, d, nQC = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.n_qchunks
+    R = cfg.route_heads
     _check(_lib.hga_route_chunks(
         ctypes.byref(cfg), _ptr(q_rot, "q_rot", cfg.torch_dtype(),
                                 (B, cfg.q_len, cfg.n_q_heads, d)),
         _ptr(chunk_sum, "chunk_sum", cfg.summary_torch_dtype(), (B, H, cfg.n_chunks, d)),
-        _ptr(qbar, "qbar", torch.float32, (B, H, nQC, d)),
-        _ptr(sel_chunks, "sel_chunks", torch.int32, (B, H, nQC, cfg.top_k_chunks)),
-        _ptr(n_sel_chunks, "n_sel_chunks", torch.int32, (B, H, nQC)),
-        _ptr(scores, "scores", torch.float32, (B, H, nQC, cfg.n_chunks), nullable=True),
+        _ptr(qbar, "qbar", torch.float32, (B, R, nQC, d)),
+        _ptr(sel_chunks, "sel_chunks", torch.int32, (B, R, nQC, cfg.top_k_chunks)),
+        _ptr(n_sel_chunks, "n_sel_chunks", torch.int32, (B, R, nQC)),
+        _ptr(scores, "scores", torch.float32, (B, R, nQC, cfg.n_chunks), nullable=True),
         _stream(stream)), "hga_route_chunks")
 
 
 def route_groups(cfg: HgaConfig, qbar, group_sum, sel_chunks, n_sel_chunks, sel_groups,
                  n_sel_groups, scores=None, stream=None) -> None:
     B, H, d, nQC, G = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.n_qchunks, cfg.groups_per_chunk
+    R = cfg.route_heads
     _check(_lib.hga_route_groups(
-        ctypes.byref(cfg), _ptr(qbar, "qbar", torch.float32, (B, H, nQC, d)),
+        ctypes.byref(cfg), _ptr(qbar, "qbar", torch.float32, (B, R, nQC, d)),
         _ptr(group_sum, "group_sum", cfg.summary_torch_dtype(), (B, H, cfg.n_chunks * G, d)),
-        _ptr(sel_chunks, "sel_chunks", torch.int32, (B, H, nQC, cfg.top_k_chunks)),
-        _ptr(n_sel_chunks, "n_sel_chunks", torch.int32, (B, H, nQC)),
-        _ptr(sel_groups, "sel_groups", torch.int32, (B, H, nQC, cfg.top_k_groups)),
-        _ptr(n_sel_groups, "n_sel_groups", torch.int32, (B, H, nQC)),
-        _ptr(scores, "scores", torch.float32, (B, H, nQC, cfg.top_k_chunks * G), nullable=True),
+        _ptr(sel_chunks, "sel_chunks", torch.int32, (B, R, nQC, cfg.top_k_chunks)),
+        _ptr(n_sel_chunks, "n_sel_chunks", torch.int32, (B, R, nQC)),
+        _ptr(sel_groups, "sel_groups", torch.int32, (B, R, nQC, cfg.top_k_groups)),
+        _ptr(n_sel_groups, "n_sel_groups", torch.int32, (B, R, nQC)),
+        _ptr(scores, "scores", torch.float32, (B, R, nQC, cfg.top_k_chunks * G), nullable=True),
         _stream(stream)), "hga_route_groups")
 
 
 def _route_ptrs(cfg: HgaConfig, q_rot, chunk_sum, group_sum, qbar, sel_chunks, n_sel_chunks,
                 sel_groups, n_sel_groups):
     B, H, d, nQC, G = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.n_qchunks, cfg.groups_per_chunk
+    R = cfg.route_heads
     return [
         _ptr(q_rot, "q_rot", cfg.torch_dtype(), (B, cfg.q_len, cfg.n_q_heads, d)),
         _ptr(chunk_sum, "chunk_sum", cfg.summary_torch_dtype(), (B, H, cfg.n_chunks, d)),
         _ptr(group_sum, "group_sum", cfg.summary_torch_dtype(), (B, H, cfg.n_chunks * G, d)),
-        _ptr(qbar, "qbar", torch.float32, (B, H, nQC, d)),
-        _ptr(sel_chunks, "sel_chunks", torch.int32, (B, H, nQC, cfg.top_k_chunks)),
-        _ptr(n_sel_chunks, "n_sel_chunks", torch.int32, (B, H, nQC)),
-        _ptr(sel_groups, "sel_groups", torch.int32, (B, H, nQC, cfg.top_k_groups)),
-        _ptr(n_sel_groups, "n_sel_groups", torch.int32, (B, H, nQC)),
+        _ptr(qbar, "qbar", torch.float32, (B, R, nQC, d)),
+        _ptr(sel_chunks, "sel_chunks", torch.int32, (B, R, nQC, cfg.top_k_chunks)),
+        _ptr(n_sel_chunks, "n_sel_chunks", torch.int32, (B, R, nQC)),
+        _ptr(sel_groups, "sel_groups", torch.int32, (B, R, nQC, cfg.top_k_groups)),
+        _ptr(n_sel_groups, "n_sel_groups", torch.int32, (B, R, nQC)),
     ]
 
 
@@ -358,8 +368,8 @@ def attend(cfg: HgaConfig, q_rot, k_res, v_res, sel_groups, n_sel_groups, out, k
         _ptr(v_res, "v_res", kvt, (B, H, res_len, d)),
         _ptr(k_gat, "k_gat", kvt, gat_shape, nullable=True),
         _ptr(v_gat, "v_gat", kvt, gat_shape, nullable=True),
-        _ptr(sel_groups, "sel_groups", torch.int32, (B, H, nQC, cfg.top_k_groups)),
-        _ptr(n_sel_groups, "n_sel_groups", torch.int32, (B, H, nQC)),
+        _ptr(sel_groups, "sel_groups", torch.int32, (B, cfg.route_heads, nQC, cfg.top_k_groups)),
+        _ptr(n_sel_groups, "n_sel_groups", torch.int32, (B, cfg.route_heads, nQC)),
         _ptr(out, "out", dt, q_shape), _stream(stream)), "hga_attend")
 
 

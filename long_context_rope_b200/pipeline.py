@@ -63,7 +63,7 @@ def alloc_summaries(cfg: hga.HgaConfig, device="cuda"):
 
 
 def alloc_route(cfg: hga.HgaConfig, device="cuda", with_scores: bool = False) -> RouteBuffers:
-    B, H, d, nQC = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.n_qchunks
+    B, H, d, nQC = cfg.batch, cfg.route_heads, cfg.head_dim, cfg.n_qchunks
     i32 = dict(dtype=torch.int32, device=device)
     rb = RouteBuffers(
         qbar=torch.empty(B, H, nQC, d, dtype=torch.float32, device=device),

@@ -31,8 +31,10 @@ def test_exports_every_declared_symbol(hga):
 
 
 def test_struct_layout_matches_header(hga):
-    # 12 int32 (48 bytes), a double at offset 48, 6 int32 (80), two floats: 88
-    assert ctypes.sizeof(hga.HgaConfig) == 88
+    # 12 int32 (48 bytes), a double at offset 48, 6 int32 (80), two floats, one
+    # int32 (92), 8-byte aligned: 96
+    assert ctypes.sizeof(hga.HgaConfig) == 96
+    assert hga.HgaConfig.routing.offset == 88
     assert hga.HgaConfig.rope_theta.offset == 48
     assert hga.HgaConfig.summary_type.offset == 72
     assert hga.HgaConfig.kv_type.offset == 76
@@ -75,6 +77,22 @@ def test_fp8_kv_validation_without_gpu(hga):
     # decode span: the host checks pass, so a NULL output is what is reported
     dec = _cfg(hga, q_begin=4095, q_len=1, **ok)
     assert L.hga_attend(by(dec), *attend[:-2], None, None) == -1
+
+
+def test_per_q_head_routing_validation_without_gpu(hga):
+    """Per-query-head routing: the separate routing calls, the gathers and
+    prefill attention refuse it; an unknown routing value is a config error."""
+    L = hga.library()
+    P = 16 * 1024  # never dereferenced: refused on the host
+    by = ctypes.byref
+    assert L.hga_route_chunks(by(_cfg(hga, routing=3)), P, P, P, P, P, None, None) == -4
+    ph = _cfg(hga, q_begin=4095, q_len=1, routing=hga.HGA_ROUTE_PER_Q_HEAD)
+    assert L.hga_route_chunks(by(ph), P, P, P, P, P, None, None) == -8
+    assert L.hga_route_groups(by(ph), P, P, P, P, P, P, None, None) == -8
+    assert L.hga_gather_kv(by(ph), P, P, 0, P, P, P, P, None) == -8
+    attend = [P] * 3 + [None, None] + [P] * 3 + [None]
+    assert L.hga_attend(by(_cfg(hga, routing=hga.HGA_ROUTE_PER_Q_HEAD)), *attend) == -8
+    assert L.hga_attend(by(ph), P, P, P, P, P, P, P, P, None) == -8  # gathered mode
 
 
 def test_tiered_step_validation_without_gpu(hga):
