@@ -38,9 +38,9 @@ TC_TRAFFIC_NOTE = ("ncu dram__bytes_read+write of attend_tc_kernel at 32K contex
                    "(profiles/attend_tc_prefill_32k_ncu.md)")
 PREFILL = "prefill_64k"
 # ":bf16sum" = the same workload with bf16 summary tables; ":fp8kv" = with an
-# FP8 (E4M3) key/value cache
+# FP8 (E4M3) key/value cache; ":perhead" = with per-query-head routing
 DECODES = ("decode_16x32k", "decode_16x32k:bf16sum", "decode_16x32k:fp8kv",
-           "tiered_decode_4x64k")
+           "decode_16x32k:perhead", "tiered_decode_4x64k")
 
 
 def load_peaks():
@@ -258,8 +258,10 @@ def run_decode(name, args, dist):
     w = synth.WORKLOADS[base]
     bf16_sum = variant == "bf16sum"
     fp8_kv = variant == "fp8kv"
+    per_head = variant == "perhead"
     kv_es = 1 if fp8_kv else 2  # bytes per K/V element
-    cfg = hga.config_from(w, summary_type=hga.HGA_SUMMARY_BF16 if bf16_sum else hga.HGA_SUMMARY_F32)
+    cfg = hga.config_from(w, summary_type=hga.HGA_SUMMARY_BF16 if bf16_sum else hga.HGA_SUMMARY_F32,
+                          routing=hga.HGA_ROUTE_PER_Q_HEAD if per_head else hga.HGA_ROUTE_PER_KV_HEAD)
     x = synth.draw(w, seed=dist.seed(args.seed))
     dev = torch.device("cuda", torch.cuda.current_device())
     st = torch.cuda.current_stream()
@@ -350,8 +352,8 @@ def run_decode(name, args, dist):
         del graph
         return times, eager
 
-    # the separate routing calls read fp32 tables only
-    times_sep, eager_sep = (None, None) if bf16_sum else timed(True)
+    # the separate routing calls read fp32 tables of per-KV-head routing only
+    times_sep, eager_sep = (None, None) if bf16_sum or per_head else timed(True)
     times, eager_us = timed(False)
     us = dist.max(float(np.median(times)))
     us_sep = dist.max(float(np.median(times_sep))) if times_sep else None
@@ -369,7 +371,16 @@ def run_decode(name, args, dist):
         warm_info["drifting"] = run_warm_drift(w, args, dist, cfg, cfg_w, cs, gs, k_win, v_win,
                                                k_host, v_host, st)
     n_sel = rb.n_sel_groups.cpu().numpy()
-    moved = int(n_sel.sum()) * 16 * w.head_dim * kv_es * 2  # routed K+V bytes
+    moved = int(n_sel.sum()) * 16 * w.head_dim * kv_es * 2  # routed K+V bytes read
+    if per_head:  # distinct routed groups per (sequence, KV head): the bytes HBM must supply
+        gq = w.n_q_heads // w.n_kv_heads
+        sg = rb.sel_groups.cpu().numpy().reshape(w.batch, w.n_kv_heads, gq, -1)
+        ng = n_sel.reshape(w.batch, w.n_kv_heads, gq)
+        uniq = sum(len(set(int(v) for i in range(gq) for v in sg[b, k, i, :ng[b, k, i]]))
+                   for b in range(w.batch) for k in range(w.n_kv_heads))
+        moved_unique = uniq * 16 * w.head_dim * kv_es * 2
+    else:
+        moved_unique = moved
     recall = planted_recall(w, x["planted"], rb.sel_chunks.cpu().numpy(),
                             rb.n_sel_chunks.cpu().numpy())
     gather_info = None
@@ -421,16 +432,25 @@ def run_decode(name, args, dist):
     se = 2 if bf16_sum else 4  # summary element bytes
     chunk_sums = w.batch * w.n_kv_heads * w.n_chunks * w.head_dim * se
     group_sums = int(rb.n_sel_chunks.cpu().numpy().sum()) * w.groups_per_chunk * w.head_dim * se
+    if per_head:  # distinct selected chunks' group rows per (sequence, KV head)
+        gq = w.n_q_heads // w.n_kv_heads
+        sc = rb.sel_chunks.cpu().numpy().reshape(w.batch, w.n_kv_heads, gq, -1)
+        nc = rb.n_sel_chunks.cpu().numpy().reshape(w.batch, w.n_kv_heads, gq)
+        uc = sum(len(set(int(v) for i in range(gq) for v in sc[b, k, i, :nc[b, k, i]]))
+                 for b in range(w.batch) for k in range(w.n_kv_heads))
+        group_sums = uc * w.groups_per_chunk * w.head_dim * se
     q_o = 2 * w.batch * w.n_q_heads * w.head_dim * 2
     # tiered: the one-launch step reads the routed groups from the host, not
     # from HBM (the three-launch path also writes and reads them in a buffer)
-    hbm_bytes = forced_kv + chunk_sums + group_sums + q_o + (0 if w.tiered else moved)
+    hbm_bytes = forced_kv + chunk_sums + group_sums + q_o + (0 if w.tiered else moved_unique)
     return dict(workload=name, summary_tables="bf16" if bf16_sum else "fp32",
-                kv_cache="e4m3" if fp8_kv else "bf16", us_per_step=us, us_min=float(np.min(times)), steps=K,
+                kv_cache="e4m3" if fp8_kv else "bf16",
+                routing="per query head" if per_head else "per KV head", us_per_step=us, us_min=float(np.min(times)), steps=K,
                 hbm_bytes_per_step=hbm_bytes, hbm_gbs=hbm_bytes / (us * 1e-6) / 1e9,
                 hbm_frac=hbm_bytes / (us * 1e-6) / 1e9 / load_peaks()["hbm"],
                 us_per_step_eager=eager_us, cuda_graph=True,
                 launches_per_step=launches, routed_kv_bytes=moved,
+                routed_kv_bytes_distinct=moved_unique,
                 us_per_step_separate_kernels=us_sep, us_per_step_separate_eager=eager_sep,
                 launches_per_step_separate=launches_sep, warm_tier=warm_info,
                 gather=gather_info, planted_recall=recall,
@@ -500,7 +520,7 @@ def planted_recall(w, planted, sel_chunks: np.ndarray, n_sel_chunks: np.ndarray)
             j = j0 + jj
             if jj >= sel_chunks.shape[2]:
                 continue
-            for h in range(w.n_kv_heads):
+            for h in range(sel_chunks.shape[1]):  # KV heads, or query heads (per-head routing)
                 sel = set(sel_chunks[b, h, jj, :n_sel_chunks[b, h, jj]].tolist())
                 for c in srcs:
                     forced = c < w.n_sink or j - w.n_local <= c <= j

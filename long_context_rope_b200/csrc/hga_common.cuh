@@ -81,6 +81,15 @@ __device__ __forceinline__ void rope_cs(double pos, double inv_freq, float& c, f
     __sincosf((float)r, &s, &c);
 }
 
+// The first 1024-byte-aligned shared address at or after p (dynamic shared
+// memory), formed by pointer arithmetic on p so that the compiler still knows
+// every access through the result is a shared-memory access (a round trip
+// through an integer would make them generic accesses).
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* p) {
+    const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+    return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);

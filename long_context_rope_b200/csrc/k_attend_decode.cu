@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
     __nv_bfloat16* __restrict__ out, int gathered) {
     extern __shared__ uint8_t smem_raw[];
     DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+        align_smem_1024(smem_raw));
     cg::cluster_group cluster = cg::this_cluster();
     const int CL = (int)cluster.num_blocks();
     const int r = (int)cluster.block_rank();

@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                                                                int n_units) {
     extern __shared__ uint8_t smem_raw[];
     TcSmem& sm = *reinterpret_cast<TcSmem*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+        align_smem_1024(smem_raw));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int span_end = p.q_begin + p.q_len;
 

@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     const uint4* __restrict__ k_host, const uint4* __restrict__ v_host) {
     extern __shared__ uint8_t smem_raw[];
     StepSmem& sm = *reinterpret_cast<StepSmem*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+        align_smem_1024(smem_raw));
     cg::cluster_group cluster = cg::this_cluster();
     const int CL = (int)cluster.num_blocks();
     const int r = (int)cluster.block_rank();
