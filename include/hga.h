@@ -365,6 +365,13 @@ hga_status hga_get_device_error(void* stream, int32_t* detail_out);
  * the default limit. */
 void hga_set_wait_limit_ns(uint64_t limit_ns);
 
+/* The cudaError_t (as an int) of the last failed CUDA call that made a
+ * library call of this host thread return HGA_ERR_CUDA; 0 if there was none. */
+int32_t hga_last_cuda_error(void);
+
+/* CUDA's description of a cudaError_t value (hga_last_cuda_error). Never NULL. */
+const char* hga_cuda_error_string(int32_t cuda_error);
+
 /* Library version as major * 10000 + minor * 100 + patch. */
 int32_t hga_version(void);
 

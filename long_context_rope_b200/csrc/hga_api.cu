@@ -148,7 +148,15 @@ hga_status make_params(const hga_config* c, Params* p) {
     return HGA_OK;
 }
 
-hga_status launched(cudaError_t e) { return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA; }
+// The last failed CUDA call of this thread that made a call return HGA_ERR_CUDA.
+thread_local int g_last_cuda_error = 0;
+
+hga_status cuda_failed(cudaError_t e) {
+    g_last_cuda_error = (int)e;
+    return HGA_ERR_CUDA;
+}
+
+hga_status launched(cudaError_t e) { return e == cudaSuccess ? HGA_OK : cuda_failed(e); }
 
 // Last step before any launch: attach the current device's error word. (A
 // call's stream must belong to the current device; that is the caller's
@@ -199,6 +207,13 @@ static_assert(offsetof(hga_config, rope_theta) == 48, "hga_config layout is part
 extern "C" {
 
 int32_t hga_version(void) { return 10800; }
+
+int32_t hga_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* hga_cuda_error_string(int32_t cuda_error) {
+    const char* s = cudaGetErrorString((cudaError_t)cuda_error);
+    return s != nullptr ? s : "unknown CUDA error";
+}
 
 void hga_set_wait_limit_ns(uint64_t limit_ns) {
     g_wait_ns.store(limit_ns == 0 ? 1000000000ull : (unsigned long long)limit_ns,
@@ -274,7 +289,7 @@ hga_status hga_route_chunks(const hga_config* cfg, const void* q_rot, const void
     cudaStream_t st = (cudaStream_t)stream;
     if (!route_chunks_fuses_qbar(p)) {
         cudaError_t e = launch_qbar(p, q_rot, qbar_out, st);
-        if (e != cudaSuccess) return HGA_ERR_CUDA;
+        if (e != cudaSuccess) return cuda_failed(e);
     }
     return launched(launch_route_chunks(p, q_rot, qbar_out, (const float*)chunk_sum, sel_chunks,
                                         n_sel_chunks, scores_out, st));
@@ -324,11 +339,11 @@ static hga_status route_separate(const Params& p, const void* q_rot, const void*
                                  int32_t* n_sel_chunks, int32_t* sel_groups,
                                  int32_t* n_sel_groups, cudaStream_t st) {
     if (p.sum_bf16 || p.Hu != p.Hkv) return HGA_ERR_UNSUPPORTED;  // one-launch path only
-    if (!route_chunks_fuses_qbar(p) && launch_qbar(p, q_rot, qbar_out, st) != cudaSuccess)
-        return HGA_ERR_CUDA;
-    if (launch_route_chunks(p, q_rot, qbar_out, (const float*)chunk_sum, sel_chunks, n_sel_chunks,
-                            nullptr, st) != cudaSuccess)
-        return HGA_ERR_CUDA;
+    cudaError_t e = route_chunks_fuses_qbar(p) ? cudaSuccess : launch_qbar(p, q_rot, qbar_out, st);
+    if (e != cudaSuccess) return cuda_failed(e);
+    e = launch_route_chunks(p, q_rot, qbar_out, (const float*)chunk_sum, sel_chunks, n_sel_chunks,
+                            nullptr, st);
+    if (e != cudaSuccess) return cuda_failed(e);
     return launched(launch_route_groups(p, qbar_out, (const float*)group_sum, sel_chunks,
                                         n_sel_chunks, sel_groups, n_sel_groups, nullptr, st));
 }
@@ -555,17 +570,18 @@ hga_status hga_attend(const hga_config* cfg, const void* q_rot, const void* k_re
 
 hga_status hga_get_device_error(void* stream, int32_t* detail_out) {
     if (detail_out) *detail_out = 0;
-    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return HGA_ERR_CUDA;
+    cudaError_t se = cudaStreamSynchronize((cudaStream_t)stream);
+    if (se != cudaSuccess) return cuda_failed(se);
     int* addr = nullptr;
     hga_status s = error_word(&addr);
     if (s != HGA_OK) return s;
     int v = 0;
-    if (cudaMemcpy(&v, addr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
-        return HGA_ERR_CUDA;
+    cudaError_t ce = cudaMemcpy(&v, addr, sizeof(int), cudaMemcpyDeviceToHost);
+    if (ce != cudaSuccess) return cuda_failed(ce);
     if (v == 0) return HGA_OK;
     const int zero = 0;
-    if (cudaMemcpy(addr, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
-        return HGA_ERR_CUDA;
+    ce = cudaMemcpy(addr, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (ce != cudaSuccess) return cuda_failed(ce);
     if (detail_out) *detail_out = v;
     return v == kDevErrTimeout ? HGA_ERR_TIMEOUT : HGA_ERR_DEVICE_INDEX;
 }

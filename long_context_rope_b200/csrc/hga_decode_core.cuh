@@ -41,7 +41,8 @@ namespace dec {
 namespace cg = cooperative_groups;
 
 constexpr int kD = 128;
-constexpr int kStages = 8;                       // ring of key blocks
+constexpr int kStages = 8;                       // ring of key blocks (bf16)
+constexpr int kStagesMax = 16;                   // E4M3: the same bytes hold 16 blocks
 constexpr int kBlkBytes = kGroupRows * kD * 2;   // 4 KiB per block per tensor (bf16)
 constexpr int kBlkBytesF8 = kGroupRows * kD;     // 2 KiB per block per tensor (E4M3)
 constexpr int kConsumers = 8;                    // consumer warps
@@ -61,6 +62,29 @@ struct Ring {
     alignas(1024) uint8_t k[kStages][kBlkBytes];
     alignas(1024) uint8_t v[kStages][kBlkBytes];
 };
+
+// Ring geometry: 8 stages of 4 KiB per tensor (bf16), or 16 stages of 2 KiB
+// (E4M3) in the same bytes, so twice as many E4M3 blocks are in flight.
+// Every stage starts on a 1024-byte boundary (the 128-byte swizzle's period).
+// The stage count must be a multiple of the consumer warps: block i goes to
+// warp i % 8 and stage i % S, so every use of a stage then belongs to one
+// warp, which waits for its phases in order. With another count two warps
+// share a stage, and a warp that reaches its wait for phase k + 2 before
+// phase k + 1 has completed passes the parity wait at once (a parity names
+// only two phases) and reads a stage that is still being refilled.
+template <bool kF8>
+__host__ __device__ constexpr int ring_stages() { return kF8 ? kStagesMax : kStages; }
+static_assert(kStages % kConsumers == 0 && kStagesMax % kConsumers == 0,
+              "ring stages must be a multiple of the consumer warps");
+static_assert(kStagesMax * kBlkBytesF8 == kStages * kBlkBytes, "E4M3 stages fill the ring");
+template <bool kF8>
+__device__ __forceinline__ uint8_t* k_stage(Ring& ring, int s) {
+    return &ring.k[0][0] + s * (kF8 ? kBlkBytesF8 : kBlkBytes);
+}
+template <bool kF8>
+__device__ __forceinline__ uint8_t* v_stage(Ring& ring, int s) {
+    return &ring.v[0][0] + s * (kF8 ? kBlkBytesF8 : kBlkBytes);
+}
 
 // Per-warp accumulator state of the online softmax.
 struct WarpAcc {
@@ -137,10 +161,11 @@ __device__ __forceinline__ bool consume_blocks(const Params& p, const uint32_t (
     const int mq = lane >> 3;
     const int krow = (mq & 1) * 8 + (lane & 7);      // K ldmatrix row
     const int vkey = (mq >> 1) * 8 + (lane & 7);     // V ldmatrix (trans) row
+    constexpr int S = ring_stages<kF8>();
     for (int i = warp; i < nloc; i += kConsumers) {
-        const int s = i % kStages;
+        const int s = i % S;
         const bool got = __all_sync(
-            0xffffffffu, ptx::mbar_wait_bounded(&full[s], (i / kStages) & 1, p.wait_ns));
+            0xffffffffu, ptx::mbar_wait_bounded(&full[s], (i / S) & 1, p.wait_ns));
         if (!got) {
             if (lane == 0) {
                 raise_timeout(p);
@@ -153,7 +178,7 @@ __device__ __forceinline__ bool consume_blocks(const Params& p, const uint32_t (
         if constexpr (kF8) {
             // rows g and g + 8, dims 32j + 8t4 .. +7: 16-byte chunk 2j + t4/2
             // of the row, XOR-swizzled by the row (g and g + 8 alike)
-            const uint8_t* kb = ring.k[s];
+            const uint8_t* kb = k_stage<true>(ring, s);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int off = (((2 * j + (t4 >> 1)) ^ g) << 4) + (t4 & 1) * 8;
@@ -171,7 +196,7 @@ __device__ __forceinline__ bool consume_blocks(const Params& p, const uint32_t (
                 ptx::mma_16816_f16(sacc2, a2, qf[2 * j + 1][0], qf[2 * j + 1][1]);
             }
         } else {
-            const uint32_t kb = ptx::smem_u32(ring.k[s]);
+            const uint32_t kb = ptx::smem_u32(k_stage<false>(ring, s));
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const int chunk = (kk & 3) * 2 + (mq >> 1);
@@ -235,7 +260,7 @@ __device__ __forceinline__ bool consume_blocks(const Params& p, const uint32_t (
             // keys 2t4, 2t4 + 1, 2t4 + 8, 2t4 + 9; dims 8g .. +7 (rows g of
             // the tiles) and 64 + 8g .. +7 (rows g + 8): 16-byte chunk g/2
             // (or 4 + g/2) of the key's row, XOR-swizzled by the key
-            const uint8_t* vb = ring.v[s];
+            const uint8_t* vb = v_stage<true>(ring, s);
             auto ldv = [&](int key, int hi) {
                 const int off = (((hi * 4 + (g >> 1)) ^ (key & 7)) << 4) + (g & 1) * 8;
                 return *reinterpret_cast<const uint2*>(vb + key * 128 + off);
@@ -256,7 +281,7 @@ __device__ __forceinline__ bool consume_blocks(const Params& p, const uint32_t (
                 ptx::mma_16816_f16(acc.o[mt], a, pb0, pb1);
             }
         } else {
-            const uint32_t vb = ptx::smem_u32(ring.v[s]);
+            const uint32_t vb = ptx::smem_u32(v_stage<false>(ring, s));
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
                 const int chunk = (mt & 3) * 2 + (mq & 1);
@@ -390,28 +415,30 @@ __device__ __forceinline__ void issue_block(Ring& ring, uint64_t* full, int s,
                                             int outer) {
     if constexpr (kF8) {
         ptx::mbar_arrive_expect_tx(&full[s], 2 * kBlkBytesF8);
-        ptx::tma_load_3d(ring.k[s], mk, 0, row, outer, &full[s]);
-        ptx::tma_load_3d(ring.v[s], mv, 0, row, outer, &full[s]);
+        ptx::tma_load_3d(k_stage<true>(ring, s), mk, 0, row, outer, &full[s]);
+        ptx::tma_load_3d(v_stage<true>(ring, s), mv, 0, row, outer, &full[s]);
     } else {
         ptx::mbar_arrive_expect_tx(&full[s], 2 * kBlkBytes);
         for (int hf = 0; hf < 2; ++hf) {
-            ptx::tma_load_3d(ring.k[s] + hf * 2048, mk, hf * 64, row, outer, &full[s]);
-            ptx::tma_load_3d(ring.v[s] + hf * 2048, mv, hf * 64, row, outer, &full[s]);
+            ptx::tma_load_3d(k_stage<false>(ring, s) + hf * 2048, mk, hf * 64, row, outer, &full[s]);
+            ptx::tma_load_3d(v_stage<false>(ring, s) + hf * 2048, mv, hf * 64, row, outer, &full[s]);
         }
     }
 }
 
 // Producer thread, before the ring's memory is reused or the CTA exits:
 // waits (bounded) until every block load of the first n_issued ring slots
-// has landed. Slot i used stage i % kStages in phase i / kStages, and a stage
+// has landed. Slot i used stage i % S in phase i / S (S = ring_stages), and a stage
 // is armed again only after its previous phase completed, so the last armed
 // phase of each stage covers all of that stage's copies. False if a copy did
 // not land within the drain limit.
+template <bool kF8>
 __device__ __forceinline__ bool drain_ring(uint64_t* full, int n_issued) {
+    constexpr int S = ring_stages<kF8>();
     bool ok = true;
-    for (int s = 0; s < kStages && s < n_issued; ++s) {
-        const int last = s + ((n_issued - 1 - s) / kStages) * kStages;
-        ok &= ptx::mbar_drain(&full[s], last / kStages);
+    for (int s = 0; s < S && s < n_issued; ++s) {
+        const int last = s + ((n_issued - 1 - s) / S) * S;
+        ok &= ptx::mbar_drain(&full[s], last / S);
     }
     return ok;
 }

@@ -9,9 +9,9 @@
 //
 // One cluster of CL CTAs per (sequence, KV head), CL chosen so the grid
 // fills every SM with two CTAs at once. CTA r owns a contiguous share of the
-// unit's 16-row key blocks and streams them through an 8-stage shared-memory ring
-// filled by TMA (tensor-map tile loads, 128-byte swizzle; one producer
-// thread). Eight consumer warps take every 8th block: S^T[16 keys x 8 heads]
+// unit's 16-row key blocks and streams them through a shared-memory ring
+// (8 stages, or 16 of E4M3 blocks) filled by TMA (tensor-map tile loads,
+// 128-byte swizzle; one producer thread). Eight consumer warps take every 8th block: S^T[16 keys x 8 heads]
 // = K_blk Q^T and O^T[128 dims x 8 heads] += V^T P^T on warp-level bf16 MMA
 // (m16n8k16, fp32 accumulate) with a per-warp online softmax in fp32. The
 // 8 x CL warp partials (max, sum, O) merge through distributed shared memory:
@@ -38,7 +38,7 @@ using dec::kBlkBytes;
 using dec::kConsumers;
 using dec::kD;
 using dec::kMaxCluster;
-using dec::kStages;
+using dec::kStagesMax;
 using dec::kThreads;
 
 struct DecodeMaps {
@@ -53,7 +53,7 @@ struct DecodeSmem {
     dec::Partial cta_part;
     float wgt[kConsumers][8];                    // warp-merge weights
     uint16_t pt[kConsumers][8][16];              // per-warp P transpose buffer
-    uint64_t full[kStages], empty[kStages];
+    uint64_t full[kStagesMax], empty[kStagesMax];
     int blk_row[kMaxBlocks];
     int blk_pos[kMaxBlocks];
     int nb;
@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
         if (lane == 0) {
             sm.nb = nb_w;
             sm.bad = 0;
-            for (int s = 0; s < kStages; ++s) {
+            for (int s = 0; s < kStagesMax; ++s) {
                 ptx::mbar_init(&sm.full[s], 1);
                 ptx::mbar_init(&sm.empty[s], 1);
             }
@@ -103,9 +103,10 @@ __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
         if (lane == 0) {
             int i = 0;
             for (; i < nloc; ++i) {
-                const int s = i % kStages;
-                if (i >= kStages &&
-                    !ptx::mbar_wait_bounded(&sm.empty[s], ((i / kStages) - 1) & 1, p.wait_ns)) {
+                constexpr int kS = dec::ring_stages<kF8>();
+                const int s = i % kS;
+                if (i >= kS &&
+                    !ptx::mbar_wait_bounded(&sm.empty[s], ((i / kS) - 1) & 1, p.wait_ns)) {
                     raise_timeout(p);
                     sm.bad = 1;
                     break;
@@ -117,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
                                  gat ? &maps.v_gat : &maps.v_res, row, (int)(gat ? prob : kvh));
             }
             // every issued load lands before the ring's memory is reused
-            if (!dec::drain_ring(sm.full, i)) {
+            if (!dec::drain_ring<kF8>(sm.full, i)) {
                 raise_timeout(p);
                 sm.bad = 1;
             }

@@ -49,7 +49,7 @@ namespace {
 using dec::kConsumers;
 using dec::kD;
 using dec::kMaxCluster;
-using dec::kStages;
+using dec::kStagesMax;
 using dec::kThreads;
 
 constexpr int kMaxSlice = 512;   // level-1 candidates per CTA
@@ -73,7 +73,7 @@ struct StepSmem {
     dec::Partial cta_part;
     float wgt[kConsumers][8];                    // warp-merge weights
     uint16_t pt[kConsumers][8][16];
-    uint64_t full[kStages], empty[kStages];
+    uint64_t full[kStagesMax], empty[kStagesMax];
     uint64_t key1[kMaxSlice];     // own level-1 candidates
     uint64_t own1[kMaxKc];        // this CTA's level-1 finalists, ascending
     uint64_t f1[kMaxF1];          // level-1 finalists of all CTAs
@@ -197,8 +197,8 @@ __device__ __forceinline__ void copy_host_block(dec::Ring& ring, int s, const ui
         const int idx = lane + 32 * u;               // 16-byte piece of the block
         const int row = idx / kRowPieces, c16 = idx % kRowPieces;
         const int off = (c16 >> 3) * 2048 + row * 128 + (((c16 & 7) ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(ring.k[s] + off) = kr[u];
-        *reinterpret_cast<uint4*>(ring.v[s] + off) = vr[u];
+        *reinterpret_cast<uint4*>(dec::k_stage<kF8>(ring, s) + off) = kr[u];
+        *reinterpret_cast<uint4*>(dec::v_stage<kF8>(ring, s) + off) = vr[u];
     }
     // a later tile load into this stage (async proxy) is ordered after these
     // stores
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
         sm.bad = 0;
         sm.n_win1 = 0;
         sm.n_wl = 0;
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kStagesMax; ++s) {
             ptx::mbar_init(&sm.full[s], 1);
             ptx::mbar_init(&sm.empty[s], 1);
         }
@@ -261,7 +261,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
         sm.blk_row[i] = host_tier ? w * p.C + kGroupRows * gm : sm.blk_pos[i];
     }
     __syncthreads();
-    const int n_pre = nf_loc < kStages ? nf_loc : kStages;
+    constexpr int kS = dec::ring_stages<kF8>();
+    const int n_pre = nf_loc < kS ? nf_loc : kS;
 
     // ---- level-1 slice: the first batch of this warp's chunk-summary rows is
     // requested before q-bar, so the two memory latencies overlap
@@ -449,11 +450,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
         int i = n_pre;
         bool ok = true;
         for (; i < nloc; ++i) {
-            const int s = i % kStages;
-            if (i >= kStages) {
+            const int s = i % kS;
+            if (i >= kS) {
                 bool got = true;
                 if (lane == 0)
-                    got = ptx::mbar_wait_bounded(&sm.empty[s], ((i / kStages) - 1) & 1, p.wait_ns);
+                    got = ptx::mbar_wait_bounded(&sm.empty[s], ((i / kS) - 1) & 1, p.wait_ns);
                 if (!__shfl_sync(0xffffffffu, got, 0)) {
                     ok = false;
                     break;
@@ -476,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
             }
             // every issued load (the early forced blocks included) lands
             // before the ring's memory is reused
-            if (!dec::drain_ring(sm.full, i)) {
+            if (!dec::drain_ring<kF8>(sm.full, i)) {
                 raise_timeout(p);
                 sm.bad = 1;
             }

@@ -34,7 +34,11 @@ STATUS = {0: "HGA_OK", -1: "HGA_ERR_NULL", -2: "HGA_ERR_SHAPE", -3: "HGA_ERR_ALI
 class HgaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {_lib.hga_status_string(status).decode()}")
+        msg = f"{where}: {_lib.hga_status_string(status).decode()}"
+        if status == -5:  # HGA_ERR_CUDA: name the failed CUDA call's error
+            code = int(_lib.hga_last_cuda_error())
+            msg += f" (cudaError {code}: {_lib.hga_cuda_error_string(code).decode()})"
+        super().__init__(msg)
 
 
 class HgaConfig(ctypes.Structure):
@@ -115,6 +119,10 @@ def _load():
     lib.hga_version.restype = ctypes.c_int32
     lib.hga_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.hga_set_wait_limit_ns.restype = None
+    lib.hga_last_cuda_error.argtypes = []
+    lib.hga_last_cuda_error.restype = ctypes.c_int32
+    lib.hga_cuda_error_string.argtypes = [ctypes.c_int32]
+    lib.hga_cuda_error_string.restype = ctypes.c_char_p
     return lib
 
 
