@@ -29,11 +29,11 @@ from long_context_rope_b200 import dist_util, synth  # noqa: E402
 METRIC = "routed attn prefill tok/s & decode µs/step at 64K; % of HBM/TC roofline"
 
 # DRAM bytes (read + write) of one prefill attention launch at 64K context,
-# from an ncu capture of attend_tc_kernel at 32K context (574.3 MB: Q and O
+# from an ncu capture of attend_tc_kernel at 32K context (579.4 MB: Q and O
 # once, K/V from L2) scaled x2 (one unit per query chunk). Valid for the
 # kernel as captured; set to None when attend_tc_kernel changes until it is
 # captured again.
-TC_TRAFFIC_BYTES = 2 * 574.3e6
+TC_TRAFFIC_BYTES = 2 * 579.4e6
 TC_TRAFFIC_NOTE = ("ncu dram__bytes_read+write of attend_tc_kernel at 32K context x2 "
                    "(profiles/attend_tc_prefill_32k_ncu.md)")
 PREFILL = "prefill_64k"

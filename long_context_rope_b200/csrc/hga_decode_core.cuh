@@ -369,41 +369,29 @@ __device__ __forceinline__ void merge_cluster_and_store(const Params& p, cg::clu
                                                         __nv_bfloat16* out) {
     const int CL = (int)cluster.num_blocks();
     const int r = (int)cluster.block_rank();
-    const int tid = threadIdx.x;
-    for (int n = r; n < p.gq; n += CL) {
-        if (tid < kD) {
-            float mc[kMaxCluster], lc[kMaxCluster], oc[kMaxCluster];
-#pragma unroll
-            for (int c = 0; c < kMaxCluster; ++c) {
-                if (c < CL) {
-                    const Partial* rp = cluster.map_shared_rank(&cta_part, c);
-                    mc[c] = rp->m[n];
-                    lc[c] = rp->l[n];
-                    oc[c] = rp->o[n][tid];
-                } else {
-                    mc[c] = -INFINITY;
-                    lc[c] = 0.f;
-                    oc[c] = 0.f;
-                }
+    // all threads over (head of this CTA, dim), so the heads' remote reads
+    // are in flight together; the CTAs' maxima first, then the weighted sums
+    const int nh = (p.gq - r + CL - 1) / CL;  // heads r, r + CL, ... below gq
+    for (int x = threadIdx.x; x < nh * kD; x += blockDim.x) {
+        const int n = r + (x / kD) * CL, d = x % kD;
+        float M = -INFINITY;
+#pragma unroll 4
+        for (int c = 0; c < CL; ++c) M = fmaxf(M, cluster.map_shared_rank(&cta_part, c)->m[n]);
+        float num = 0.f, den = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll 4
+            for (int c = 0; c < CL; ++c) {
+                const Partial* rp = cluster.map_shared_rank(&cta_part, c);
+                const float mc = rp->m[n];
+                const float wgt = mc == -INFINITY ? 0.f : ptx::ex2_approx(mc - M);
+                num = fmaf(wgt, rp->o[n][d], num);
+                den = fmaf(wgt, rp->l[n], den);
             }
-            float M = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < kMaxCluster; ++c) M = fmaxf(M, mc[c]);
-            float num = 0.f, den = 0.f;
-            if (M != -INFINITY) {
-#pragma unroll
-                for (int c = 0; c < kMaxCluster; ++c) {
-                    if (mc[c] == -INFINITY) continue;
-                    const float wgt = ptx::ex2_approx(mc[c] - M);
-                    num = fmaf(wgt, oc[c], num);
-                    den = fmaf(wgt, lc[c], den);
-                }
-            }
-            float o = den > 0.f ? num / den : 0.f;
-            if (p.kv_f8) o *= p.v_scale;
-            out[((int64_t)b * p.q_len * p.Hq + (int64_t)h * p.gq + n) * kD + tid] =
-                __float2bfloat16_rn(o);
         }
+        float o = den > 0.f ? num / den : 0.f;
+        if (p.kv_f8) o *= p.v_scale;
+        out[((int64_t)b * p.q_len * p.Hq + (int64_t)h * p.gq + n) * kD + d] =
+            __float2bfloat16_rn(o);
     }
 }
 

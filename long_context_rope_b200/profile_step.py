@@ -11,8 +11,11 @@ Setup (input draw, query rotation, and for decode the summaries/cache build)
 happens before the steps; each prefill step is summaries -> q-bar ->
 route_chunks -> route_groups -> attend; a decode step over the resident
 cache is one decode_step_kernel launch (--separate: route_chunks ->
-route_groups -> attend), a tiered decode step decode_step_kernel (routing
-only) -> gather -> attend. Kernel names: summaries_kernel, qbar_kernel,
+route_groups -> attend), a tiered decode step one decode_step_kernel launch
+reading the routed groups from host memory (--separate: decode_step_kernel
+routing only -> gather -> attend). Variants of the resident decode:
+--fp8-kv (E4M3 cache), --per-q-head (per-query-head routing),
+--bf16-summaries (bf16 tables). Kernel names: summaries_kernel, qbar_kernel,
 route_chunks_tiled_kernel / route_chunks_kernel, route_groups_kernel,
 attend_tc_kernel / attend_decode_kernel / attend_simt_kernel,
 decode_step_kernel, gather_*_kernel.
@@ -41,13 +44,18 @@ def main():
                     help="decode: routing levels and attention as separate launches")
     ap.add_argument("--seq-len", type=int, default=None, help="override the context length")
     ap.add_argument("--batch", type=int, default=None, help="override the batch")
+    ap.add_argument("--fp8-kv", action="store_true", help="decode: E4M3 key/value cache")
+    ap.add_argument("--per-q-head", action="store_true", help="decode: per-query-head routing")
+    ap.add_argument("--bf16-summaries", action="store_true", help="bf16 summary tables")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
     if args.seq_len is not None:
         w = w.replace(seq_len=args.seq_len)
     if args.batch is not None:
         w = w.replace(batch=args.batch)
-    cfg = hga.config_from(w)
+    cfg = hga.config_from(
+        w, summary_type=hga.HGA_SUMMARY_BF16 if args.bf16_summaries else hga.HGA_SUMMARY_F32,
+        routing=hga.HGA_ROUTE_PER_Q_HEAD if args.per_q_head else hga.HGA_ROUTE_PER_KV_HEAD)
     x = synth.draw(w, seed=0)
     k_raw = x["k_raw"].cuda()
     q_rot = pipeline.rotate_queries(cfg, x["q_raw"].cuda())
@@ -75,11 +83,18 @@ def main():
             cfg_w = cfg.copy(kv_layout=hga.HGA_KV_WINDOWS)
             gat = pipeline.alloc_gathered(cfg)
             for _ in range(args.steps):
-                pipeline.decode(cfg_w, q_rot, cs, gs, k_win, v_win, rb, out, gathered=gat,
-                                k_src=k_host, v_src=v_host, src_is_host=True,
-                                separate=args.separate)
+                if args.separate:
+                    pipeline.decode(cfg_w, q_rot, cs, gs, k_win, v_win, rb, out, gathered=gat,
+                                    k_src=k_host, v_src=v_host, src_is_host=True)
+                else:
+                    pipeline.decode_tiered(cfg_w, q_rot, cs, gs, k_win, v_win, k_host, v_host,
+                                           rb, out)
         else:
             v = x["v"].cuda()
+            if args.fp8_kv:  # the cache as E4M3 codes with a per-tensor scale each
+                k_rot, ks = synth.to_e4m3(k_rot)
+                v, vs = synth.to_e4m3(v)
+                cfg = cfg.copy(kv_type=hga.HGA_KV_E4M3, k_scale=ks, v_scale=vs)
             gat = pipeline.alloc_gathered(cfg) if args.gathered else None
             for _ in range(args.steps):
                 pipeline.decode(cfg, q_rot, cs, gs, k_rot, v, rb, out, gathered=gat,
