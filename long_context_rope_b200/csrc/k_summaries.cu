@@ -219,44 +219,44 @@ __global__ void summaries_kernel(Params p, const T* __restrict__ k_raw, S* __res
 }
 
 // ------------------------------------------------ streaming summaries
-// Form for bf16 keys with d = 128 and 4 groups of 16 rows per chunk (every
-// bf16 workload here). Persistent CTAs walk the (sequence x KV head, chunk)
-// items in order; one thread issues each chunk's rows (64 x 256 contiguous
-// bytes) as one bulk copy into a ring of kSumStages shared-memory stages,
-// so the next chunks' reads are in flight while this one is rotated and
-// summed, and the rotated rows leave as plain coalesced 16-byte stores.
-// Warp k owns group k; lane (r = lane / 8, u = lane % 8) owns pairs
-// 8u .. 8u+7 of tokens 16k + 4i + r (i = 0..3), so one warp-wide 16-byte
-// shared load reads four whole 128-byte half-rows (no bank conflict).
+// Form for bf16 keys with d = 128, 4 groups of 16 rows per chunk and F a
+// multiple of 4 (every bf16 workload here). Persistent CTAs walk the
+// (sequence x KV head, chunk) items in order; one thread issues each chunk's
+// rows (64 x 256 contiguous bytes) as one bulk copy into a ring of
+// kSumStages shared-memory stages, so the next chunk's read is in flight
+// while this one is rotated and summed; the rotated rows leave as plain
+// coalesced 8-byte stores. Warp k owns group k; lane (r = lane / 16,
+// u = lane % 16) owns pairs 4u .. 4u+3 of tokens 16k + 2i + r (i = 0..7), so
+// one warp-wide 8-byte shared load reads two whole 128-byte half-rows (no
+// bank conflict).
 //
 // Angles by the angle-addition formulas, so that no double-precision
-// reduction or special-function op runs per element: a token's rotation is
-// R((c0 + 16k) theta) R(o theta) with o < 16. Per CTA (once) a table holds
-// R(o theta) for o < 16 and R(m theta) for m = 16, 32, 48 (group bases from
-// the chunk base) and m = 7.5, 31.5 (the mean positions of a full group and
-// chunk, from their bases), all from rope_cs. Per item only R(c0 theta) and
-// R((c0 + 32) theta) come from rope_cs; the other bases are one complex
-// product each. A token's rotation is then within about 8e-7 of the exact
-// one (two rope_cs errors of at most 2^-21.4 each plus the product's
-// rounding), far below one bf16 ulp of the rotated key.
+// reduction or special-function op runs per element: a lane's first token
+// is rotated by R((c0 + 16k) theta) R(r theta) and each next one by a further
+// R(2 theta). R(r theta) and R(2 theta) are per-lane constants, and R(m theta)
+// for m = 16, 32, 48 (group bases from the chunk bases) and m = 7.5, 31.5
+// (mean positions of a full group and chunk) a per-CTA table, all from
+// cs_accurate (about one fp32 ulp). Per item only R(c0 theta) and
+// R((c0 + 32) theta) come from rope_cs (within 2^-21.4 absolute); the other
+// bases are one complex product each. Along a lane's 8 tokens the rotation
+// then stays within about 1.5e-6 of the exact one, far below one bf16 ulp of
+// the rotated key (2^-8 relative).
 constexpr int kSumStages = 2;
-constexpr int kSumCtasPerSm = 4;
+constexpr int kSumCtasPerSm = 5;
 constexpr int kSumG = 4;                                  // groups per chunk = warps per CTA
 constexpr int kSumRows = kSumG * kGroupRows;              // 64 rows per chunk
 constexpr int kSumChunkBytes = kSumRows * 128 * 2;        // 16 KiB of bf16 key rows
 constexpr int kSumThreads = 32 * kSumG;
 
-// Rotations (cos, sin) of the 64 pairs, laid out [e/2][u] as float4
-// (cos e, cos e+1, sin e, sin e+1) of the pairs 8u+e and 8u+e+1, ready for
-// the packed fp32x2 operations: the slot a lane (r, u) reads for its pairs
-// 8u + 2q, 8u + 2q + 1 is [q][u], and 8 lanes of one r read 128 bytes.
+// Rotations (cos, sin) of the 64 pairs, laid out [q][u] as float4
+// (cos e, cos e+1, sin e, sin e+1) of the pairs e = 4u + 2q and e + 1, ready
+// for the packed fp32x2 operations: lane u's slots are [0][u] and [1][u].
 struct __align__(16) PairRot {
-    float4 s[4][8];
+    float4 s[2][16];
 };
 enum SumExtra { kX16 = 0, kX32, kX48, kXGroupMean, kXChunkMean, kSumExtras };
 
 struct __align__(16) SumShared {
-    PairRot tab[16];               // R(o theta), o < 16
     PairRot ext[kSumExtras];       // R(16 theta), R(32 theta), R(48 theta), R(7.5 theta), R(31.5 theta)
     PairRot base[2][kSumG];        // per item parity, group k: R((c0 + 16k) theta)
     float gsum[2][kSumG][128];     // per item parity: raw group sums (chunk-sum input)
@@ -267,22 +267,41 @@ constexpr int kSumSmemBytes = kSumStages * kSumChunkBytes + (int)sizeof(SumShare
 static_assert(kSumCtasPerSm * (kSumSmemBytes + 1024) <= 228 * 1024, "CTAs per SM");
 
 bool summaries_stream_supports(const Params& p) {
-    // F a multiple of 8: each lane's 8 pairs are all high- or all low-frequency
-    return p.dtype == HGA_BF16 && p.d == 128 && p.G == kSumG && p.C == kSumRows && p.F % 8 == 0;
+    // F a multiple of 4: each lane's 4 pairs are all high- or all low-frequency
+    return p.dtype == HGA_BF16 && p.d == 128 && p.G == kSumG && p.C == kSumRows && p.F % 4 == 0;
 }
 
 __device__ __forceinline__ float2 get_cs(const PairRot& t, int pr) {
-    const float* v = reinterpret_cast<const float*>(&t.s[(pr & 7) >> 1][pr >> 3]);
+    const float* v = reinterpret_cast<const float*>(&t.s[(pr & 3) >> 1][pr >> 2]);
     return make_float2(v[pr & 1], v[2 + (pr & 1)]);
 }
 __device__ __forceinline__ void put_cs(PairRot& t, int pr, float2 cs) {
-    float* v = reinterpret_cast<float*>(&t.s[(pr & 7) >> 1][pr >> 3]);
+    float* v = reinterpret_cast<float*>(&t.s[(pr & 3) >> 1][pr >> 2]);
     v[pr & 1] = cs.x;
     v[2 + (pr & 1)] = cs.y;
 }
 // R(x) R(y) = R(x + y) on (cos, sin) pairs
 __device__ __forceinline__ float2 rot_mul(float2 x, float2 y) {
     return make_float2(x.x * y.x - x.y * y.y, x.y * y.x + x.x * y.y);
+}
+// (cos, sin) of a small angle a (|a| < 2^20): reduced to [-pi, pi] in double,
+// split into a float head and the float remainder, the library sincosf of
+// the head corrected to first order by the remainder (the remainder's square,
+// below 2^-46, is dropped), so the cast to float costs no accuracy.
+__device__ __forceinline__ float2 cs_accurate(double a) {
+    const double red = fma(-rint(a * 0.15915494309189535), 6.283185307179586, a);
+    const float hi = (float)red, lo = (float)(red - (double)hi);
+    float c, sn;
+    sincosf(hi, &sn, &c);
+    return make_float2(fmaf(-sn, lo, c), fmaf(c, lo, sn));
+}
+
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t x) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x));
+}
+__device__ __forceinline__ uint32_t f2_to_bf16x2(float2 v) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+    return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 __device__ __forceinline__ void store_pair2(float* out, float x0, float x1) {
@@ -296,9 +315,9 @@ __device__ __forceinline__ void store_one(__nv_bfloat16* out, float x) {
     *out = __float2bfloat16_rn(x);
 }
 
-// Summary value of pair pr from its raw sums over n tokens (n >= 1): the
-// mean; the low-frequency pairs (pr >= F) are then rotated by `mean_rot`,
-// the rotation to the mean position.
+// Summary value of pair pr from its raw sums (times 1/n): the mean; the
+// low-frequency pairs (pr >= F) are then rotated by `mean_rot`, the rotation
+// to the mean position.
 __device__ __forceinline__ void summary_pair(const Params& p, int pr, float sa, float sb,
                                              float inv_n, float2 mean_rot, float& oa,
                                              float& ob) {
@@ -326,10 +345,11 @@ template <typename S>
 __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) summaries_stream_kernel(
     Params p, const __nv_bfloat16* __restrict__ k_raw, S* __restrict__ cs, S* __restrict__ gs,
     __nv_bfloat16* __restrict__ k_rot, int chunk_begin, int n_chunks) {
+    using namespace ptx;
     extern __shared__ __align__(16) uint8_t stages[];  // bulk copies need 16-byte alignment
     SumShared& sh = *reinterpret_cast<SumShared*>(stages + kSumStages * kSumChunkBytes);
     const int tid = threadIdx.x, lane = tid & 31, k = tid >> 5;
-    const int r = lane >> 3, u = lane & 7;
+    const int r = lane >> 4, u = lane & 15;
     // item cursor (sequence x KV head, chunk offset), stepped by the grid
     // size without a division per item (B * Hkv * n_chunks < 2^31)
     struct Cursor {
@@ -356,9 +376,9 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) summaries_stream_k
         const int ch = chunk_begin + c.off;
         const uint32_t bytes = (uint32_t)rows_of(ch) * 256u;
         uint64_t* bar = &sh.full[j % kSumStages];
-        ptx::mbar_arrive_expect_tx(bar, bytes);
-        ptx::bulk_g2s(stages + (j % kSumStages) * kSumChunkBytes,
-                      k_raw + ((int64_t)c.bh * p.L + (int64_t)ch * kSumRows) * 128, bytes, bar);
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(stages + (j % kSumStages) * kSumChunkBytes,
+                 k_raw + ((int64_t)c.bh * p.L + (int64_t)ch * kSumRows) * 128, bytes, bar);
     };
     // group bases of an item: thread (pair pr, half h) forms R((c0 + 32h) theta)
     // and its product with R(16 theta)
@@ -366,9 +386,9 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) summaries_stream_k
         if (c.bh >= n_bh) return;
         const int ch = chunk_begin + c.off;
         const int pr = tid & 63, h = tid >> 6;
-        float cs_, sn;
-        rope_cs((double)((int64_t)ch * kSumRows + 2 * kGroupRows * h), p.inv_freq[pr], cs_, sn);
-        const float2 b0 = make_float2(cs_, sn);
+        float c_, sn;
+        rope_cs((double)((int64_t)ch * kSumRows + 2 * kGroupRows * h), p.inv_freq[pr], c_, sn);
+        const float2 b0 = make_float2(c_, sn);
         put_cs(sh.base[parity][2 * h], pr, b0);
         put_cs(sh.base[parity][2 * h + 1], pr, rot_mul(b0, get_cs(sh.ext[kX16], pr)));
     };
@@ -376,126 +396,119 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) summaries_stream_k
     const Cursor first = {(int)blockIdx.x / n_chunks, (int)blockIdx.x % n_chunks};
     Cursor iss = first;  // thread 0: the next item to issue
     if (tid == 0) {
-        for (int s = 0; s < kSumStages; ++s) ptx::mbar_init(&sh.full[s], 1);
-        ptx::fence_mbar_init();
+        for (int s = 0; s < kSumStages; ++s) mbar_init(&sh.full[s], 1);
+        fence_mbar_init();
         sh.abort = 0;
         for (int j = 0; j < kSumStages; ++j) {
             issue(iss, j);
             iss = advance(iss);
         }
     }
-    // the first copies are in flight while the tables are built
-    for (int i = tid; i < (16 + kSumExtras) * 64; i += kSumThreads) {
-        const int o = i >> 6, pr = i & 63;
-        // o < 16: o; then 16, 32, 48, 7.5, 31.5 (the SumExtra order)
-        const double m = o <= 16 + kX48 ? (double)(o < 16 ? o : 16 * (o - 15))
-                                        : (o == 16 + kXGroupMean ? 7.5 : 31.5);
-        float c, sn;
-        rope_cs(m, p.inv_freq[pr], c, sn);
-        put_cs(o < 16 ? sh.tab[o] : sh.ext[o - 16], pr, make_float2(c, sn));
+    // the first copies are in flight while the constants are formed
+    for (int i = tid; i < kSumExtras * 64; i += kSumThreads) {
+        const int x = i >> 6, pr = i & 63;
+        const double m = x <= kX48 ? 16.0 * (x + 1) : (x == kXGroupMean ? 7.5 : 31.5);
+        put_cs(sh.ext[x], pr, cs_accurate(m * p.inv_freq[pr]));
     }
-    __syncthreads();  // tables (make_base reads ext)
+    // this lane's step R(2 theta) and first-token offset R(r theta), pairs
+    // (4u, 4u+1) in [0] and (4u+2, 4u+3) in [1]
+    float2 stc[2], sts[2], ofc[2], ofs[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const float2 s0 = cs_accurate(2.0 * p.inv_freq[4 * u + 2 * q]);
+        const float2 s1 = cs_accurate(2.0 * p.inv_freq[4 * u + 2 * q + 1]);
+        const float2 o0 = cs_accurate((double)r * p.inv_freq[4 * u + 2 * q]);
+        const float2 o1 = cs_accurate((double)r * p.inv_freq[4 * u + 2 * q + 1]);
+        stc[q] = make_float2(s0.x, s1.x);
+        sts[q] = make_float2(s0.y, s1.y);
+        ofc[q] = make_float2(o0.x, o1.x);
+        ofs[q] = make_float2(o0.y, o1.y);
+    }
+    __syncthreads();  // ext (make_base reads it)
     make_base(first, 0);
     __syncthreads();
 
     const bool write_rot = k_rot != nullptr;
+    const bool hi = 4 * u < p.F;  // all 4 of this lane's pairs rotate before averaging
     Cursor cur = first, nxt = advance(first);
     for (int j = 0; cur.bh < n_bh; ++j, cur = nxt, nxt = advance(nxt)) {
         const int64_t bh = cur.bh;
         const int ch = chunk_begin + cur.off;
         const int64_t c0 = (int64_t)ch * kSumRows;
         const int nrows = rows_of(ch);
-        const int st = (int)(j % kSumStages);
-        const bool ok = ptx::mbar_wait_bounded(&sh.full[st], (uint32_t)(j / kSumStages) & 1u,
-                                               p.wait_ns);
+        const int st = j % kSumStages;
+        const bool ok = mbar_wait_bounded(&sh.full[st], (uint32_t)(j / kSumStages) & 1u,
+                                          p.wait_ns);
         if (!ok) {
             *reinterpret_cast<volatile int*>(&sh.abort) = 1;
             raise_timeout(p);
         }
         make_base(nxt, (j + 1) & 1);
 
-        float2 acc0v[4], acc1v[4];  // pairs 8u + 2q, 8u + 2q + 1: a half, b half
+        float2 acc0[2], acc1[2];  // raw sums of pairs (4u + 2q, +1): a half, b half
 #pragma unroll
-        for (int q = 0; q < 4; ++q) acc0v[q] = acc1v[q] = make_float2(0.f, 0.f);
+        for (int q = 0; q < 2; ++q) acc0[q] = acc1[q] = make_float2(0.f, 0.f);
         const PairRot& bk = sh.base[j & 1][k];
         if (ok) {
             const uint8_t* sb = stages + st * kSumChunkBytes;
-            float4 bq[4];
+            // rotation of this lane's first token: R((c0 + 16k) theta) R(r theta)
+            float2 rc[2], rs[2];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) bq[q] = bk.s[q][u];
-            const bool hi = 8 * u < p.F;  // F is a multiple of 8 here: all 8 pairs alike
-            __nv_bfloat16* orow =
-                k_rot + (bh * p.L + c0 + kGroupRows * k + r) * 128 + 8 * u;
+            for (int q = 0; q < 2; ++q) {
+                const float4 b4 = bk.s[q][u];
+                const float2 bc = make_float2(b4.x, b4.y), bs = make_float2(b4.z, b4.w);
+                rc[q] = sub2(mul2(bc, ofc[q]), mul2(bs, ofs[q]));
+                rs[q] = fma2(bs, ofc[q], mul2(bc, ofs[q]));
+            }
+            __nv_bfloat16* orow = k_rot + (bh * p.L + c0 + kGroupRows * k + r) * 128 + 4 * u;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int o = kGroupRows * k + 4 * i + r;
+            for (int i = 0; i < 8; ++i) {
+                const int o = kGroupRows * k + 2 * i + r;
                 if (o < nrows) {
-                    float a[8], b[8];
-                    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sb + o * 256 + u * 16), a);
-                    bf16x8_to_f32(*reinterpret_cast<const uint4*>(sb + o * 256 + 128 + u * 16), b);
-                    float ra[8], rb[8];
+                    const uint2 va = *reinterpret_cast<const uint2*>(sb + o * 256 + u * 8);
+                    const uint2 vb = *reinterpret_cast<const uint2*>(sb + o * 256 + 128 + u * 8);
+                    const float2 av[2] = {bf16x2_to_f2(va.x), bf16x2_to_f2(va.y)};
+                    const float2 bv[2] = {bf16x2_to_f2(vb.x), bf16x2_to_f2(vb.y)};
+                    float2 xa[2], xb[2];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        // two pairs at once: R = R(base) R(o theta), then R applied to (a, b)
-                        using namespace ptx;
-                        const float4 t = sh.tab[4 * i + r].s[q][u];
-                        const float2 tc = make_float2(t.x, t.y), ts = make_float2(t.z, t.w);
-                        const float2 bc = make_float2(bq[q].x, bq[q].y);
-                        const float2 bs = make_float2(bq[q].z, bq[q].w);
-                        const float2 c = sub2(mul2(bc, tc), mul2(bs, ts));
-                        const float2 sn = fma2(bs, tc, mul2(bc, ts));
-                        const float2 av = make_float2(a[2 * q], a[2 * q + 1]);
-                        const float2 bv = make_float2(b[2 * q], b[2 * q + 1]);
-                        const float2 xa = sub2(mul2(av, c), mul2(bv, sn));
-                        const float2 xb = fma2(av, sn, mul2(bv, c));
-                        ra[2 * q] = xa.x;
-                        ra[2 * q + 1] = xa.y;
-                        rb[2 * q] = xb.x;
-                        rb[2 * q + 1] = xb.y;
+                    for (int q = 0; q < 2; ++q) {
+                        xa[q] = sub2(mul2(av[q], rc[q]), mul2(bv[q], rs[q]));
+                        xb[q] = fma2(av[q], rs[q], mul2(bv[q], rc[q]));
                         if (hi) {
-                            acc0v[q] = add2(acc0v[q], xa);
-                            acc1v[q] = add2(acc1v[q], xb);
+                            acc0[q] = add2(acc0[q], xa[q]);
+                            acc1[q] = add2(acc1[q], xb[q]);
                         } else {
-                            acc0v[q] = add2(acc0v[q], av);
-                            acc1v[q] = add2(acc1v[q], bv);
+                            acc0[q] = add2(acc0[q], av[q]);
+                            acc1[q] = add2(acc1[q], bv[q]);
                         }
                     }
                     if (write_rot) {
-                        *reinterpret_cast<uint4*>(orow + 4 * 128 * i) = f32x8_to_bf16(ra);
-                        *reinterpret_cast<uint4*>(orow + 4 * 128 * i + 64) = f32x8_to_bf16(rb);
+                        *reinterpret_cast<uint2*>(orow + 2 * 128 * i) =
+                            make_uint2(f2_to_bf16x2(xa[0]), f2_to_bf16x2(xa[1]));
+                        *reinterpret_cast<uint2*>(orow + 2 * 128 * i + 64) =
+                            make_uint2(f2_to_bf16x2(xb[0]), f2_to_bf16x2(xb[1]));
+                    }
+                }
+                if (i < 7) {  // on to token o + 2
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const float2 nc = sub2(mul2(rc[q], stc[q]), mul2(rs[q], sts[q]));
+                        rs[q] = fma2(rs[q], stc[q], mul2(rc[q], sts[q]));
+                        rc[q] = nc;
                     }
                 }
             }
         }
-        // group sums: reduce-scatter over r (lane bits 4, 3); lane (r, u)
-        // ends with pairs 8u + 2r + {0, 1}
-        float acc0[8], acc1[8];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            acc0[2 * q] = acc0v[q].x;
-            acc0[2 * q + 1] = acc0v[q].y;
-            acc1[2 * q] = acc1v[q].x;
-            acc1[2 * q + 1] = acc1v[q].y;
-        }
-        const bool hiA = (lane >> 4) & 1, hiB = (lane >> 3) & 1;
-        float x0[4], x1[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float k0 = hiA ? acc0[q + 4] : acc0[q], s0 = hiA ? acc0[q] : acc0[q + 4];
-            const float k1 = hiA ? acc1[q + 4] : acc1[q], s1 = hiA ? acc1[q] : acc1[q + 4];
-            x0[q] = k0 + __shfl_xor_sync(0xffffffffu, s0, 16);
-            x1[q] = k1 + __shfl_xor_sync(0xffffffffu, s1, 16);
-        }
-        float y0[2], y1[2];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const float k0 = hiB ? x0[q + 2] : x0[q], s0 = hiB ? x0[q] : x0[q + 2];
-            const float k1 = hiB ? x1[q + 2] : x1[q], s1 = hiB ? x1[q] : x1[q + 2];
-            y0[q] = k0 + __shfl_xor_sync(0xffffffffu, s0, 8);
-            y1[q] = k1 + __shfl_xor_sync(0xffffffffu, s1, 8);
-        }
+        // group sums: reduce-scatter over r (lane bit 4); lane (r, u) ends
+        // with the pairs 4u + 2r and 4u + 2r + 1
+        const float2 ka = r ? acc0[1] : acc0[0], sa_ = r ? acc0[0] : acc0[1];
+        const float2 kb = r ? acc1[1] : acc1[0], sb_ = r ? acc1[0] : acc1[1];
+        const float2 ya = add2(ka, make_float2(__shfl_xor_sync(0xffffffffu, sa_.x, 16),
+                                               __shfl_xor_sync(0xffffffffu, sa_.y, 16)));
+        const float2 yb = add2(kb, make_float2(__shfl_xor_sync(0xffffffffu, sb_.x, 16),
+                                               __shfl_xor_sync(0xffffffffu, sb_.y, 16)));
         {
-            const int pr = 8 * u + 2 * r;
+            const int pr = 4 * u + 2 * r;
             const int left = nrows - kGroupRows * k;
             const int n = left <= 0 ? 0 : (left >= kGroupRows ? kGroupRows : left);
             float oa0 = 0.f, ob0 = 0.f, oa1 = 0.f, ob1 = 0.f;
@@ -503,11 +516,11 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) summaries_stream_k
                 const float inv_n = __frcp_rn((float)n);
                 const int64_t g0 = c0 + kGroupRows * k;
                 const float4 bb = bk.s[r][u], xx = sh.ext[kXGroupMean].s[r][u];
-                summary_pair(p, pr, y0[0], y1[0], inv_n,
+                summary_pair(p, pr, ya.x, yb.x, inv_n,
                              mean_rotation(p, pr, g0, n, kGroupRows, make_float2(bb.x, bb.z),
                                            make_float2(xx.x, xx.z)),
                              oa0, ob0);
-                summary_pair(p, pr + 1, y0[1], y1[1], inv_n,
+                summary_pair(p, pr + 1, ya.y, yb.y, inv_n,
                              mean_rotation(p, pr + 1, g0, n, kGroupRows, make_float2(bb.y, bb.w),
                                            make_float2(xx.y, xx.w)),
                              oa1, ob1);
@@ -515,8 +528,8 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) summaries_stream_k
             S* out = gs + ((bh * p.nC + ch) * kSumG + k) * (int64_t)128;
             store_pair2(out + pr, oa0, oa1);
             store_pair2(out + 64 + pr, ob0, ob1);
-            *reinterpret_cast<float2*>(&sh.gsum[j & 1][k][pr]) = make_float2(y0[0], y0[1]);
-            *reinterpret_cast<float2*>(&sh.gsum[j & 1][k][64 + pr]) = make_float2(y1[0], y1[1]);
+            *reinterpret_cast<float2*>(&sh.gsum[j & 1][k][pr]) = ya;
+            *reinterpret_cast<float2*>(&sh.gsum[j & 1][k][64 + pr]) = yb;
         }
         __syncthreads();  // stage st read; gsum[j & 1] and base[(j + 1) & 1] written
         if (*reinterpret_cast<volatile int*>(&sh.abort)) {
@@ -525,7 +538,7 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) summaries_stream_k
             if (tid == 0) {
                 Cursor c = cur;
                 for (int jj = j; jj < j + kSumStages && c.bh < n_bh; ++jj, c = advance(c))
-                    ptx::mbar_drain(&sh.full[jj % kSumStages], jj / kSumStages);
+                    mbar_drain(&sh.full[jj % kSumStages], jj / kSumStages);
             }
             return;
         }
