@@ -329,63 +329,79 @@ __device__ __forceinline__ void store_warp_partial(const WarpAcc& acc, Partial& 
     }
 }
 
-// All threads of the CTA: merge the 8 warp partials into cta. First the
-// per-(warp, head) weights 2^(m_w - M) and the merged max and sum (64 + 8
-// threads), then the weighted sums of O; wgt is an 8 x 8 scratch. Ends with
-// the CTA's barrier.
-__device__ __forceinline__ void merge_warps(const Partial* warp_part, Partial& cta,
-                                            float (*wgt)[8]) {
+// The heads a CTA finalises: CTA r of a cluster of CL owns heads r, r + CL,
+// ... (below gq); every CTA of the cluster writes its merged partial of such
+// a head into the owner's Owned buffer, slot src * owned_per_cta(CL) + n / CL.
+// CL * ceil(8 / CL) <= kOwnSlots for every CL <= 16. The buffer must not
+// share memory with the ring: a peer may write it while this CTA still
+// consumes blocks.
+constexpr int kOwnSlots = 16;
+__host__ __device__ constexpr int owned_per_cta(int CL) { return (8 + CL - 1) / CL; }
+static_assert(kMaxCluster * owned_per_cta(kMaxCluster) <= kOwnSlots, "owned slots");
+
+struct Owned {
+    float m[kOwnSlots], l[kOwnSlots];  // per slot: max, sum
+    float o[kOwnSlots][kD];            // per slot: un-normalised O
+};
+
+// All threads of CTA r: merge the 8 warp partials of each head n < gq (max
+// M, weights 2^(m_w - M), weighted sums of l and O) and write the result
+// straight into the Owned buffer of the head's owner (CTA n % CL) through
+// distributed shared memory. wgt is an 8 x 8 scratch. The caller's cluster
+// barrier then publishes these writes to the owners.
+__device__ __forceinline__ void merge_warps_push(const Partial* warp_part, cg::cluster_group& cluster,
+                                                 Owned& owned, float (*wgt)[8], int gq) {
     const int t = threadIdx.x;
-    if (t < 8 * kConsumers) {
-        const int w = t >> 3, n = t & 7;
+    const int CL = (int)cluster.num_blocks();
+    const int r = (int)cluster.block_rank();
+    const int per = owned_per_cta(CL);
+    if (t < gq) {
+        const int n = t;
         float M = -INFINITY;
 #pragma unroll
-        for (int v = 0; v < kConsumers; ++v) M = fmaxf(M, warp_part[v].m[n]);
-        const float mw = warp_part[w].m[n];
-        wgt[w][n] = (M == -INFINITY || mw == -INFINITY) ? 0.f : ptx::ex2_approx(mw - M);
-        if (w == 0) cta.m[n] = M;
-    }
-    __syncthreads();
-    if (t < 8) {
+        for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, warp_part[w].m[n]);
         float den = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumers; ++w) den = fmaf(wgt[w][t], warp_part[w].l[t], den);
-        cta.l[t] = den;
+        for (int w = 0; w < kConsumers; ++w) {
+            const float mw = warp_part[w].m[n];
+            const float wt = (M == -INFINITY || mw == -INFINITY) ? 0.f : ptx::ex2_approx(mw - M);
+            wgt[w][n] = wt;
+            den = fmaf(wt, warp_part[w].l[n], den);
+        }
+        Owned* dst = cluster.map_shared_rank(&owned, n % CL);
+        dst->m[r * per + n / CL] = M;
+        dst->l[r * per + n / CL] = den;
     }
-    for (int x = t; x < 8 * kD; x += blockDim.x) {
+    __syncthreads();
+    for (int x = t; x < gq * kD; x += blockDim.x) {
         const int n = x / kD, d = x % kD;
         float num = 0.f;
 #pragma unroll
         for (int w = 0; w < kConsumers; ++w) num = fmaf(wgt[w][n], warp_part[w].o[n][d], num);
-        cta.o[n][d] = num;
+        cluster.map_shared_rank(&owned, n % CL)->o[r * per + n / CL][d] = num;
     }
-    __syncthreads();
 }
 
-// After a cluster barrier: CTA r merges the CL CTA partials of heads
-// r, r + CL, ... and writes the normalised output rows (bf16).
-__device__ __forceinline__ void merge_cluster_and_store(const Params& p, cg::cluster_group& cluster,
-                                                        Partial& cta_part, int b, int h,
-                                                        __nv_bfloat16* out) {
-    const int CL = (int)cluster.num_blocks();
-    const int r = (int)cluster.block_rank();
-    // all threads over (head of this CTA, dim), so the heads' remote reads
-    // are in flight together; the CTAs' maxima first, then the weighted sums
+// After the cluster barrier that published merge_warps_push's writes: CTA r
+// merges the CL partials of each head it owns and writes the normalised
+// output rows (bf16). It reads only its own shared memory, so no CTA waits
+// for another afterwards.
+__device__ __forceinline__ void merge_owned_and_store(const Params& p, int CL, int r,
+                                                      const Owned& owned, int b, int h,
+                                                      __nv_bfloat16* out) {
+    const int per = owned_per_cta(CL);
     const int nh = (p.gq - r + CL - 1) / CL;  // heads r, r + CL, ... below gq
     for (int x = threadIdx.x; x < nh * kD; x += blockDim.x) {
-        const int n = r + (x / kD) * CL, d = x % kD;
+        const int k = x / kD, d = x % kD, n = r + k * CL;
         float M = -INFINITY;
-#pragma unroll 4
-        for (int c = 0; c < CL; ++c) M = fmaxf(M, cluster.map_shared_rank(&cta_part, c)->m[n]);
+        for (int c = 0; c < CL; ++c) M = fmaxf(M, owned.m[c * per + k]);
         float num = 0.f, den = 0.f;
         if (M != -INFINITY) {
-#pragma unroll 4
             for (int c = 0; c < CL; ++c) {
-                const Partial* rp = cluster.map_shared_rank(&cta_part, c);
-                const float mc = rp->m[n];
+                const float mc = owned.m[c * per + k];
                 const float wgt = mc == -INFINITY ? 0.f : ptx::ex2_approx(mc - M);
-                num = fmaf(wgt, rp->o[n][d], num);
-                den = fmaf(wgt, rp->l[n], den);
+                num = fmaf(wgt, owned.o[c * per + k][d], num);
+                den = fmaf(wgt, owned.l[c * per + k], den);
             }
         }
         float o = den > 0.f ? num / den : 0.f;

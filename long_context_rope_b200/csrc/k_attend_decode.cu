@@ -50,7 +50,7 @@ struct DecodeSmem {
         dec::Ring ring;
         dec::Partial warp_part[kConsumers];      // reused once the ring is drained
     } u;
-    dec::Partial cta_part;
+    dec::Owned owned;                            // partials of the heads this CTA finalises
     float wgt[kConsumers][8];                    // warp-merge weights
     uint16_t pt[kConsumers][8][16];              // per-warp P transpose buffer
     uint64_t full[kStagesMax], empty[kStagesMax];
@@ -139,10 +139,10 @@ __global__ void __launch_bounds__(kThreads, 2) attend_decode_kernel(
     // ---- per-warp partials -> shared memory (the ring's space is reused)
     if (warp < kConsumers) dec::store_warp_partial<kF8>(acc, sm.u.warp_part[warp]);
     __syncthreads();
-    dec::merge_warps(sm.u.warp_part, sm.cta_part, sm.wgt);
-    cluster.sync();
-    dec::merge_cluster_and_store(p, cluster, sm.cta_part, b, h, out);
-    cluster.sync();
+    dec::merge_warps_push(sm.u.warp_part, cluster, sm.owned, sm.wgt, p.gq);
+    cluster.sync();  // every partial is in its owner's shared memory
+    dec::merge_owned_and_store(p, (int)cluster.num_blocks(), (int)cluster.block_rank(), sm.owned, b,
+                               h, out);
 }
 
 std::mutex g_decode_mu;

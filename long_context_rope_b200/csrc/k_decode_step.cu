@@ -70,7 +70,7 @@ struct StepSmem {
         dec::Ring ring;
         dec::Partial warp_part[kConsumers];
     } u;
-    dec::Partial cta_part;
+    dec::Owned owned;                            // partials of the heads this CTA finalises
     float wgt[kConsumers][8];                    // warp-merge weights
     uint16_t pt[kConsumers][8][16];
     uint64_t full[kStagesMax], empty[kStagesMax];
@@ -78,7 +78,7 @@ struct StepSmem {
     uint64_t own1[kMaxKc];        // this CTA's level-1 finalists, ascending
     alignas(16) uint64_t f1[kMaxF1];          // level-1 finalists of all CTAs
     alignas(16) uint64_t key2[kMaxCand2];     // level-2 candidates (all of them, every CTA)
-    int rank[kMaxSlice > kMaxCand2 ? kMaxSlice : kMaxCand2];  // rank scratch
+    int wcnt[2][kConsumers];      // rank_select's per-warp winner counts
     int win1[kMaxKc];             // selected chunks, ascending
     int routed[kMaxKg];           // selected groups, ascending
     int blk_pos[kMaxLocal];       // position of a local block's first key
@@ -93,21 +93,28 @@ __device__ __forceinline__ int index_of(uint64_t k) {
     return 0x7fffffff - (int)(uint32_t)(k & 0xffffffffu);
 }
 
-// Consumer threads (kRankThreads): rank[x] = number of b[0..nb) larger than
-// a[x], for every present a[x] (0 = absent: not ranked, never counted). Two
-// threads share a candidate and each streams every other pair of b through
-// it with 16-byte loads (b 16-byte aligned); the two counts are summed with
-// one shuffle. (Four candidates per thread over eight threads, with 8-byte
-// loads, took twice as long: 2.9-3.9 K cycles against 1.4-1.9 K per rank of
-// 128 keys, measured alone.)
+// Consumer threads (kRankThreads): the exact top k of the present keys
+// a[0..na) (0 = absent, never selected, never counted) by rank = number of
+// b[0..nb) larger; emit(pos, x) receives the winners (rank < k) with
+// positions 0, 1, ... in candidate order, and the count is returned to every
+// consumer thread. Two threads share a candidate and each streams every
+// other pair of b through it with 16-byte loads (b 16-byte aligned); the two
+// counts are summed with one shuffle. (Four candidates per thread over eight
+// threads, with 8-byte loads, took twice as long.) The compaction is
+// stable and parallel: a ballot per warp, the warps' counts through wcnt
+// (2 x kConsumers ints, alternating per 128 candidates) and one named
+// barrier of the consumer warps per 128 candidates.
 constexpr int kRankTpc = 2;
-__device__ __forceinline__ void count_greater(const uint64_t* a, int na, const uint64_t* b,
-                                              int nb, int* rank) {
-    const int t = threadIdx.x;
+constexpr int kRankBarrier = 1;  // named barrier id (0 is __syncthreads)
+template <typename Emit>
+__device__ __forceinline__ int rank_select(const uint64_t* a, int na, const uint64_t* b, int nb,
+                                           int k, int (*wcnt)[kConsumers], Emit emit) {
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int sub = t & (kRankTpc - 1);
     const ulonglong2* b2 = reinterpret_cast<const ulonglong2*>(b);
     const int npairs = nb >> 1;
-    for (int x0 = 0; x0 < na; x0 += kRankThreads / kRankTpc) {
+    int base = 0;
+    for (int x0 = 0, it = 0; x0 < na; x0 += kRankThreads / kRankTpc, ++it) {
         const int x = x0 + t / kRankTpc;
         const uint64_t ax = x < na ? a[x] : 0ull;
         int c = 0;
@@ -118,8 +125,21 @@ __device__ __forceinline__ void count_greater(const uint64_t* a, int na, const u
         }
         if ((nb & 1) && sub == 0) c += b[nb - 1] > ax ? 1 : 0;
         c += __shfl_xor_sync(0xffffffffu, c, 1);
-        if (sub == 0 && x < na && ax != 0ull) rank[x] = c;
+        const bool win = sub == 0 && x < na && ax != 0ull && c < k;
+        const unsigned m = __ballot_sync(0xffffffffu, win);
+        if (lane == 0) wcnt[it & 1][warp] = __popc(m);
+        asm volatile("bar.sync %0, %1;" ::"n"(kRankBarrier), "n"(kRankThreads) : "memory");
+        int before = 0, total = 0;
+#pragma unroll
+        for (int w = 0; w < kConsumers; ++w) {
+            const int cw = wcnt[it & 1][w];
+            before += w < warp ? cw : 0;
+            total += cw;
+        }
+        if (win) emit(base + before + __popc(m & ((1u << lane) - 1u)), x);
+        base += total;
     }
+    return base;
 }
 
 // Elements 4 * lane .. 4 * lane + 3 of a summary row as fp32 (fp32 or bf16
@@ -340,23 +360,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     if (attend && warp == kConsumers && lane == 0)
         for (int i = 0; i < n_pre; ++i)
             dec::issue_block<kF8>(sm.u.ring, sm.full, i, &maps.k, &maps.v, sm.blk_row[i], (int)kvh);
-    if (consumer) count_greater(sm.key1, ns, sm.key1, ns, sm.rank);
-    __syncthreads();
     // this CTA's winners, in candidate (= ascending chunk) order, padded
     // with 0 to cap1 entries. (Prefetching the winners' group rows into L2
     // here, with one bulk prefetch per winner, cost more in this phase than
-    // it saved at level 2: +0.9 against -0.2 us.)
-    if (warp == 0) {
-        int base = 0;
-        for (int x0 = 0; x0 < ns; x0 += 32) {
-            const int x = x0 + lane;
-            const uint64_t k = x < ns ? sm.key1[x] : 0ull;
-            const bool win = k != 0ull && sm.rank[x] < cap1;
-            const unsigned m = __ballot_sync(0xffffffffu, win);
-            if (win) sm.own1[base + __popc(m & ((1u << lane) - 1u))] = k;
-            base += __popc(m);
-        }
-        for (int x = base + lane; x < cap1; x += 32) sm.own1[x] = 0ull;
+    // it saved at level 2: +0.9 against -0.2 us; so did prefetching the
+    // selected chunks' K/V rows after level 1: +4 us, the attention phase
+    // being HBM-bound already.)
+    if (consumer) {
+        const int n1 = rank_select(sm.key1, ns, sm.key1, ns, cap1, sm.wcnt,
+                                   [&](int pos, int x) { sm.own1[pos] = sm.key1[x]; });
+        for (int x = n1 + tid; x < cap1; x += kRankThreads) sm.own1[x] = 0ull;
     }
     cluster.sync();
     // the finalist table: CTA t's winners at slots [t * cap1, (t + 1) * cap1),
@@ -369,19 +382,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     // ---- every CTA ranks the whole finalist table: the global top k_c,
     // compacted in table order, which is ascending chunk order
     const int nF1 = CL * cap1;
-    if (consumer) count_greater(sm.f1, nF1, sm.f1, nF1, sm.rank);
-    __syncthreads();
-    if (warp == 0) {
-        int base = 0;
-        for (int x0 = 0; x0 < nF1; x0 += 32) {
-            const int x = x0 + lane;
-            const uint64_t k = x < nF1 ? sm.f1[x] : 0ull;
-            const bool win = k != 0ull && sm.rank[x] < p.kc;
-            const unsigned m = __ballot_sync(0xffffffffu, win);
-            if (win) sm.win1[base + __popc(m & ((1u << lane) - 1u))] = index_of(k);
-            base += __popc(m);
-        }
-        if (lane == 0) sm.n_win1 = base;
+    if (consumer) {
+        const int n = rank_select(sm.f1, nF1, sm.f1, nF1, p.kc, sm.wcnt,
+                                  [&](int pos, int x) { sm.win1[pos] = index_of(sm.f1[x]); });
+        if (tid == 0) sm.n_win1 = n;
     }
     __syncthreads();
     const int nsel1 = sm.n_win1;  // min(k_c, number of candidates)
@@ -402,20 +406,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
                            sm.key2[x] = rank_key(score_key32(s), sm.win1[x / p.G] * p.G + x % p.G);
                        });
     __syncthreads();
-    if (consumer) count_greater(sm.key2, n2, sm.key2, n2, sm.rank);
-    __syncthreads();
-    // winners (rank < k_g) in candidate order = ascending group index: one
-    // warp compacts them with ballots
-    if (warp == 0) {
-        int base = 0;
-        for (int x0 = 0; x0 < n2; x0 += 32) {
-            const int x = x0 + lane;
-            const bool win = x < n2 && sm.rank[x] < p.kg;
-            const unsigned m = __ballot_sync(0xffffffffu, win);
-            if (win) sm.routed[base + __popc(m & ((1u << lane) - 1u))] = index_of(sm.key2[x]);
-            base += __popc(m);
-        }
-        if (lane == 0) sm.n_wl = base;
+    // winners (rank < k_g) in candidate order = ascending group index
+    if (consumer) {
+        const int n = rank_select(sm.key2, n2, sm.key2, n2, p.kg, sm.wcnt,
+                                  [&](int pos, int x) { sm.routed[pos] = index_of(sm.key2[x]); });
+        if (tid == 0) sm.n_wl = n;
     }
     __syncthreads();
     const int nw = sm.n_wl;
@@ -423,7 +418,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
         for (int i = tid; i < p.kg; i += blockDim.x) sel_g[prob * p.kg + i] = i < nw ? sm.routed[i] : -1;
         if (tid == 0) nsel_g[prob] = nw;
     }
-    if (!attend) return;  // no distributed shared memory access is pending
+    if (!attend) {
+        // peers read this CTA's finalist table (own1) after the first cluster
+        // barrier; it stays valid until every CTA has passed this one
+        cluster.sync();
+        return;
+    }
 
     // ---- attention over this CTA's forced share, then its routed share
     const int pr = (nw + CL - 1) / CL;
@@ -487,10 +487,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step_kernel(
     __syncthreads();
     if (consumer) dec::store_warp_partial<kF8>(acc, sm.u.warp_part[warp]);
     __syncthreads();
-    dec::merge_warps(sm.u.warp_part, sm.cta_part, sm.wgt);
-    cluster.sync();
-    dec::merge_cluster_and_store(p, cluster, sm.cta_part, b, h, out);
-    cluster.sync();
+    dec::merge_warps_push(sm.u.warp_part, cluster, sm.owned, sm.wgt, p.gq);
+    cluster.sync();  // every partial is in its owner's shared memory
+    dec::merge_owned_and_store(p, (int)cluster.num_blocks(), (int)cluster.block_rank(), sm.owned, b,
+                               h, out);
 }
 
 // Table sizes a cluster of cl CTAs needs; false if one is over its cap.
