@@ -313,9 +313,13 @@ def run_decode(name, args, dist):
     K = max(args.steps, 20)
 
     def timed(separate, warm=False, fn=None):
-        """Median device time of one step replayed from a CUDA graph (L2
-        flushed between steps), plus the eager median for reference. `fn`
-        (no arguments) replaces the step when given."""
+        """Device time of one step, L2 flushed before every step. Primary: one
+        CUDA graph of KP x (flush, step) minus one graph of the same KP
+        flushes, each replayed 5 times between events (medians), over KP: the
+        time a step adds to a stream of device work, its launch following the
+        previous kernel as in a decode loop. Also the median of single graph
+        replays between events after a flush (each then starts on an idle
+        device, launch latency included) and of eager launches."""
         if fn is not None:
             step = lambda separate, warm: fn()  # noqa: E731
         else:
@@ -350,20 +354,48 @@ def run_decode(name, args, dist):
         torch.cuda.synchronize()
         eager = float(np.median([ev2.ms(2 * i, 2 * i + 1) * 1000.0 for i in range(5)]))
         del graph
-        return times, eager
+        KP = 16
+        g_pipe, g_flush = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_pipe, capture_error_mode="relaxed"):
+            for i in range(KP):
+                flush.fill_(i & 0xff)
+                step(separate, warm)
+        with torch.cuda.graph(g_flush, capture_error_mode="relaxed"):
+            for i in range(KP):
+                flush.fill_(i & 0xff)
+
+        def graph_ms(g):
+            g.replay()
+            e = Events(2 * 5)
+            for i in range(5):
+                e.rec(2 * i, st)
+                g.replay()
+                e.rec(2 * i + 1, st)
+            torch.cuda.synchronize()
+            return float(np.median([e.ms(2 * i, 2 * i + 1) for i in range(5)]))
+
+        pipelined = (graph_ms(g_pipe) - graph_ms(g_flush)) * 1000.0 / KP
+        if hga.get_device_error() != 0:
+            raise RuntimeError(f"device error word set in {name} (pipelined graph)")
+        del g_pipe, g_flush
+        return dict(pipelined=pipelined, single=times, eager=eager)
 
     # the separate routing calls read fp32 tables of per-KV-head routing only
-    times_sep, eager_sep = (None, None) if bf16_sum or per_head else timed(True)
-    times, eager_us = timed(False)
-    us = dist.max(float(np.median(times)))
-    us_sep = dist.max(float(np.median(times_sep))) if times_sep else None
+    t_sep = None if bf16_sum or per_head else timed(True)
+    t_one = timed(False)
+    times, eager_us = t_one["single"], t_one["eager"]
+    us = dist.max(t_one["pipelined"])
+    us_single = dist.max(float(np.median(times)))
+    us_sep = dist.max(t_sep["pipelined"]) if t_sep else None
+    eager_sep = t_sep["eager"] if t_sep else None
     warm_info = None
     if w.tiered:
         # steady state of the warm tier for this (fixed) query: its routed groups
         # stay in the pool, so no group crosses the host link after the first step
-        times_warm, _ = timed(False, warm=True)
+        t_warm = timed(False, warm=True)
         hits_misses = pool.stats.cpu().numpy().reshape(-1, 2).sum(0)
-        warm_info = dict(us_per_step=dist.max(float(np.median(times_warm))),
+        warm_info = dict(us_per_step=dist.max(t_warm["pipelined"]),
+                         us_per_step_single_replay=dist.max(float(np.median(t_warm["single"]))),
                          pool_slots=int(pool.tag.shape[-1]),
                          hit_rate=float(hits_misses[0] / max(1, hits_misses.sum())),
                          host_bytes_per_step=int(hits_misses[1]) * 16 * w.head_dim * 2 * 2,
@@ -393,7 +425,7 @@ def run_decode(name, args, dist):
         # the launch latency overlaps the previous launch (the kernel's
         # throughput). Each launch reads and writes every routed group's K
         # and V once.
-        times_g, _ = timed(False, fn=lambda: hga.gather_kv(
+        t_g = timed(False, fn=lambda: hga.gather_kv(
             cfg, k_rot, v, False, rb.sel_groups, rb.n_sel_groups, gat[0], gat[1]))
         sels = []
         for i in range(8):
@@ -415,7 +447,7 @@ def run_decode(name, args, dist):
         if hga.get_device_error() != 0:
             raise RuntimeError("device error word set in the gather run")
         seq_us = dist.max(ev.ms(0, 1) * 1000.0 / n_seq)
-        g_us = dist.max(float(np.median(times_g)))
+        g_us = dist.max(float(np.median(t_g["single"])))
         g_bytes = 2 * moved
         peak = load_peaks()["hbm"]
         gather_info = dict(kernel="gather_hbm_kernel (hga_gather_kv, HBM source)",
@@ -445,7 +477,11 @@ def run_decode(name, args, dist):
     hbm_bytes = forced_kv + chunk_sums + group_sums + q_o + (0 if w.tiered else moved_unique)
     return dict(workload=name, summary_tables="bf16" if bf16_sum else "fp32",
                 kv_cache="e4m3" if fp8_kv else "bf16",
-                routing="per query head" if per_head else "per KV head", us_per_step=us, us_min=float(np.min(times)), steps=K,
+                routing="per query head" if per_head else "per KV head", us_per_step=us,
+                timing="device time a step adds to a CUDA graph of 16 x (L2 flush, step), "
+                       "less the graph of the 16 flushes alone",
+                us_per_step_single_replay=us_single, us_min_single_replay=float(np.min(times)),
+                steps=K,
                 hbm_bytes_per_step=hbm_bytes, hbm_gbs=hbm_bytes / (us * 1e-6) / 1e9,
                 hbm_frac=hbm_bytes / (us * 1e-6) / 1e9 / load_peaks()["hbm"],
                 us_per_step_eager=eager_us, cuda_graph=True,
