@@ -223,15 +223,12 @@ def run_prefill(args, dist, peaks):
     if not args.no_e2e:
         hk, hv, hq = (t.cpu().pin_memory() for t in (k_raw, v, q_rot))
         ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        e_k, e_v, e_q = torch.empty_like(k_raw), torch.empty_like(v), torch.empty_like(q_rot)
-        e_out = torch.empty_like(out)
+        # the public API with host buffers: K, V and Q in, O out over the host
+        # link, overlapped with slice-by-slice routing and attention
+        hp = pipeline.HostPrefill(cfg, chunks_per_slice=64, device=dev)
 
         def e2e_step():
-            e_k.copy_(hk, non_blocking=True)
-            e_v.copy_(hv, non_blocking=True)
-            e_q.copy_(hq, non_blocking=True)
-            pipeline.prefill(cfg, e_k, e_v, e_q, cs, gs, k_rot, rb, e_out)
-            ho.copy_(e_out, non_blocking=True)
+            hp.run(hk, hv, hq, ho)
 
         for _ in range(2):
             e2e_step()

@@ -201,3 +201,99 @@ def decode_append(cfg_cap: hga.HgaConfig, pos: int, k_new_raw, v_new, q_rot_new,
     cfg_q = cfg_cap.copy(q_begin=pos, q_len=1)
     hga.decode_step(cfg_q, q_rot_new, cs, gs, k_rot_cache, v_cache, rb.qbar, rb.sel_chunks,
                     rb.n_sel_chunks, rb.sel_groups, rb.n_sel_groups, out, stream)
+
+
+class HostPrefill:
+    """Prefill whose inputs and output live in (pinned) host memory, with the
+    host-link copies overlapped with the computation.
+
+    The query span is cut into slices of at least `chunks_per_slice` query
+    chunks (all of them if there are fewer), per sequence. One copy stream brings K, then the first slice's queries,
+    then V, then the other slices' queries to the device; the compute stream
+    builds the summaries once K has landed and routes and attends each slice
+    (hga_route and hga_attend on the slice's span, q_begin / q_len) once its
+    queries have landed; a second copy stream returns each slice's output as
+    soon as it is computed. Host-to-device and device-to-host copies use
+    separate copy engines, so after the first slice the link carries both
+    directions at once and the kernels run under the copies. A slice's
+    routing and attention are exactly those of the whole span restricted to
+    its query chunks (every unit is independent), so the output equals the
+    one-call prefill bitwise.
+
+    Device buffers (allocated once, by torch): k_raw, v, q_rot, out of the
+    whole problem, the summaries, the rotated keys and one RouteBuffers per
+    slice. run() enqueues on the caller's current stream and makes it wait
+    for the last output copy."""
+
+    def __init__(self, cfg: hga.HgaConfig, chunks_per_slice: int = 64, device="cuda"):
+        if cfg.q_begin % cfg.chunk_size != 0:
+            raise ValueError("HostPrefill: the span must start on a chunk boundary")
+        self.cfg = cfg
+        B, L, Hq, d = cfg.batch, cfg.q_len, cfg.n_q_heads, cfg.head_dim
+        dt = cfg.kv_torch_dtype()
+        self.k_raw = torch.empty(B, cfg.n_kv_heads, cfg.seq_len, d, dtype=dt, device=device)
+        self.v = torch.empty_like(self.k_raw)
+        self.k_rot = torch.empty_like(self.k_raw)
+        self.q_rot = torch.empty(B, L, Hq, d, dtype=dt, device=device)
+        self.out = torch.empty_like(self.q_rot)
+        self.cs, self.gs = alloc_summaries(cfg, device)
+        self.cfg1 = cfg.copy(batch=1)
+        # slice boundaries on chunk boundaries, about chunks_per_slice query
+        # chunks each and never fewer (so every slice is routed by the same
+        # kernel as the whole span would be)
+        nqc, C = cfg.n_qchunks, cfg.chunk_size
+        n_sl = max(1, nqc // max(1, chunks_per_slice))
+        bounds = [min(L, (i * nqc // n_sl) * C) for i in range(n_sl)] + [L]
+        self.slices = []  # (b, row0, row1, cfg of the span, RouteBuffers)
+        for b in range(B):
+            for r0, r1 in zip(bounds[:-1], bounds[1:]):
+                c = self.cfg1.copy(q_begin=cfg.q_begin + r0, q_len=r1 - r0)
+                self.slices.append((b, r0, r1, c, alloc_route(c, device)))
+        self.s_in = torch.cuda.Stream(device=device)
+        self.s_out = torch.cuda.Stream(device=device)
+
+    def sel_groups_of(self, b: int) -> torch.Tensor:
+        """Group selections of sequence b, all slices' query chunks in order
+        ([Hkv, nQC, k_g], host copy)."""
+        return torch.cat([rb.sel_groups[0].cpu() for (bb, _, _, _, rb) in self.slices if bb == b],
+                         dim=1)
+
+    def run(self, hk, hv, hq, ho):
+        """hk, hv [B, Hkv, L, d], hq (rotated queries) [B, q_len, Hq, d] in,
+        ho [B, q_len, Hq, d] out; pinned host tensors."""
+        comp = torch.cuda.current_stream()
+        s_in, s_out = self.s_in, self.s_out
+        s_in.wait_stream(comp)   # the device buffers are free
+        s_out.wait_stream(comp)
+        B = self.cfg.batch
+        ev_k = [torch.cuda.Event() for _ in range(B)]
+        ev_v = [torch.cuda.Event() for _ in range(B)]
+        ev_q = [torch.cuda.Event() for _ in self.slices]
+        ev_c = [torch.cuda.Event() for _ in self.slices]
+        with torch.cuda.stream(s_in):
+            for i, (b, r0, r1, _, _) in enumerate(self.slices):
+                if r0 == 0:
+                    self.k_raw[b].copy_(hk[b], non_blocking=True)
+                    ev_k[b].record(s_in)
+                self.q_rot[b, r0:r1].copy_(hq[b, r0:r1], non_blocking=True)
+                ev_q[i].record(s_in)
+                if r0 == 0:
+                    self.v[b].copy_(hv[b], non_blocking=True)
+                    ev_v[b].record(s_in)
+        for i, (b, r0, r1, c, rb) in enumerate(self.slices):
+            k_b, v_b, kr_b = self.k_raw[b:b + 1], self.v[b:b + 1], self.k_rot[b:b + 1]
+            cs_b, gs_b = self.cs[b:b + 1], self.gs[b:b + 1]
+            if r0 == 0:
+                comp.wait_event(ev_k[b])
+                hga.build_summaries(self.cfg1, k_b, cs_b, gs_b, kr_b, 0, self.cfg1.n_chunks)
+            comp.wait_event(ev_q[i])
+            q_s, o_s = self.q_rot[b:b + 1, r0:r1], self.out[b:b + 1, r0:r1]
+            route(c, q_s, cs_b, gs_b, rb)
+            if r0 == 0:
+                comp.wait_event(ev_v[b])
+            hga.attend(c, q_s, kr_b, v_b, rb.sel_groups, rb.n_sel_groups, o_s)
+            ev_c[i].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_c[i])
+                ho[b, r0:r1].copy_(self.out[b, r0:r1], non_blocking=True)
+        comp.wait_stream(s_out)
