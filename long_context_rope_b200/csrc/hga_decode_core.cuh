@@ -337,7 +337,10 @@ __device__ __forceinline__ void store_warp_partial(const WarpAcc& acc, Partial& 
 // consumes blocks.
 constexpr int kOwnSlots = 16;
 __host__ __device__ constexpr int owned_per_cta(int CL) { return (8 + CL - 1) / CL; }
-static_assert(kMaxCluster * owned_per_cta(kMaxCluster) <= kOwnSlots, "owned slots");
+__host__ __device__ constexpr bool owned_slots_fit(int cl = 1) {
+    return cl > kMaxCluster || (cl * owned_per_cta(cl) <= kOwnSlots && owned_slots_fit(cl + 1));
+}
+static_assert(owned_slots_fit(), "owned slots for every cluster size");
 
 struct Owned {
     float m[kOwnSlots], l[kOwnSlots];  // per slot: max, sum

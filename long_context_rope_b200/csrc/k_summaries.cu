@@ -287,7 +287,7 @@ __device__ __forceinline__ float2 rot_mul(float2 x, float2 y) {
 // (cos, sin) of a small angle a (|a| < 2^20): reduced to [-pi, pi] in double,
 // split into a float head and the float remainder, the library sincosf of
 // the head corrected to first order by the remainder (the remainder's square,
-// below 2^-46, is dropped), so the cast to float costs no accuracy.
+// below 2^-44, is dropped), so the cast to float costs no accuracy.
 __device__ __forceinline__ float2 cs_accurate(double a) {
     const double red = fma(-rint(a * 0.15915494309189535), 6.283185307179586, a);
     const float hi = (float)red, lo = (float)(red - (double)hi);
