@@ -179,16 +179,21 @@ def test_prefill_parity_chunked_span():
     compare_prefill(w, x)
 
 
-def test_host_prefill_overlapped_equals_one_call():
+@pytest.mark.parametrize("span", [None, (256, 1244)])
+def test_host_prefill_overlapped_equals_one_call(span):
     """pipeline.HostPrefill (inputs and output in pinned host memory, the copies
     overlapped with slice-by-slice routing and attention on other streams):
     two sequences, ragged length (24 query chunks each, the last one partial),
-    two slices of 12 query chunks per sequence. Its output must equal the one-call prefill on device buffers
-    bitwise, and that one the oracle (compare_prefill on the same inputs)."""
+    two slices of 12 query chunks per sequence; or a chunked-prefill span from
+    token 256 (20 query chunks: slices of 10). Its output must equal the
+    one-call prefill on device buffers bitwise, and that one the oracle
+    (compare_prefill on the same inputs)."""
     hga, pipeline = _mods()
     w = synth.WORKLOADS["prefill_4k"].replace(
         name="host_prefill", batch=2, seq_len=1500, n_q_heads=8, n_kv_heads=2, top_k_chunks=5,
         top_k_groups=13, n_local=1, n_sink=1)
+    if span is not None:
+        w = w.replace(span_begin=span[0], span_len=span[1])
     x = synth.draw(w, seed=6)
     cfg = hga.config_from(w)
     k_raw, v = x["k_raw"].cuda(), x["v"].cuda()
@@ -199,7 +204,8 @@ def test_host_prefill_overlapped_equals_one_call():
     out = torch.full_like(q_rot, float("nan"))
     pipeline.prefill(cfg, k_raw, v, q_rot, cs, gs, k_rot, rb, out)
     hp = pipeline.HostPrefill(cfg, chunks_per_slice=10)
-    assert [(r0, r1) for (_, r0, r1, _, _) in hp.slices] == [(0, 768), (768, 1500)] * 2
+    want = [(0, 768), (768, 1500)] if span is None else [(0, 640), (640, 1244)]
+    assert [(r0, r1) for (_, r0, r1, _, _) in hp.slices] == want * 2
     hk, hv, hq = (t.cpu().pin_memory() for t in (k_raw, v, q_rot))
     ho = torch.full(out.shape, float("nan"), dtype=out.dtype).pin_memory()
     for _ in range(2):  # the second run reuses every buffer
