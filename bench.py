@@ -176,16 +176,14 @@ def run_prefill(args, dist, peaks):
         pipeline.summaries(cfg, k_raw, cs, gs, k_rot)
         if ev:
             ev.rec(base + 1, st)
-        hga.route_chunks(cfg, q_rot, cs, rb.qbar, rb.sel_chunks, rb.n_sel_chunks)
+        # q-bar, then both routing levels in one launch (hga_route, prefill form)
+        hga.route(cfg, q_rot, cs, gs, rb.qbar, rb.sel_chunks, rb.n_sel_chunks, rb.sel_groups,
+                  rb.n_sel_groups)
         if ev:
             ev.rec(base + 2, st)
-        hga.route_groups(cfg, rb.qbar, gs, rb.sel_chunks, rb.n_sel_chunks, rb.sel_groups,
-                         rb.n_sel_groups)
-        if ev:
-            ev.rec(base + 3, st)
         hga.attend(cfg, q_rot, k_rot, v, rb.sel_groups, rb.n_sel_groups, out)
         if ev:
-            ev.rec(base + 4, st)
+            ev.rec(base + 3, st)
 
     for _ in range(args.warmup):
         step()
@@ -197,27 +195,27 @@ def run_prefill(args, dist, peaks):
                             rb.n_sel_chunks.cpu().numpy())
 
     K = args.steps
-    ev = Events(5 * K)
+    ev = Events(4 * K)
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev) as clk:
         start.record(st)
         for i in range(K):
-            step(ev, 5 * i)
+            step(ev, 4 * i)
         stop.record(st)
         torch.cuda.synchronize()
     dist.barrier()
     total_ms = start.elapsed_time(stop)
-    stage = {n: [] for n in ("summaries", "route_chunks", "route_groups", "attend")}
+    stage = {n: [] for n in ("summaries", "route", "attend")}
     for i in range(K):
         for s_i, n in enumerate(stage):
-            stage[n].append(ev.ms(5 * i + s_i, 5 * i + s_i + 1))
+            stage[n].append(ev.ms(4 * i + s_i, 4 * i + s_i + 1))
     attend_ms = float(np.mean(stage["attend"]))
     res = dict(total_ms=dist.max(total_ms), attend_ms=dist.max(attend_ms),
                stage_ms={n: float(np.mean(vs)) for n, vs in stage.items()},
                flops=flops, tokens=w.batch * w.q_len, clocks=clk.summary(), recall=recall,
-               launches_per_step=5)
+               launches_per_step=4)
 
     # end to end through the public API with host buffers (pinned), H2D + D2H inside
     if not args.no_e2e:

@@ -341,6 +341,11 @@ static hga_status route_separate(const Params& p, const void* q_rot, const void*
     if (p.sum_bf16 || p.Hu != p.Hkv) return HGA_ERR_UNSUPPORTED;  // one-launch path only
     cudaError_t e = route_chunks_fuses_qbar(p) ? cudaSuccess : launch_qbar(p, q_rot, qbar_out, st);
     if (e != cudaSuccess) return cuda_failed(e);
+    if (route_tiled_fuses_groups(p))  // prefill: both levels in one launch after q-bar
+        return launched(launch_route_chunks_tiled(p, qbar_out, (const float*)chunk_sum, sel_chunks,
+                                                  n_sel_chunks, nullptr, st,
+                                                  (const float*)group_sum, sel_groups,
+                                                  n_sel_groups));
     e = launch_route_chunks(p, q_rot, qbar_out, (const float*)chunk_sum, sel_chunks, n_sel_chunks,
                             nullptr, st);
     if (e != cudaSuccess) return cuda_failed(e);

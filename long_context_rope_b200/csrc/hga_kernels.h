@@ -43,11 +43,15 @@ cudaError_t launch_route_chunks(const Params& p, const void* q_rot, float* qbar,
                                 float* scores, cudaStream_t st);
 
 // Prefill form of level-1 routing: 8 query chunks per CTA share one pass
-// over the chunk-summary table (needs nQC >= 8 and nC <= 2048).
+// over the chunk-summary table (needs nQC >= 8 and nC <= 2048). With a group
+// table (group_sum != nullptr; route_tiled_fuses_groups(p)) the same launch
+// also runs level 2 and writes sel_g / n_sel_g, bitwise as launch_route_groups.
 bool route_chunks_tiled_supports(const Params& p);
+bool route_tiled_fuses_groups(const Params& p);
 cudaError_t launch_route_chunks_tiled(const Params& p, const float* qbar, const float* chunk_sum,
                                       int32_t* sel, int32_t* n_sel, float* scores,
-                                      cudaStream_t st);
+                                      cudaStream_t st, const float* group_sum = nullptr,
+                                      int32_t* sel_g = nullptr, int32_t* n_sel_g = nullptr);
 
 cudaError_t launch_route_groups(const Params& p, const float* qbar, const float* group_sum,
                                 const int32_t* sel_chunks, const int32_t* n_sel_chunks,

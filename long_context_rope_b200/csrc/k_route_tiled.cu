@@ -16,6 +16,16 @@
 // go to the lower chunk index; NaN ranks last. Work grows with the query
 // chunk index (more earlier chunks to score), so CTAs take the last query
 // chunks first and the block scheduler fills in with the short ones.
+//
+// Level 2 in the same warp (hga_route, when a group table is given; Niveau
+// 2 of the same item): the warp that selected a query chunk's chunks then
+// scores all G group rows of each of them (read from L2 eight rows at a
+// time) and selects the top-k groups with the same radix select. Lane L
+// holds dims L*DPL.. of every row and each score is the same per-lane
+// partial dot product and butterfly sum as in route_groups_small_kernel and
+// the decode step, so the fused and the separate routing select the same
+// groups, bitwise. This replaces a second launch of one short CTA per query
+// chunk and its round trip of the chunk lists through global memory.
 #include "hga_kernels.h"
 #include "hga_topk.cuh"
 
@@ -32,10 +42,18 @@ static_assert(kKS == 32 && kCT % 32 == 0, "a slice row is 8 float4, rows come in
 static_assert(kThreads / 32 == kQB, "one warp per query chunk");
 static_assert(kThreads / 32 * 256 <= kKS * kCT, "histograms fit in the tile buffer");
 
+// Shared words of the tile buffer reused once the products are done: the
+// radix histograms [8 warps][256], then (level 2) group keys [8][256] and
+// the selected chunks [8][64].
+constexpr int kGroupKeysAt = kQB * 256;
+constexpr int kSelChunksAt = kGroupKeysAt + kQB * 256;
+static_assert(kSelChunksAt + kQB * 64 <= kKS * kCT, "level-2 scratch fits in the tile buffer");
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 3) route_chunks_tiled_kernel(
     Params p, const float* __restrict__ qbar, const float* __restrict__ cs,
-    int32_t* __restrict__ sel, int32_t* __restrict__ nsel, float* __restrict__ scores_out) {
+    int32_t* __restrict__ sel, int32_t* __restrict__ nsel, float* __restrict__ scores_out,
+    const float* __restrict__ gs, int32_t* __restrict__ sel_g, int32_t* __restrict__ nsel_g) {
     extern __shared__ __align__(16) float smem_f[];
     float* qT = smem_f;                         // [D][kQB]   transposed q-bar
     float* tile = qT + D * kQB;                 // [kKS][kCT] transposed table slice
@@ -139,6 +157,50 @@ __global__ void __launch_bounds__(kThreads, 3) route_chunks_tiled_kernel(
         const int kept = warp_radix_topk(krow, j, p.kc, p.kc, sel + prob * p.kc, h,
                                          [](int x) { return x; });
         if (lane == 0) nsel[prob] = kept;
+        if (gs == nullptr) continue;
+
+        // ---- level 2: all G groups of the kept chunks, then their top k_g
+        constexpr int DPL = D / 32;
+        const int G = p.G;
+        uint32_t* gkeys = reinterpret_cast<uint32_t*>(tile) + kGroupKeysAt + warp * 256;
+        int32_t* s_chunk = reinterpret_cast<int32_t*>(tile) + kSelChunksAt + warp * 64;
+        __syncwarp();  // this warp's lanes wrote the kept chunks
+        for (int s = lane; s < kept; s += 32) s_chunk[s] = sel[prob * p.kc + s];
+        float qv[DPL];
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) qv[e] = qT[(lane * DPL + e) * kQB + q];
+        __syncwarp();
+        const float* gtab = gs + bh * (int64_t)p.nC * G * D;
+        const int n_rows = kept * G;  // row x: group x % G of the (x / G)-th kept chunk
+        for (int x0 = 0; x0 < n_rows; x0 += 8) {
+            float v[8][DPL];  // eight group rows in flight
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int x = x0 + i < n_rows ? x0 + i : x0;
+                const float* row = gtab + ((int64_t)s_chunk[x / G] * G + x % G) * D + lane * DPL;
+                if constexpr (DPL == 4) {
+                    const float4 t = __ldg(reinterpret_cast<const float4*>(row));
+                    v[i][0] = t.x; v[i][1] = t.y; v[i][2] = t.z; v[i][3] = t.w;
+                } else {
+                    const float2 t = __ldg(reinterpret_cast<const float2*>(row));
+                    v[i][0] = t.x; v[i][1] = t.y;
+                }
+            }
+            float sc2 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float a = 0.f;
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) a = fmaf(qv[e], v[i][e], a);
+                a = warp_sum(a);
+                if (lane == i) sc2 = a;
+            }
+            if (lane < 8 && x0 + lane < n_rows) gkeys[x0 + lane] = score_key32(sc2);
+        }
+        __syncwarp();
+        const int kept2 = warp_radix_topk(gkeys, kept * G, p.kg, p.kg, sel_g + prob * p.kg, h,
+                                          [&](int x) { return s_chunk[x / G] * G + x % G; });
+        if (lane == 0) nsel_g[prob] = kept2;
     }
 }
 
@@ -148,9 +210,14 @@ bool route_chunks_tiled_supports(const Params& p) {
     return p.nQC >= 8 && p.nC <= 2048 && (p.d == 128 || p.d == 64);
 }
 
+bool route_tiled_fuses_groups(const Params& p) {
+    return route_chunks_tiled_supports(p) && p.G <= 8 && p.kc <= 64 && p.kc * p.G <= 256;
+}
+
 cudaError_t launch_route_chunks_tiled(const Params& p, const float* qbar, const float* chunk_sum,
                                       int32_t* sel, int32_t* n_sel, float* scores,
-                                      cudaStream_t st) {
+                                      cudaStream_t st, const float* group_sum, int32_t* sel_g,
+                                      int32_t* n_sel_g) {
     const int ncp = (p.nC + 3) & ~3;
     const size_t smem = (size_t)(p.d * kQB + kKS * kCT + kQB * ncp) * sizeof(float);
     dim3 grid((p.nQC + kQB - 1) / kQB, p.B * p.Hkv);
@@ -166,7 +233,8 @@ cudaError_t launch_route_chunks_tiled(const Params& p, const float* qbar, const 
         if (e != cudaSuccess) return e;
     }
     Params pp = p;
-    void* args[] = {&pp, (void*)&qbar, (void*)&chunk_sum, &sel, &n_sel, &scores};
+    void* args[] = {&pp,    (void*)&qbar,       (void*)&chunk_sum, &sel,   &n_sel,
+                    &scores, (void*)&group_sum, &sel_g,            &n_sel_g};
     return cudaLaunchKernel(fn, grid, dim3(kThreads), args, smem, st);
 }
 

@@ -157,21 +157,28 @@ def test_decode_step_repeat_and_prefill_route():
     assert torch.equal(res[0][1], res[1][1])
     assert torch.equal(res[0][0].sel_groups, res[1][0].sel_groups)
 
-    wp = synth.WORKLOADS["prefill_4k"]
-    xp = synth.draw(wp, seed=1)
-    cfgp = hga.config_from(wp)
-    k_raw = xp["k_raw"].cuda()
-    csp, gsp = pipeline.alloc_summaries(cfgp)
-    pipeline.summaries(cfgp, k_raw, csp, gsp, None)
-    qp = pipeline.rotate_queries(cfgp, xp["q_raw"].cuda())
-    rb1 = pipeline.alloc_route(cfgp)
-    pipeline.route(cfgp, qp, csp, gsp, rb1, separate=True)
-    rb2 = pipeline.alloc_route(cfgp)
-    pipeline.route(cfgp, qp, csp, gsp, rb2)
-    torch.cuda.synchronize()
-    assert hga.get_device_error() == 0
-    for name in ("qbar", "sel_chunks", "n_sel_chunks", "sel_groups", "n_sel_groups"):
-        assert torch.equal(getattr(rb1, name), getattr(rb2, name)), name
+    # prefill: hga_route runs both levels in one launch after q-bar (the tiled
+    # chunk router with level 2 fused); the separate calls must agree bitwise
+    base = synth.WORKLOADS["prefill_4k"]
+    for wp in (base,
+               base.replace(batch=2, seq_len=1500, n_q_heads=8, n_kv_heads=2, top_k_chunks=5,
+                            top_k_groups=13, n_local=1, n_sink=1),
+               base.replace(seq_len=4000, chunk_size=128, groups_per_chunk=8, top_k_chunks=16,
+                            top_k_groups=60)):
+        xp = synth.draw(wp, seed=1)
+        cfgp = hga.config_from(wp)
+        k_raw = xp["k_raw"].cuda()
+        csp, gsp = pipeline.alloc_summaries(cfgp)
+        pipeline.summaries(cfgp, k_raw, csp, gsp, None)
+        qp = pipeline.rotate_queries(cfgp, xp["q_raw"].cuda())
+        rb1 = pipeline.alloc_route(cfgp)
+        pipeline.route(cfgp, qp, csp, gsp, rb1, separate=True)
+        rb2 = pipeline.alloc_route(cfgp)
+        pipeline.route(cfgp, qp, csp, gsp, rb2)
+        torch.cuda.synchronize()
+        assert hga.get_device_error() == 0
+        for name in ("qbar", "sel_chunks", "n_sel_chunks", "sel_groups", "n_sel_groups"):
+            assert torch.equal(getattr(rb1, name), getattr(rb2, name)), (wp.seq_len, name)
 
 
 def test_decode_loop_appends_and_finalises_chunks():
