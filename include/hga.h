@@ -223,7 +223,11 @@ hga_status hga_route_groups(const hga_config* cfg, const float* qbar, const void
  * followed by hga_route_groups on these arguments, without the score
  * outputs. For a one-token query span (decode) in bf16 with d = 128 and
  * top_k_chunks <= 64 this is one launch (both levels split across a
- * thread-block cluster); otherwise the two calls' kernels run in sequence.
+ * thread-block cluster). For a prefill span of at least 8 query chunks with
+ * nC <= 2048, groups_per_chunk <= 8, top_k_chunks <= 64 and
+ * top_k_chunks * groups_per_chunk <= 256 it is two launches: q-bar, then both
+ * levels in one kernel (each level-1 warp goes on to the groups of its query
+ * chunk). Otherwise the two calls' kernels run in sequence.
  * qbar_out [B,Hkv,nQC,d] fp32, sel_chunks / n_sel_chunks, sel_groups /
  * n_sel_groups as for the two calls; all required. */
 hga_status hga_route(const hga_config* cfg, const void* q_rot, const void* chunk_sum,
