@@ -3,10 +3,12 @@
 Allocates the device buffers of a configuration (torch supplies the memory)
 and calls the library's entry points in order:
 
-  prefill: hga_build_summaries -> hga_route_chunks -> hga_route_groups
-           -> hga_attend (index mode: the kernel fetches routed groups itself)
-  decode:  hga_route_chunks -> hga_route_groups -> [hga_gather_kv] -> hga_attend
-           (summaries are built once beforehand, as for a KV cache)
+  prefill: hga_build_summaries -> hga_route (q-bar, then both levels in one
+           launch) -> hga_attend (index mode: the kernel fetches routed groups
+           itself); HostPrefill does the same slice by slice from host buffers
+  decode:  hga_decode_step (one launch), or hga_route -> [hga_gather_kv]
+           -> hga_attend (summaries are built once beforehand, as for a KV
+           cache; decode_append keeps them current in a decode loop)
 
 Nothing here computes: every step is a kernel of libhga.so.
 """
@@ -99,7 +101,8 @@ def route(cfg: hga.HgaConfig, q_rot, cs, gs, rb: RouteBuffers, stream=None,
           separate: bool = False):
     """Both routing levels. With score buffers (or separate=True) the two
     levels run as their own calls, which also write the scores; otherwise
-    one hga_route call (a single launch for decode)."""
+    one hga_route call (decode: one launch; prefill: q-bar, then one launch
+    for both levels)."""
     if separate or rb.chunk_scores is not None or rb.group_scores is not None:
         hga.route_chunks(cfg, q_rot, cs, rb.qbar, rb.sel_chunks, rb.n_sel_chunks,
                          rb.chunk_scores, stream)
@@ -203,6 +206,16 @@ def decode_append(cfg_cap: hga.HgaConfig, pos: int, k_new_raw, v_new, q_rot_new,
                     rb.n_sel_chunks, rb.sel_groups, rb.n_sel_groups, out, stream)
 
 
+def slice_bounds(n_qchunks: int, chunk_size: int, q_len: int, chunks_per_slice: int):
+    """Row boundaries [0, ..., q_len] of HostPrefill's slices of a query span
+    that starts on a chunk boundary: on chunk boundaries, about
+    chunks_per_slice query chunks each and never fewer (all of them if there
+    are fewer), so every slice is routed by the same kernel as the whole span
+    would be."""
+    n_sl = max(1, n_qchunks // max(1, chunks_per_slice))
+    return [min(q_len, (i * n_qchunks // n_sl) * chunk_size) for i in range(n_sl)] + [q_len]
+
+
 class HostPrefill:
     """Prefill whose inputs and output live in (pinned) host memory, with the
     host-link copies overlapped with the computation.
@@ -238,12 +251,7 @@ class HostPrefill:
         self.out = torch.empty_like(self.q_rot)
         self.cs, self.gs = alloc_summaries(cfg, device)
         self.cfg1 = cfg.copy(batch=1)
-        # slice boundaries on chunk boundaries, about chunks_per_slice query
-        # chunks each and never fewer (so every slice is routed by the same
-        # kernel as the whole span would be)
-        nqc, C = cfg.n_qchunks, cfg.chunk_size
-        n_sl = max(1, nqc // max(1, chunks_per_slice))
-        bounds = [min(L, (i * nqc // n_sl) * C) for i in range(n_sl)] + [L]
+        bounds = slice_bounds(cfg.n_qchunks, cfg.chunk_size, L, chunks_per_slice)
         self.slices = []  # (b, row0, row1, cfg of the span, RouteBuffers)
         for b in range(B):
             for r0, r1 in zip(bounds[:-1], bounds[1:]):
